@@ -1,0 +1,300 @@
+"""Plain fp64 CPU oracle of the DeepSeek-V4 hybrid (CSA / HCA) attention path.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference arm of ``bench.py`` may import or run this module.
+The CUDA library never calls it and shares no code with it; the two meet
+only in the seeded generator (``gen/``), which holds no attention arithmetic.
+
+Everything is float64, computed in the order the pages describe it, with no
+tiling, no online softmax and no fusion.  numpy matmul and sort serve as
+library steps.  Sources (page title, then section / equation):
+
+[V4-inside]  "DeepSeek V4 Inside: One Token Through Every Block"
+             (sections on layer-0 SWA, CSA, HCA, "What is stored").
+[beyond]     "DeepSeek-v4 Beyond Basics", sections 3.2.2 (CSA, eqs. 9-17)
+             and 3.3 (HCA, eqs. 20-27).
+[module1]    "Phase 1 Module 1 - The model & the cost of attention",
+             section "The indexer: a learned retrieval mechanism".
+[hf-doc]     "DeepSeek-V4" (Transformers documentation), sections on hybrid
+             attention and the attention-mask layout.
+
+Readings taken where the pages are silent or garbled (each one is also
+listed with its reason in the design notes):
+ R1  compressor overlap: stream a covers the entry's own m tokens, stream b
+     the previous block's m tokens; per channel one softmax over the 2m
+     logits (m for entry 0 and for HCA).           -- parity unpinned
+ R2  visibility is applied before top-k: entry s is visible to a query at
+     position t iff s < floor((t + 1) / m).
+ R3  top-k ties: higher score first, then lower index; the output lists the
+     chosen indices ascending and pads with -1.
+ R4  the index score has no scale, norm or RoPE: sum_h w_h ReLU(q_h . k).
+ R5  softmax scale 1 / sqrt(head_dim).
+ R6  RoPE on interleaved pairs (2j, 2j+1) of the last R dims, angle
+     pos * base^(-2j/R), base 10000, no YaRN.        -- base parity unpinned
+ R7  compressed entry i carries position i * m.      -- parity unpinned
+ R8  RMSNorm eps 1e-6 with a learned gain after normalising; window K=V
+     rows arrive in final form.
+ R9  window = positions max(0, t - W + 1) .. t inclusive; no dedup with
+     compressed entries.
+ R10 positions are 0-based.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+# --------------------------------------------------------------------------
+# storage helpers
+# --------------------------------------------------------------------------
+def widen(x) -> np.ndarray:
+    """bfloat16 bit patterns (uint16) or float32 -> float64."""
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    return x.astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# RMSNorm and partial interleaved RoPE
+# [beyond] 3.3: RMSNorm on every query head and on the single compressed KV
+# head; RoPE on the last 64 dims of each.  [V4-inside] layer-0 SWA: RoPE
+# rotates the pair (x, y) at position i into (x cos - y sin, x sin + y cos).
+# --------------------------------------------------------------------------
+def rms_norm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * g over the last axis (R8)."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * np.asarray(g, dtype=np.float64)
+
+
+def rope_frequencies(rope_dim: int, base: float) -> np.ndarray:
+    """theta_j = base^(-2j/R), j = 0 .. R/2-1 (R6)."""
+    j = np.arange(rope_dim // 2, dtype=np.float64)
+    return base ** (-2.0 * j / rope_dim)
+
+
+def rope(x: np.ndarray, pos, rope_dim: int, base: float) -> np.ndarray:
+    """Rotate the interleaved pairs of the last ``rope_dim`` dims of x by
+    angle pos * theta_j.  ``pos`` may be negative (the output de-rotation of
+    [hf-doc] / paper eq. 26 uses position -i).  x: [..., D]; pos broadcasts
+    against x[..., 0]."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    if rope_dim == 0:
+        return x
+    D = x.shape[-1]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_frequencies(rope_dim, base)
+    c, s = np.cos(ang), np.sin(ang)
+    xe = x[..., D - rope_dim::2].copy()  # first of each pair
+    xo = x[..., D - rope_dim + 1::2].copy()  # second of each pair
+    x[..., D - rope_dim::2] = xe * c - xo * s
+    x[..., D - rope_dim + 1::2] = xe * s + xo * c
+    return x
+
+
+# --------------------------------------------------------------------------
+# (1) KV compressor
+# [beyond] 3.2.2, eqs. 9-12: two token-level streams C^a, C^b with logits
+# Z^a, Z^b; position biases B^a, B^b; softmax per channel along the rows
+# that gather elements of both Z^a and Z^b; Hadamard-weighted sum; every m
+# tokens give one entry.  [V4-inside] CSA: the blocks overlap, 2m weights
+# normalised per block.  [beyond] 3.3, eqs. 20-23: HCA is the same with
+# m' = 128 and a single stream, no overlap.
+# --------------------------------------------------------------------------
+def compress_entry(i: int, m: int, tok_begin: int, ca, za, ba, cb=None, zb=None, bb=None) -> np.ndarray:
+    """Entry i (unnormalised) from float64 streams [T_tok, c] whose row 0 is
+    absolute token ``tok_begin``.  a-half: tokens i*m + r (r < m) with logits
+    Z^a + B^a[r]; b-half (CSA, i >= 1): tokens (i-1)*m + r with Z^b + B^b[r]
+    (reading R1).  One softmax per channel over all the logits present."""
+    logits, values = [], []
+    for r in range(m):
+        t = i * m + r - tok_begin
+        logits.append(za[t] + ba[r])
+        values.append(ca[t])
+    if cb is not None and i >= 1:
+        for r in range(m):
+            t = (i - 1) * m + r - tok_begin
+            logits.append(zb[t] + bb[r])
+            values.append(cb[t])
+    L = np.stack(logits)  # [n_terms, c]
+    V = np.stack(values)
+    L = L - L.max(axis=0, keepdims=True)
+    e = np.exp(L)
+    wgt = e / e.sum(axis=0, keepdims=True)
+    return (wgt * V).sum(axis=0)
+
+
+def compress(m: int, entry_begin: int, entry_end: int, tok_begin: int,
+             ca, za, ba, cb=None, zb=None, bb=None,
+             norm_g=None, rope_dim: int = 0, rope_base: float = 10000.0,
+             eps: float = 1e-6) -> np.ndarray:
+    """Entries entry_begin .. entry_end-1 of one sequence -> float64 [n, c].
+    With ``norm_g``: RMSNorm(.) * g, then RoPE of the last ``rope_dim`` dims
+    at the entry position i*m (readings R7, R8).  Without it (the indexer-key
+    compressor of [beyond] 3.2.2 / [module1] "its own compressed stream"):
+    the weighted sum only (reading R4)."""
+    ca, za = widen(ca), widen(za)
+    ba = widen(ba)
+    if cb is not None:
+        cb, zb, bb = widen(cb), widen(zb), widen(bb)
+    out = []
+    for i in range(entry_begin, entry_end):
+        e = compress_entry(i, m, tok_begin, ca, za, ba, cb, zb, bb)
+        if norm_g is not None:
+            e = rms_norm(e, widen(norm_g), eps)
+            e = rope(e, i * m, rope_dim, rope_base)
+        out.append(e)
+    if not out:
+        return np.zeros((0, ca.shape[-1]))
+    return np.stack(out)
+
+
+# --------------------------------------------------------------------------
+# (2) Lightning indexer and top-k selector
+# [beyond] 3.2.2, eqs. 13-17; [module1] "It scores every compressed row",
+# "Top-k selects", "only kicks in once there are more than 512 rows";
+# [hf-doc] attention-mask layout: -1 sentinels, visibility w < (t+1)//m.
+# --------------------------------------------------------------------------
+def visible_entries(pos: int, m: int) -> int:
+    """Number of compressed entries whose source tokens all lie at or before
+    position ``pos``: floor((pos + 1) / m) (reading R2)."""
+    return (int(pos) + 1) // int(m)
+
+
+def index_scores(qi, wi, ki, n_vis: int) -> np.ndarray:
+    """I_s = sum_h w_h * ReLU(q_h . K_s) for s < n_vis.
+    qi [H_I, D_I], wi [H_I], ki [>= n_vis, D_I] -> float64 [n_vis]."""
+    qi, wi, ki = widen(qi), widen(wi), widen(ki)
+    dots = ki[:n_vis] @ qi.T  # [n_vis, H_I]
+    return np.maximum(dots, 0.0) @ wi
+
+
+def topk_select(scores: np.ndarray, k: int) -> np.ndarray:
+    """Keep the k highest scores (reading R3: ties to the lower index);
+    return their indices ascending, padded with -1 to length k.  When there
+    are no more than k scores every index is kept."""
+    n = scores.shape[0]
+    order = np.lexsort((np.arange(n), -scores))  # primary: score desc
+    chosen = np.sort(order[:k])
+    out = np.full(k, -1, dtype=np.int64)
+    out[: chosen.size] = chosen
+    return out
+
+
+def index_topk(qi, wi, ki, pos: int, m: int, k: int, n_c: int):
+    """One query: (indices [k], scores of the visible entries)."""
+    n_vis = min(visible_entries(pos, m), n_c)
+    s = index_scores(qi, wi, ki, n_vis)
+    return topk_select(s, k), s
+
+
+# --------------------------------------------------------------------------
+# (3)+(4) shared K=V MQA with sink, merged with the sliding window
+# [beyond] 3.2.2 (the selected entries serve as both key and value, eq. 19)
+# and 3.3 (eqs. 24-27); [V4-inside] layer-0 SWA sink example and the CSA
+# "1 compressed + 2 window keys" example (one normaliser, sink in the
+# denominator only); [hf-doc] output de-rotation by -i on the rope slice.
+# --------------------------------------------------------------------------
+def window_positions(pos: int, window: int) -> np.ndarray:
+    """Positions max(0, pos - W + 1) .. pos (reading R9)."""
+    return np.arange(max(0, int(pos) - window + 1), int(pos) + 1, dtype=np.int64)
+
+
+def sink_softmax(z: np.ndarray, sink) -> tuple[np.ndarray, np.ndarray]:
+    """p_j = exp(z_j) / (sum_k exp(z_k) + exp(sink)), per row of z [H, n];
+    returns (p, sink mass exp(sink) / denominator).  A max shift keeps the
+    exponentials finite; it cancels in the ratio."""
+    z = np.asarray(z, dtype=np.float64)
+    sink = np.asarray(sink, dtype=np.float64).reshape(-1, 1)
+    mx = np.maximum(z.max(axis=1, keepdims=True) if z.shape[1] else -np.inf, sink)
+    e = np.exp(z - mx)
+    es = np.exp(sink - mx)
+    den = e.sum(axis=1, keepdims=True) + es
+    return e / den, (es / den)[:, 0]
+
+
+def attend_rows(q, q_norm_g, rows, sink, pos: int, head_dim_scale: float,
+                rope_dim: int, rope_base: float, eps: float) -> np.ndarray:
+    """Core MQA for one query over explicit K=V rows [n, D]:
+    q_hat = RoPE_pos(RMSNorm(q_h) * g); z = q_hat . kv * scale;
+    p = sink_softmax(z); o = sum p kv; o = RoPE_{-pos}(o).  -> [H, D]."""
+    q = widen(q)
+    rows = widen(rows)
+    qh = rope(rms_norm(q, widen(q_norm_g), eps), pos, rope_dim, rope_base)
+    z = (qh @ rows.T) * head_dim_scale
+    p, _ = sink_softmax(z, widen(sink))
+    o = p @ rows
+    return rope(o, -pos, rope_dim, rope_base)
+
+
+def window_rows(win, win_cap: int, pos: int, window: int) -> np.ndarray:
+    """K=V rows of the window read from a ring: slot = position mod win_cap."""
+    return widen(win)[window_positions(pos, window) % win_cap]
+
+
+def csa_attend(q, q_norm_g, pool, idx, win, win_cap: int, sink, pos: int, cfg) -> np.ndarray:
+    """CSA: keys = pool[idx >= 0] followed by the window (one softmax)."""
+    sel = np.asarray(idx)
+    sel = sel[sel >= 0]
+    rows = np.concatenate([widen(pool)[sel], window_rows(win, win_cap, pos, cfg.window)], axis=0)
+    return attend_rows(q, q_norm_g, rows, sink, pos, cfg.sm_scale, cfg.rope_dim, cfg.rope_base, cfg.rms_eps)
+
+
+def hca_attend(q, q_norm_g, pool, n_c: int, win, win_cap: int, sink, pos: int, cfg) -> np.ndarray:
+    """HCA: keys = every visible pool entry followed by the window."""
+    n_vis = min(visible_entries(pos, cfg.ratio), n_c)
+    rows = np.concatenate([widen(pool)[:n_vis], window_rows(win, win_cap, pos, cfg.window)], axis=0)
+    return attend_rows(q, q_norm_g, rows, sink, pos, cfg.sm_scale, cfg.rope_dim, cfg.rope_base, cfg.rms_eps)
+
+
+def attended_key_count(pos: int, cfg, n_c: int, sparse: bool) -> int:
+    """Keys one query scores: min(k, visible) + window (CSA) or visible +
+    window (HCA); [V4-inside] "What does HCA change?" table."""
+    n_vis = min(visible_entries(pos, cfg.ratio), n_c)
+    n_win = window_positions(pos, cfg.window).size
+    return (min(cfg.topk, n_vis) if sparse else n_vis) + n_win
+
+
+# --------------------------------------------------------------------------
+# batch drivers (loops over sequences and queries)
+# --------------------------------------------------------------------------
+def index_topk_batch(qi, wi, ki, q_pos, m: int, k: int, n_c: int, rows=None):
+    """qi [B,T,H_I,D_I], wi [B,T,H_I], ki [B,N_c,D_I], q_pos [B,T] ->
+    idx int64 [B,T,k] and a dict (b,t) -> scores.  ``rows`` limits the work
+    to a list of (b, t)."""
+    B, T = np.asarray(q_pos).shape
+    idx = np.full((B, T, k), -1, dtype=np.int64)
+    scores = {}
+    todo = rows if rows is not None else [(b, t) for b in range(B) for t in range(T)]
+    for b, t in todo:
+        idx[b, t], scores[(b, t)] = index_topk(qi[b, t], wi[b, t], ki[b], int(q_pos[b][t]), m, k, n_c)
+    return idx, scores
+
+
+def csa_attend_batch(q, q_norm_g, pool, idx, win, win_cap, sink, q_pos, cfg, rows=None):
+    B, T = np.asarray(q_pos).shape
+    out = np.zeros(q.shape, dtype=np.float64)
+    todo = rows if rows is not None else [(b, t) for b in range(B) for t in range(T)]
+    for b, t in todo:
+        out[b, t] = csa_attend(q[b, t], q_norm_g, pool[b], idx[b, t], win[b], win_cap, sink, int(q_pos[b][t]), cfg)
+    return out
+
+
+def hca_attend_batch(q, q_norm_g, pool, n_c, win, win_cap, sink, q_pos, cfg, rows=None):
+    B, T = np.asarray(q_pos).shape
+    out = np.zeros(q.shape, dtype=np.float64)
+    todo = rows if rows is not None else [(b, t) for b in range(B) for t in range(T)]
+    for b, t in todo:
+        out[b, t] = hca_attend(q[b, t], q_norm_g, pool[b], n_c, win[b], win_cap, sink, int(q_pos[b][t]), cfg)
+    return out
+
+
+def compress_batch(m, entry_begin, entry_end, tok_begin, ca, za, ba, cb=None, zb=None, bb=None,
+                   norm_g=None, rope_dim=0, rope_base=10000.0, eps=1e-6) -> np.ndarray:
+    """Streams [B, T_tok, c] -> entries float64 [B, n, c]."""
+    B = np.asarray(ca).shape[0]
+    outs = []
+    for b in range(B):
+        outs.append(compress(m, entry_begin, entry_end, tok_begin, ca[b], za[b], ba,
+                             None if cb is None else cb[b], None if zb is None else zb[b], bb,
+                             norm_g, rope_dim, rope_base, eps))
+    return np.stack(outs)

@@ -1,0 +1,74 @@
+"""Planted mistakes: each mutant is a copy of the oracle source with one
+plausible error; at least one pin must reject every mutant."""
+import importlib.util
+import os
+import types
+
+import pytest
+
+from pins import PINS
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "ds4a_oracle.py")
+
+# name -> list of (old, new) source replacements (each old must occur once,
+# unless the name ends in "*": then every occurrence is replaced)
+MUTANTS = {
+    "sink dropped from denominator": [("den = e.sum(axis=1, keepdims=True) + es", "den = e.sum(axis=1, keepdims=True)")],
+    "no output de-rotation": [("return rope(o, -pos, rope_dim, rope_base)", "return o")],
+    "de-rotation with +pos": [("return rope(o, -pos, rope_dim, rope_base)", "return rope(o, pos, rope_dim, rope_base)")],
+    "rope angle sign": [("ang = np.asarray(pos, dtype=np.float64)[..., None]", "ang = -np.asarray(pos, dtype=np.float64)[..., None]")],
+    "rope half-split pairs*": [("D - rope_dim::2]", "D - rope_dim:D - rope_dim // 2]"),
+                               ("D - rope_dim + 1::2]", "D - rope_dim // 2:]")],
+    "rope non-rotation": [("x[..., D - rope_dim::2] = xe * c - xo * s", "x[..., D - rope_dim::2] = xe * c + xo * s")],
+    "visibility off by one": [("return (int(pos) + 1) // int(m)", "return int(pos) // int(m)")],
+    "window off by one": [("np.arange(max(0, int(pos) - window + 1), int(pos) + 1,", "np.arange(max(0, int(pos) - window), int(pos),")],
+    "missing ReLU": [("return np.maximum(dots, 0.0) @ wi", "return dots @ wi")],
+    "ReLU after head sum": [("return np.maximum(dots, 0.0) @ wi", "return np.maximum(dots @ wi, 0.0)")],
+    "top-k keeps lowest": [("order = np.lexsort((np.arange(n), -scores))", "order = np.lexsort((np.arange(n), scores))")],
+    "ties to higher index": [("order = np.lexsort((np.arange(n), -scores))", "order = np.lexsort((-np.arange(n), -scores))")],
+    "scale 1/D": [("z = (qh @ rows.T) * head_dim_scale", "z = (qh @ rows.T) * head_dim_scale ** 2")],
+    "query not normalised": [("qh = rope(rms_norm(q, widen(q_norm_g), eps), pos, rope_dim, rope_base)",
+                              "qh = rope(q * widen(q_norm_g), pos, rope_dim, rope_base)")],
+    "query not rotated": [("qh = rope(rms_norm(q, widen(q_norm_g), eps), pos, rope_dim, rope_base)",
+                           "qh = rms_norm(q, widen(q_norm_g), eps)")],
+    "rmsnorm without eps": [("return x / np.sqrt(ms + eps) * np.asarray(g, dtype=np.float64)",
+                             "return x / np.sqrt(ms) * np.asarray(g, dtype=np.float64)")],
+    "rmsnorm without gain": [("return x / np.sqrt(ms + eps) * np.asarray(g, dtype=np.float64)",
+                              "return x / np.sqrt(ms + eps)")],
+    "overlap forward": [("t = (i - 1) * m + r - tok_begin", "t = (i + 1) * m + r - tok_begin")],
+    "softmax over channels": [("wgt = e / e.sum(axis=0, keepdims=True)", "wgt = e / e.sum(axis=1, keepdims=True)")],
+    "biases swapped": [("logits.append(za[t] + ba[r])", "logits.append(za[t] + (bb[r] if bb is not None else ba[r]))")],
+    "entry position (i+1)m-1": [("e = rope(e, i * m, rope_dim, rope_base)", "e = rope(e, (i + 1) * m - 1, rope_dim, rope_base)")],
+    "HCA ignores visibility": [('"""HCA: keys = every visible pool entry followed by the window."""\n    n_vis = min(visible_entries(pos, cfg.ratio), n_c)',
+                                '"""HCA: keys = every visible pool entry followed by the window."""\n    n_vis = n_c')],
+    "window ring slot": [("return widen(win)[window_positions(pos, window) % win_cap]",
+                          "return widen(win)[window_positions(pos, window) % win.shape[0] if False else window_positions(pos, window) - window_positions(pos, window)[0]]")],
+    "pool row ignores idx": [("rows = np.concatenate([widen(pool)[sel], window_rows",
+                              "rows = np.concatenate([widen(pool)[: sel.size], window_rows")],
+}
+
+
+def _load(name, edits, replace_all):
+    src = open(SRC).read()
+    for old, new in edits:
+        n = src.count(old)
+        assert n >= 1, f"mutant {name!r}: {old!r} not found"
+        if not replace_all:
+            assert n == 1, f"mutant {name!r}: {old!r} found {n} times"
+        src = src.replace(old, new)
+    mod = types.ModuleType("oracle_mutant")
+    mod.__file__ = SRC
+    exec(compile(src, SRC, "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name):
+    mod = _load(name, MUTANTS[name], name.endswith("*"))
+    failed = []
+    for pin in PINS:
+        try:
+            pin(mod)
+        except Exception as e:  # AssertionError or a crash both reject it
+            failed.append(pin.__name__)
+    assert failed, f"no pin rejects the mutant {name!r}"

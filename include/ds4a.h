@@ -1,0 +1,212 @@
+/*
+ * ds4a.h -- C ABI of the B200 (sm_100a) DeepSeek-V4 hybrid attention hot path:
+ * KV compressor, Lightning-Indexer top-k, and shared K=V multi-query attention
+ * with a per-head sink merged with the sliding window (CSA), or over every
+ * pooled entry (HCA).
+ *
+ * Sources of the operations (page title, then section / equation):
+ *   [V4-inside] "DeepSeek V4 Inside: One Token Through Every Block"
+ *   [beyond]    "DeepSeek-v4 Beyond Basics", sections 3.2.2 and 3.3
+ *   [module1]   "Phase 1 Module 1 - The model & the cost of attention"
+ *   [hf-doc]    "DeepSeek-V4" (Transformers documentation)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Ownership: the caller owns every buffer.  The library allocates nothing
+ *   per call; scratch memory ("workspace") is passed in by the caller and
+ *   sized by the *_workspace queries.  Library state: one device error word
+ *   per device, and an optional launch trace (ds4a_trace_*), off by default.
+ * - Execution: every call is asynchronous on the given CUDA stream (NULL =
+ *   the legacy default stream).  Pointers named "device" must be device (or
+ *   managed) memory of the current device; "host" pointers are host memory.
+ * - Storage types: ds4a_bf16 is a bfloat16 bit pattern.  Arithmetic is
+ *   float32 (bf16 x bf16 products accumulated in float32 on tensor cores).
+ * - Layouts: contiguous row-major, dimensions listed outermost first; batch
+ *   strides, where given, are in elements.  Every bf16 / float / int32 array
+ *   must start on a 16-byte boundary.
+ * - Positions are absolute and 0-based.  A compressed entry i of ratio m is
+ *   visible to a query at position t iff i < floor((t + 1) / m).  The window
+ *   of a query at t is positions max(0, t - window + 1) .. t, read from a
+ *   ring at slot (position mod win_cap).
+ * - Return codes: DS4A_OK, or DS4A_EINVAL (null / misaligned pointer, bad
+ *   size or configuration; nothing is launched), DS4A_EUNSUPPORTED (no kernel
+ *   for this shape), DS4A_ECUDA (a launch failed), DS4A_ENOSPACE (workspace
+ *   too small).  Errors found by kernels (an index out of range, a negative
+ *   position, a bounded wait that ran out) are recorded in the device error
+ *   word and reported by ds4a_check; kernels never trap.
+ */
+#ifndef DS4A_H
+#define DS4A_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t ds4a_bf16;
+typedef struct CUstream_st* ds4a_stream; /* same type as cudaStream_t */
+
+enum {
+  DS4A_OK = 0,
+  DS4A_EINVAL = 1,
+  DS4A_EUNSUPPORTED = 2,
+  DS4A_ECUDA = 3,
+  DS4A_EDEVICE = 4,
+  DS4A_ETIMEOUT = 5,
+  DS4A_ENOSPACE = 6
+};
+
+/* Bits of the device error word (ds4a_check). */
+enum {
+  DS4A_DEV_BAD_INDEX = 1u, /* an index >= N_c or < -1 was skipped             */
+  DS4A_DEV_BAD_POS = 2u,   /* a negative query position was skipped          */
+  DS4A_DEV_TIMEOUT = 4u    /* a bounded wait inside a kernel ran out          */
+};
+
+/* One attention layer.  Flash-0731 CSA: {64, 512, 64, 128, 64, 128, 512, 4,
+ * 1/sqrt(512), 10000, 1e-6}; HCA: the same with ratio 128 ([V4-inside]
+ * config JSON and knob table).
+ *   n_heads   query heads H (all share one K=V head)
+ *   head_dim  D, channels of a query head and of a K=V row
+ *   rope_dim  R, the last R channels carry interleaved-pair RoPE
+ *   window    W, sliding-window length (0 = no window)
+ *   idx_heads H_I, idx_dim D_I: indexer heads and their width
+ *   topk      k, entries kept by the indexer
+ *   ratio     m, tokens per compressed entry (CSA 4, HCA 128)
+ *   sm_scale  softmax scale (1/sqrt(D))
+ *   rope_base theta_j = rope_base^(-2j/R)
+ *   rms_eps   RMSNorm epsilon */
+typedef struct ds4a_layer_cfg {
+  int32_t n_heads, head_dim, rope_dim, window, idx_heads, idx_dim, topk, ratio;
+  float sm_scale, rope_base, rms_eps;
+} ds4a_layer_cfg;
+
+/*
+ * ds4a_compress -- KV compressor ([beyond] 3.2.2 eqs. 9-12 for CSA with
+ * overlapping blocks; 3.3 eqs. 20-23 for HCA; [V4-inside] "How does CSA
+ * compress 8 tokens into 4 KV entries?").
+ *
+ * For entry i and channel ch, one softmax over the logits
+ *   Z^a[i*m + r][ch] + B^a[r][ch]                     (r < m, own block)
+ *   Z^b[(i-1)*m + r][ch] + B^b[r][ch]                 (r < m, previous block;
+ *                                                      CSA only, i >= 1)
+ * weights the matching C^a / C^b values; their sum is the entry.  With
+ * norm_g the entry is then RMS-normalised (eps cfg->rms_eps) times norm_g,
+ * and RoPE at position i*m rotates its last cfg->rope_dim channels.  Without
+ * norm_g (indexer keys) the weighted sum is stored as is.
+ *
+ *   B, T_tok, c   streams ca/cb/za/zb are device bf16 [B, T_tok, c]; row r is
+ *                 token tok_begin + r.  cb == NULL (and zb, bias_b NULL)
+ *                 selects the single-stream HCA form.
+ *   bias_a/b      device float [m, c] (m = cfg->ratio)
+ *   norm_g        device float [c] or NULL
+ *   entries       entry_begin .. entry_end-1 are written; every token they
+ *                 read must lie in [tok_begin, tok_begin + T_tok)
+ *   pool          device bf16; entry i of batch b goes to
+ *                 pool + b * pool_bstride + i * c
+ * c must be even and <= 1024, and a multiple of 8 when above 512 (a
+ * multiple of 8 takes 16-byte vector loads);
+ * cfg->rope_dim <= c when norm_g is given.
+ */
+int ds4a_compress(const ds4a_layer_cfg* cfg, int B, int T_tok, int tok_begin, int c,
+                  const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                  const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                  const float* norm_g, int entry_begin, int entry_end, ds4a_bf16* pool,
+                  int64_t pool_bstride, ds4a_stream stream);
+
+/* Bytes of workspace ds4a_index_topk needs for these sizes. */
+size_t ds4a_index_topk_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c);
+
+/*
+ * ds4a_index_topk -- Lightning Indexer score and top-k selector ([beyond]
+ * 3.2.2 eqs. 13-17; [module1] "The indexer"; [hf-doc] mask layout).
+ *
+ *   I[t][s] = sum_h w[t][h] * ReLU(q[t][h] . K[s])   for visible s
+ * keeps the cfg->topk highest scores per query (ties to the lower index) and
+ * writes their indices ascending, padded with -1 when fewer are visible.
+ *
+ *   q_pos   device int32 [B, T_q]      query positions
+ *   q_idx   device bf16 [B, T_q, H_I, D_I]
+ *   w_idx   device bf16 [B, T_q, H_I]
+ *   k_idx   device bf16, batch b's entries at k_idx + b * k_bstride,
+ *           [N_c, D_I] each (the indexer-key pool)
+ *   idx_out device int32 [B, T_q, k]
+ *   score_out device float [B, T_q, k] (score of each kept index, -inf for
+ *           -1 slots) or NULL
+ *   ws      device workspace of ws_bytes >= ds4a_index_topk_workspace(...)
+ */
+int ds4a_index_topk(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                    const ds4a_bf16* q_idx, const ds4a_bf16* w_idx, const ds4a_bf16* k_idx,
+                    int64_t k_bstride, int N_c, int32_t* idx_out, float* score_out, void* ws,
+                    size_t ws_bytes, ds4a_stream stream);
+
+/* Bytes of workspace the attend calls can use for these sizes (split over
+ * more thread blocks when few queries are given).  Passing less (even 0)
+ * is allowed: the work is then split less. */
+size_t ds4a_attend_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c, int sparse);
+
+/*
+ * ds4a_sparse_attend -- CSA core attention ([beyond] 3.2.2 eq. 19 and 3.3
+ * eqs. 24-27; [V4-inside] layer-0 SWA sink example and the CSA example with
+ * one compressed and two window keys; [hf-doc] partial RoPE, sink, window).
+ *
+ * Per query (b, t) at position p and head h:
+ *   q^ = RoPE_p(RMSNorm(q[b][t][h]) * q_norm_g)
+ *   keys = pool[idx[b][t][j]] for idx >= 0, then the window rows
+ *   z = q^ . kv * sm_scale;  p = exp(z) / (sum exp(z) + exp(sink[h]))
+ *   o = sum p * kv;  out[b][t][h] = RoPE_{-p}(o) on the last R channels
+ * K and V are the same row (shared K=V MQA).
+ *
+ *   q       device bf16 [B, T_q, H, D]; q_norm_g device float [D]
+ *   pool    device bf16, batch b at pool + b * pool_bstride, [N_c, D]
+ *   idx     device int32 [B, T_q, k] ascending, -1 padded (ds4a_index_topk)
+ *   win     device bf16, batch b at win + b * win_bstride, [win_cap, D]: the
+ *           raw K=V rows of the window, slot = position mod win_cap
+ *   sink    device float [H]
+ *   out     device bf16 [B, T_q, H, D]
+ *   ws      device workspace (may be NULL with ws_bytes 0)
+ */
+int ds4a_sparse_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                       const ds4a_bf16* q, const float* q_norm_g, const ds4a_bf16* pool,
+                       int64_t pool_bstride, int N_c, const int32_t* idx, const ds4a_bf16* win,
+                       int win_cap, int64_t win_bstride, const float* sink, ds4a_bf16* out,
+                       void* ws, size_t ws_bytes, ds4a_stream stream);
+
+/*
+ * ds4a_hca_attend -- HCA core attention ([beyond] 3.3; [V4-inside] "What
+ * does HCA change?"; [hf-doc] HCA layer).  As ds4a_sparse_attend with the
+ * keys = every visible pool entry (i < floor((p+1)/m), i < N_c), then the
+ * window.  With N_c = 0 it is the sliding-window-only layer.
+ */
+int ds4a_hca_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                    const ds4a_bf16* q, const float* q_norm_g, const ds4a_bf16* pool,
+                    int64_t pool_bstride, int N_c, const ds4a_bf16* win, int win_cap,
+                    int64_t win_bstride, const float* sink, ds4a_bf16* out, void* ws,
+                    size_t ws_bytes, ds4a_stream stream);
+
+/* Synchronise the stream, then read and clear the current device's error
+ * word.  Returns DS4A_OK, DS4A_EDEVICE (bad index / position),
+ * DS4A_ETIMEOUT (a bounded wait ran out) or DS4A_ECUDA (a CUDA error is
+ * pending).  bits_out (host, nullable) receives the DS4A_DEV_* bits. */
+int ds4a_check(ds4a_stream stream, uint32_t* bits_out);
+
+/* Static text for a return code. */
+const char* ds4a_strerror(int code);
+
+/* Launch trace (for benchmarking): while enabled, every kernel launch is
+ * bracketed by CUDA events on its stream.  ds4a_trace_read synchronises the
+ * device and copies up to cap records (kernel name, milliseconds) into the
+ * host arrays, returning how many launches were recorded; names point to
+ * static strings.  Enabling clears the trace.  Not thread safe. */
+int ds4a_trace_enable(int on);
+int ds4a_trace_read(const char** names, float* ms, int cap);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int ds4a_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DS4A_H */

@@ -1,0 +1,293 @@
+// extern "C" entry points of libds4a: argument checks (before any launch),
+// dispatch to the kernels, the device error word and the launch trace.
+#include "ds4a_internal.cuh"
+
+#include <math.h>
+#include <stdio.h>
+#include <vector>
+
+namespace ds4a {
+
+__device__ unsigned int g_err_word = 0;
+
+unsigned int* err_word() {
+  static unsigned int* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return addr[dev];
+}
+
+// ---------------------------------------------------------------------------
+// launch trace
+// ---------------------------------------------------------------------------
+namespace {
+struct TraceRec {
+  const char* name;
+  cudaEvent_t e0, e1;
+};
+bool g_trace_on = false;
+std::vector<TraceRec> g_trace;
+std::vector<cudaEvent_t> g_event_pool;
+size_t g_event_used = 0;
+
+cudaEvent_t next_event() {
+  if (g_event_used == g_event_pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    g_event_pool.push_back(e);
+  }
+  return g_event_pool[g_event_used++];
+}
+}  // namespace
+
+TraceScope::TraceScope(const char* n, cudaStream_t s) : name(n), stream(s), slot(-1) {
+  if (!g_trace_on) return;
+  TraceRec r{n, next_event(), next_event()};
+  if (!r.e0 || !r.e1) return;
+  cudaEventRecord(r.e0, s);
+  g_trace.push_back(r);
+  slot = (int)g_trace.size() - 1;
+}
+
+TraceScope::~TraceScope() {
+  if (slot >= 0) cudaEventRecord(g_trace[slot].e1, stream);
+}
+
+}  // namespace ds4a
+
+using namespace ds4a;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const ds4a_layer_cfg* c) {
+  if (!c) return DS4A_EINVAL;
+  if (c->n_heads < 1 || c->n_heads > 128) return DS4A_EINVAL;
+  if (c->head_dim < 8 || c->head_dim > 512 || (c->head_dim % 8) != 0) return DS4A_EINVAL;
+  if (c->rope_dim < 0 || c->rope_dim > c->head_dim || (c->rope_dim & 1)) return DS4A_EINVAL;
+  if (c->window < 0 || c->ratio < 1) return DS4A_EINVAL;
+  if (!(c->sm_scale > 0.f) || !(c->rope_base > 0.f) || !(c->rms_eps >= 0.f)) return DS4A_EINVAL;
+  return DS4A_OK;
+}
+
+int check_index_cfg(const ds4a_layer_cfg* c) {
+  if (!c) return DS4A_EINVAL;
+  if (c->idx_heads < 1 || c->idx_heads > 128) return DS4A_EINVAL;
+  if (c->idx_dim < 1 || c->idx_dim > 128) return DS4A_EINVAL;
+  if (c->topk < 1 || c->topk > 4096 || c->ratio < 1) return DS4A_EINVAL;
+  return DS4A_OK;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? DS4A_OK : DS4A_ECUDA; }
+
+size_t index_ws_bytes(int B, int T_q, int N_c) {
+  return (size_t)B * (size_t)T_q * (size_t)(N_c > 0 ? N_c : 0) * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ds4a_version(void) { return 100; }
+
+const char* ds4a_strerror(int code) {
+  switch (code) {
+    case DS4A_OK: return "ok";
+    case DS4A_EINVAL: return "invalid argument (null or misaligned pointer, bad size or config)";
+    case DS4A_EUNSUPPORTED: return "unsupported shape";
+    case DS4A_ECUDA: return "CUDA error";
+    case DS4A_EDEVICE: return "device reported a bad index or position";
+    case DS4A_ETIMEOUT: return "a bounded wait inside a kernel ran out";
+    case DS4A_ENOSPACE: return "workspace too small";
+    default: return "unknown error";
+  }
+}
+
+int ds4a_compress(const ds4a_layer_cfg* cfg, int B, int T_tok, int tok_begin, int c,
+                  const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                  const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                  const float* norm_g, int entry_begin, int entry_end, ds4a_bf16* pool,
+                  int64_t pool_bstride, ds4a_stream stream) {
+  if (!cfg || cfg->ratio < 1) return DS4A_EINVAL;
+  if (B < 0 || T_tok < 0 || c < 2 || c > 1024 || (c % 2) != 0) return DS4A_EINVAL;
+  if ((c % 8) != 0 && c > 512) return DS4A_EINVAL;  // the 2-wide path covers up to 512
+  if (entry_begin < 0 || entry_end < entry_begin) return DS4A_EINVAL;
+  if (entry_end == entry_begin || B == 0) return DS4A_OK;
+  if (!ca || !za || !bias_a || !pool) return DS4A_EINVAL;
+  const bool overlap = cb != nullptr;
+  if (overlap && (!zb || !bias_b)) return DS4A_EINVAL;
+  if (!overlap && (zb || bias_b)) return DS4A_EINVAL;
+  if (!aligned16(ca) || !aligned16(za) || !aligned16(bias_a) || !aligned16(pool)) return DS4A_EINVAL;
+  if (overlap && (!aligned16(cb) || !aligned16(zb) || !aligned16(bias_b))) return DS4A_EINVAL;
+  if (norm_g) {
+    if (check_cfg(cfg) != DS4A_OK) return DS4A_EINVAL;
+    if (cfg->rope_dim > c) return DS4A_EINVAL;
+  }
+  if (pool_bstride < (int64_t)entry_end * c || (pool_bstride % 8) != 0) return DS4A_EINVAL;
+  const int m = cfg->ratio;
+  // every token the entries read must be in the streams
+  const int64_t first_tok = (overlap && entry_begin >= 1) ? (int64_t)(entry_begin - 1) * m
+                                                          : (int64_t)entry_begin * m;
+  const int64_t last_tok = (int64_t)entry_end * m - 1;
+  if (first_tok < tok_begin || last_tok >= (int64_t)tok_begin + T_tok) return DS4A_EINVAL;
+
+  CompressArgs a;
+  a.B = B; a.T_tok = T_tok; a.tok_begin = tok_begin; a.c = c; a.m = m;
+  a.rope_dim = norm_g ? cfg->rope_dim : 0;
+  a.rope_base = cfg->rope_base; a.eps = cfg->rms_eps;
+  a.ca = ca; a.cb = cb; a.za = za; a.zb = zb;
+  a.bias_a = bias_a; a.bias_b = bias_b; a.norm_g = norm_g;
+  a.entry_begin = entry_begin; a.entry_end = entry_end;
+  a.pool = pool; a.pool_bstride = pool_bstride;
+  a.err = err_word();
+  if (!a.err) return DS4A_ECUDA;
+  return cuda_rc(launch_compress(a, (cudaStream_t)stream));
+}
+
+size_t ds4a_index_topk_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c) {
+  (void)cfg;
+  if (B <= 0 || T_q <= 0 || N_c <= 0) return 0;
+  return index_ws_bytes(B, T_q, N_c);
+}
+
+int ds4a_index_topk(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                    const ds4a_bf16* q_idx, const ds4a_bf16* w_idx, const ds4a_bf16* k_idx,
+                    int64_t k_bstride, int N_c, int32_t* idx_out, float* score_out, void* ws,
+                    size_t ws_bytes, ds4a_stream stream) {
+  if (check_index_cfg(cfg) != DS4A_OK) return DS4A_EINVAL;
+  if (B < 0 || T_q < 0 || N_c < 0) return DS4A_EINVAL;
+  if (B == 0 || T_q == 0) return DS4A_OK;
+  if (!q_pos || !q_idx || !w_idx || !idx_out) return DS4A_EINVAL;
+  if (N_c > 0 && (!k_idx || !ws)) return DS4A_EINVAL;
+  if (!aligned16(q_pos) || !aligned16(q_idx) || !aligned16(w_idx) || !aligned16(idx_out))
+    return DS4A_EINVAL;
+  if ((k_idx && !aligned16(k_idx)) || (score_out && !aligned16(score_out)) || (ws && !aligned16(ws)))
+    return DS4A_EINVAL;
+  if (N_c > 0 && k_bstride < (int64_t)N_c * cfg->idx_dim) return DS4A_EINVAL;
+  if (ws_bytes < index_ws_bytes(B, T_q, N_c)) return DS4A_ENOSPACE;
+
+  IndexArgs a;
+  a.B = B; a.T_q = T_q; a.H = cfg->idx_heads; a.D = cfg->idx_dim; a.m = cfg->ratio;
+  a.k = cfg->topk; a.N_c = N_c;
+  a.q_pos = q_pos; a.q = q_idx; a.w = w_idx; a.kidx = k_idx; a.k_bstride = k_bstride;
+  a.scores = reinterpret_cast<float*>(ws);
+  a.idx_out = idx_out; a.score_out = score_out;
+  a.err = err_word();
+  if (!a.err) return DS4A_ECUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (N_c > 0) {
+    e = index_scores_tc_supported(a) ? launch_index_scores_tc(a, s) : launch_index_scores_generic(a, s);
+    if (e != cudaSuccess) return DS4A_ECUDA;
+  }
+  return cuda_rc(launch_topk(a, s));
+}
+
+size_t ds4a_attend_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c, int sparse) {
+  if (check_cfg(cfg) != DS4A_OK || B <= 0 || T_q <= 0) return 0;
+  const int keys_max = (sparse ? cfg->topk : (N_c > 0 ? N_c : 0)) + cfg->window;
+  size_t need = 0;
+  attend_splits(B, T_q, keys_max, cfg->n_heads, cfg->head_dim, (size_t)-1, &need);
+  return need;
+}
+
+static int attend_common(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                         const ds4a_bf16* q, const float* q_norm_g, const ds4a_bf16* pool,
+                         int64_t pool_bstride, int N_c, const int32_t* idx, const ds4a_bf16* win,
+                         int win_cap, int64_t win_bstride, const float* sink, ds4a_bf16* out,
+                         void* ws, size_t ws_bytes, ds4a_stream stream, int sparse) {
+  if (check_cfg(cfg) != DS4A_OK) return DS4A_EINVAL;
+  if (sparse && (cfg->topk < 1 || cfg->topk > 4096)) return DS4A_EINVAL;
+  if (B < 0 || T_q < 0 || N_c < 0) return DS4A_EINVAL;
+  if (B == 0 || T_q == 0) return DS4A_OK;
+  if (!q_pos || !q || !q_norm_g || !sink || !out) return DS4A_EINVAL;
+  if (N_c > 0 && !pool) return DS4A_EINVAL;
+  if (sparse && !idx) return DS4A_EINVAL;
+  if (cfg->window > 0 && (!win || win_cap < cfg->window)) return DS4A_EINVAL;
+  if (!aligned16(q_pos) || !aligned16(q) || !aligned16(q_norm_g) || !aligned16(sink) || !aligned16(out))
+    return DS4A_EINVAL;
+  if ((pool && !aligned16(pool)) || (idx && !aligned16(idx)) || (win && !aligned16(win)) ||
+      (ws && !aligned16(ws)))
+    return DS4A_EINVAL;
+  const int D = cfg->head_dim;
+  if (N_c > 0 && (pool_bstride < (int64_t)N_c * D || (pool_bstride % 8) != 0)) return DS4A_EINVAL;
+  if (cfg->window > 0 && (win_bstride < (int64_t)win_cap * D || (win_bstride % 8) != 0))
+    return DS4A_EINVAL;
+  if (ws_bytes > 0 && !ws) return DS4A_EINVAL;
+
+  AttendArgs a;
+  a.B = B; a.T_q = T_q; a.H = cfg->n_heads; a.D = D; a.R = cfg->rope_dim; a.W = cfg->window;
+  a.m = cfg->ratio; a.k = cfg->topk; a.N_c = N_c; a.win_cap = win_cap; a.sparse = sparse;
+  a.scale = cfg->sm_scale; a.rope_base = cfg->rope_base; a.eps = cfg->rms_eps;
+  a.q_pos = q_pos; a.q = q; a.q_norm_g = q_norm_g; a.pool = pool; a.pool_bstride = pool_bstride;
+  a.idx = idx; a.win = win; a.win_bstride = win_bstride; a.sink = sink; a.out = out;
+  a.ws = reinterpret_cast<float*>(ws);
+  a.keys_max = (sparse ? cfg->topk : N_c) + cfg->window;
+  a.err = err_word();
+  if (!a.err) return DS4A_ECUDA;
+  a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, ws ? ws_bytes : 0, nullptr);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (attend_tc_supported(a)) return cuda_rc(launch_attend_tc(a, s));
+  return cuda_rc(launch_attend_generic(a, s));
+}
+
+int ds4a_sparse_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                       const ds4a_bf16* q, const float* q_norm_g, const ds4a_bf16* pool,
+                       int64_t pool_bstride, int N_c, const int32_t* idx, const ds4a_bf16* win,
+                       int win_cap, int64_t win_bstride, const float* sink, ds4a_bf16* out,
+                       void* ws, size_t ws_bytes, ds4a_stream stream) {
+  return attend_common(cfg, B, T_q, q_pos, q, q_norm_g, pool, pool_bstride, N_c, idx, win, win_cap,
+                       win_bstride, sink, out, ws, ws_bytes, stream, 1);
+}
+
+int ds4a_hca_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                    const ds4a_bf16* q, const float* q_norm_g, const ds4a_bf16* pool,
+                    int64_t pool_bstride, int N_c, const ds4a_bf16* win, int win_cap,
+                    int64_t win_bstride, const float* sink, ds4a_bf16* out, void* ws,
+                    size_t ws_bytes, ds4a_stream stream) {
+  return attend_common(cfg, B, T_q, q_pos, q, q_norm_g, pool, pool_bstride, N_c, nullptr, win,
+                       win_cap, win_bstride, sink, out, ws, ws_bytes, stream, 0);
+}
+
+int ds4a_check(ds4a_stream stream, uint32_t* bits_out) {
+  if (bits_out) *bits_out = 0;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return DS4A_ECUDA;
+  unsigned int bits = 0;
+  if (cudaMemcpyFromSymbol(&bits, g_err_word, sizeof(bits)) != cudaSuccess) return DS4A_ECUDA;
+  if (bits) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero)) != cudaSuccess) return DS4A_ECUDA;
+  }
+  if (bits_out) *bits_out = bits;
+  if (bits & DS4A_DEV_TIMEOUT) return DS4A_ETIMEOUT;
+  if (bits) return DS4A_EDEVICE;
+  return cuda_rc(cudaGetLastError());
+}
+
+int ds4a_trace_enable(int on) {
+  g_trace_on = on != 0;
+  g_trace.clear();
+  g_event_used = 0;
+  return DS4A_OK;
+}
+
+int ds4a_trace_read(const char** names, float* ms, int cap) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -DS4A_ECUDA;
+  const int n = (int)g_trace.size();
+  for (int i = 0; i < n && i < cap; ++i) {
+    if (names) names[i] = g_trace[i].name;
+    float t = 0.f;
+    cudaEventElapsedTime(&t, g_trace[i].e0, g_trace[i].e1);
+    if (ms) ms[i] = t;
+  }
+  return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,664 @@
+// Shape-generic CUDA kernels of the ds4a path: the KV compressor, the
+// indexer score (CUDA-core form), the top-k selector, the split attention
+// (CUDA-core form) and its combine.  They serve every shape the ABI accepts
+// (the toy widths included); the Flash-0731 shapes take the tensor-core
+// kernels of ds4a_index_tc.cu / ds4a_attend_tc.cu where those apply.
+#include "ds4a_internal.cuh"
+
+#include <float.h>
+
+namespace ds4a {
+
+// ===========================================================================
+// KV compressor ("DeepSeek-v4 Beyond Basics" 3.2.2 eqs. 9-12 and 3.3
+// eqs. 20-23): per channel, a softmax over the 2m (CSA) or m (HCA) logits
+// Z + B weights the matching C values; then RMSNorm * g and RoPE at i*m.
+// One thread block per (entry, sequence).  Thread t owns channels
+// [8*(t % NC), 8*(t % NC) + 8) (NC = c/8) and the terms g, g+G, ... of the
+// entry (g = t / NC, G = 256 / NC); the G partial softmaxes merge in shared
+// memory.  Loads are 16-byte vectors of 8 bf16.
+// ===========================================================================
+constexpr int kCompressThreads = 256;
+
+template <int V>
+struct VecLoad;
+template <>
+struct VecLoad<8> {  // 8 bf16 = 16 bytes
+  __device__ static void load(const uint16_t* p, float* out) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    const unsigned int w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = bf2x2_to_f2(w[u]);
+      out[2 * u] = f.x;
+      out[2 * u + 1] = f.y;
+    }
+  }
+  __device__ static void load_f(const float* p, float* out) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+  }
+};
+template <>
+struct VecLoad<2> {  // 2 bf16 = 4 bytes
+  __device__ static void load(const uint16_t* p, float* out) {
+    const float2 f = bf2x2_to_f2(*reinterpret_cast<const unsigned int*>(p));
+    out[0] = f.x;
+    out[1] = f.y;
+  }
+  __device__ static void load_f(const float* p, float* out) {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    out[0] = a.x;
+    out[1] = a.y;
+  }
+};
+
+template <int V>
+__global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs a) {
+  extern __shared__ float csm[];
+  const int c = a.c, m = a.m;
+  const int NC = c / V;
+  const int G = kCompressThreads / NC;
+  const int tid = threadIdx.x;
+  const int cc = tid % NC;
+  const int g = tid / NC;
+  const int i = a.entry_begin + blockIdx.x;
+  const int b = blockIdx.y;
+  const bool overlap = a.cb != nullptr;
+  const int n_terms = (overlap && i >= 1) ? 2 * m : m;
+
+  float mx[V], l[V], acc[V];
+#pragma unroll
+  for (int u = 0; u < V; ++u) { mx[u] = -INFINITY; l[u] = 0.f; acc[u] = 0.f; }
+
+  if (g < G) {
+    for (int term = g; term < n_terms; term += G) {
+      const bool half_a = term < m;
+      const int r = half_a ? term : term - m;
+      const int tok = half_a ? i * m + r : (i - 1) * m + r;
+      const int64_t row = (int64_t)b * a.T_tok + (tok - a.tok_begin);
+      float vals[V], zs[V], bs[V];
+      VecLoad<V>::load((half_a ? a.ca : a.cb) + row * c + cc * V, vals);
+      VecLoad<V>::load((half_a ? a.za : a.zb) + row * c + cc * V, zs);
+      VecLoad<V>::load_f((half_a ? a.bias_a : a.bias_b) + (int64_t)r * c + cc * V, bs);
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const float x = zs[q] + bs[q];
+        if (x > mx[q]) {
+          const float sc = __expf(mx[q] - x);
+          l[q] = l[q] * sc + 1.f;
+          acc[q] = acc[q] * sc + vals[q];
+          mx[q] = x;
+        } else {
+          const float e = __expf(x - mx[q]);
+          l[q] += e;
+          acc[q] += e * vals[q];
+        }
+      }
+    }
+  }
+  // merge the G partials of every channel
+  float* s_m = csm;                 // [G * c]
+  float* s_l = s_m + G * c;         // [G * c]
+  float* s_a = s_l + G * c;         // [G * c]
+  float* s_v = s_a + G * c;         // [c]
+  __shared__ float s_red[kCompressThreads / 32];
+  if (g < G) {
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      s_m[g * c + cc * V + u] = mx[u];
+      s_l[g * c + cc * V + u] = l[u];
+      s_a[g * c + cc * V + u] = acc[u];
+    }
+  }
+  __syncthreads();
+  float ss = 0.f;
+  for (int ch = tid; ch < c; ch += kCompressThreads) {
+    float M = -INFINITY;
+    for (int gg = 0; gg < G; ++gg) M = fmaxf(M, s_m[gg * c + ch]);
+    float Ls = 0.f, A = 0.f;
+    for (int gg = 0; gg < G; ++gg) {
+      const float mm = s_m[gg * c + ch];
+      if (mm == -INFINITY) continue;
+      const float e = __expf(mm - M);
+      Ls += s_l[gg * c + ch] * e;
+      A += s_a[gg * c + ch] * e;
+    }
+    const float v = A / Ls;
+    s_v[ch] = v;
+    ss += v * v;
+  }
+  uint16_t* dst = a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c;
+  if (a.norm_g == nullptr) {
+    __syncthreads();
+    for (int ch = tid; ch < c; ch += kCompressThreads) dst[ch] = f2bf(s_v[ch]);
+    return;
+  }
+  ss = warp_sum(ss);
+  if ((tid & 31) == 0) s_red[tid >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCompressThreads / 32; ++w) tot += s_red[w];
+  const float rstd = rsqrtf(tot / (float)c + a.eps);
+  const int R = a.rope_dim;
+  const int pos = i * m;
+  for (int p2 = tid; p2 < c / 2; p2 += kCompressThreads) {
+    const int ch = 2 * p2;
+    float x0 = s_v[ch] * rstd * a.norm_g[ch];
+    float x1 = s_v[ch + 1] * rstd * a.norm_g[ch + 1];
+    if (ch >= c - R) {
+      float cs, sn;
+      rope_cos_sin(pos, (ch - (c - R)) >> 1, R, a.rope_base, &cs, &sn);
+      const float y0 = x0 * cs - x1 * sn;
+      const float y1 = x0 * sn + x1 * cs;
+      x0 = y0;
+      x1 = y1;
+    }
+    *reinterpret_cast<unsigned int*>(dst + ch) = f2_to_bf2x2(x0, x1);
+  }
+}
+
+cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
+  const int n = a.entry_end - a.entry_begin;
+  if (n <= 0 || a.B <= 0) return cudaSuccess;
+  const int V = (a.c % 8 == 0) ? 8 : 2;
+  const int NC = a.c / V;
+  const int G = NC >= kCompressThreads ? 1 : kCompressThreads / NC;
+  const size_t smem = (size_t)(3 * G * a.c + a.c) * sizeof(float);
+  static unsigned long long attr_mask = 0;
+  set_smem_attr_once(compress_kernel<8>, 200 * 1024, &attr_mask, 0);
+  set_smem_attr_once(compress_kernel<2>, 200 * 1024, &attr_mask, 1);
+  TraceScope tr("compress", s);
+  if (V == 8)
+    compress_kernel<8><<<dim3(n, a.B), kCompressThreads, smem, s>>>(a);
+  else
+    compress_kernel<2><<<dim3(n, a.B), kCompressThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// Indexer score, CUDA-core form (any H_I, D_I <= 128)
+// ("DeepSeek-v4 Beyond Basics" 3.2.2 eq. 16):
+//   I[s] = sum_h w[h] * ReLU(q[h] . K[s])  for visible s.
+// One thread per key; the key tile is staged in shared memory (stride D+1
+// keeps the per-thread row reads free of bank conflicts).
+// ===========================================================================
+constexpr int kIdxKeys = 128;
+
+__global__ void __launch_bounds__(kIdxKeys) index_score_generic_kernel(IndexArgs a) {
+  extern __shared__ float ism[];
+  const int H = a.H, D = a.D;
+  float* qs = ism;              // [H * D]
+  float* wsum = qs + H * D;     // [H]
+  float* kt = wsum + H;         // [128 * (D + 1)]
+  const int row = blockIdx.x;
+  const int b = row / a.T_q;
+  const int pos = a.q_pos[row];
+  if (pos < 0) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
+    return;
+  }
+  const int n_vis = min((pos + 1) / a.m, a.N_c);
+  const int s0 = blockIdx.y * kIdxKeys;
+  if (s0 >= n_vis) return;
+  for (int e = threadIdx.x; e < H * D; e += kIdxKeys) qs[e] = bf2f(a.q[(int64_t)row * H * D + e]);
+  for (int e = threadIdx.x; e < H; e += kIdxKeys) wsum[e] = bf2f(a.w[(int64_t)row * H + e]);
+  const int nk = min(kIdxKeys, n_vis - s0);
+  const uint16_t* kb = a.kidx + (int64_t)b * a.k_bstride + (int64_t)s0 * D;
+  for (int e = threadIdx.x; e < nk * D; e += kIdxKeys) kt[(e / D) * (D + 1) + (e % D)] = bf2f(kb[e]);
+  __syncthreads();
+  const int t = threadIdx.x;
+  if (t >= nk) return;
+  const float* kr = kt + t * (D + 1);
+  float score = 0.f;
+  for (int h = 0; h < H; ++h) {
+    const float* qh = qs + h * D;
+    float dot = 0.f;
+    for (int d = 0; d < D; ++d) dot = fmaf(qh[d], kr[d], dot);
+    score = fmaf(wsum[h], fmaxf(dot, 0.f), score);
+  }
+  a.scores[(int64_t)row * a.N_c + s0 + t] = score;
+}
+
+cudaError_t launch_index_scores_generic(const IndexArgs& a, cudaStream_t s) {
+  const int rows = a.B * a.T_q;
+  if (rows <= 0 || a.N_c <= 0) return cudaSuccess;
+  const size_t smem = (size_t)(a.H * a.D + a.H + kIdxKeys * (a.D + 1)) * sizeof(float);
+  static unsigned long long attr_mask = 0;
+  set_smem_attr_once(index_score_generic_kernel, 200 * 1024, &attr_mask, 0);
+  TraceScope tr("index_score_generic", s);
+  index_score_generic_kernel<<<dim3(rows, (a.N_c + kIdxKeys - 1) / kIdxKeys), kIdxKeys, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// Top-k selector ("DeepSeek-v4 Beyond Basics" 3.2.2 eq. 17; "Phase 1
+// Module 1" "Top-k selects"): keep the k highest of the n_vis visible scores,
+// ties to the lower index; indices ascending, -1 padded.
+// One thread block per query row.  A 4-pass 8-bit radix select on the
+// order-preserving uint32 image of the scores finds the k-th largest key T
+// and how many of the entries equal to T are needed; entries above T are
+// appended in any order, the needed ties are taken in index order (the scan
+// stops once it has enough), and each kept index is placed at its rank.
+// ===========================================================================
+constexpr int kTopkThreads = 1024;
+
+__device__ __forceinline__ int block_excl_count(bool flag, int* s_warp, int* total) {
+  // exclusive prefix count of flag over the block, in thread order
+  const unsigned int ballot = __ballot_sync(0xffffffffu, flag);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int in_warp = __popc(ballot & ((1u << lane) - 1u));
+  if (lane == 0) s_warp[warp] = __popc(ballot);
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int v = lane < nw ? s_warp[lane] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane < nw) s_warp[32 + lane] = incl - v;
+    if (lane == 31) s_warp[64] = incl;
+  }
+  __syncthreads();
+  const int r = s_warp[32 + warp] + in_warp;
+  *total = s_warp[64];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
+  extern __shared__ int tsm[];
+  int* cand = tsm;  // [k]
+  __shared__ unsigned int hist[256];
+  __shared__ int s_warp[65];
+  __shared__ unsigned int s_digit;
+  __shared__ int s_above;
+  __shared__ int s_cnt;
+
+  const int row = blockIdx.x;
+  const int k = a.k;
+  const int pos = a.q_pos[row];
+  const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
+  const float* sc = a.scores + (int64_t)row * a.N_c;
+  int32_t* out = a.idx_out + (int64_t)row * k;
+  float* so = a.score_out ? a.score_out + (int64_t)row * k : nullptr;
+  const int tid = threadIdx.x;
+
+  if (n_vis <= k) {
+    for (int i = tid; i < k; i += blockDim.x) {
+      out[i] = i < n_vis ? i : -1;
+      if (so) so[i] = i < n_vis ? sc[i] : -INFINITY;
+    }
+    return;
+  }
+  unsigned int prefix = 0, mask = 0;
+  int remaining = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n_vis; i += blockDim.x) {
+      const unsigned int u = f2key(sc[i]);
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l holds digits 255-8l .. 248-8l (descending)
+      int cnt[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { cnt[j] = (int)hist[255 - 8 * tid - j]; sum += cnt[j]; }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += n;
+      }
+      const int excl = incl - sum;
+      if (excl < remaining && incl >= remaining) {
+        int above = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (above + cnt[j] >= remaining) {
+            s_digit = 255u - 8u * tid - j;
+            s_above = above;
+            break;
+          }
+          above += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= s_digit << shift;
+    mask |= 255u << shift;
+    remaining -= s_above;
+    __syncthreads();
+  }
+  const unsigned int T = prefix;
+  const int need = remaining;  // ties (== T) to keep, >= 1
+  if (tid == 0) s_cnt = 0;
+  __syncthreads();
+  for (int i = tid; i < n_vis; i += blockDim.x) {
+    if (f2key(sc[i]) > T) cand[atomicAdd(&s_cnt, 1)] = i;
+  }
+  __syncthreads();
+  const int n_gt = k - need;
+  int taken = 0;
+  for (int base = 0; base < n_vis && taken < need; base += blockDim.x) {
+    const int i = base + tid;
+    const bool eq = i < n_vis && f2key(sc[i]) == T;
+    int tot;
+    const int r = block_excl_count(eq, s_warp, &tot);
+    if (eq && taken + r < need) cand[n_gt + taken + r] = i;
+    taken += tot;
+  }
+  __syncthreads();
+  // place each kept index at its rank (number of kept indices below it)
+  for (int j = tid; j < k; j += blockDim.x) {
+    const int v = cand[j];
+    int rank = 0;
+    for (int q = 0; q < k; ++q) rank += cand[q] < v;
+    out[rank] = v;
+    if (so) so[rank] = sc[v];
+  }
+}
+
+cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
+  const int rows = a.B * a.T_q;
+  if (rows <= 0) return cudaSuccess;
+  static unsigned long long attr_mask = 0;
+  set_smem_attr_once(topk_kernel, 64 * 1024, &attr_mask, 0);
+  TraceScope tr("topk", s);
+  topk_kernel<<<rows, kTopkThreads, (size_t)a.k * sizeof(int), s>>>(a);
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// Attention, CUDA-core form ("DeepSeek-v4 Beyond Basics" 3.2.2 eq. 19,
+// 3.3 eqs. 24-27; "DeepSeek V4 Inside" sink and window examples).
+// Thread block = (split, query, sequence).  The query's key list is the
+// selected (CSA) or visible (HCA) pool rows followed by the window rows;
+// split s takes a contiguous range of it.  q^ = RoPE_p(RMSNorm(q) * g) is
+// kept in shared memory as bf16 (the rounding the tensor-core form uses);
+// logits, the running max / sum and the output accumulator are float32.
+// With one split the block also finishes: divides by the sum plus
+// exp(sink), rotates the rope slice back by -p and stores bf16.  With
+// several, each writes (max, sum, accumulator) to the workspace and the
+// combine kernel finishes.
+// ===========================================================================
+constexpr int kAttThreads = 256;
+constexpr int kAttKT = 8;
+
+struct KeyList {
+  int n_sel, n_win, win_start;
+};
+
+__device__ __forceinline__ KeyList key_list(const AttendArgs& a, int b, int t, int pos,
+                                            const int32_t* idx_row) {
+  KeyList kl;
+  if (a.sparse) {
+    // idx rows are ascending with -1 padding at the end
+    int lo = 0, hi = a.k;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (idx_row[mid] >= 0) lo = mid + 1; else hi = mid;
+    }
+    kl.n_sel = lo;
+  } else {
+    kl.n_sel = min((pos + 1) / a.m, a.N_c);
+  }
+  kl.win_start = max(0, pos - a.W + 1);
+  kl.n_win = a.W > 0 ? pos - kl.win_start + 1 : 0;
+  return kl;
+}
+
+__device__ __forceinline__ const uint16_t* key_row(const AttendArgs& a, int b, const KeyList& kl,
+                                                   const int32_t* idx_row, int j, bool* ok) {
+  *ok = true;
+  if (j < kl.n_sel) {
+    int e = a.sparse ? idx_row[j] : j;
+    if (e >= a.N_c || e < 0) {
+      *ok = false;
+      return nullptr;
+    }
+    return a.pool + (int64_t)b * a.pool_bstride + (int64_t)e * a.D;
+  }
+  const int p = kl.win_start + (j - kl.n_sel);
+  return a.win + (int64_t)b * a.win_bstride + (int64_t)(p % a.win_cap) * a.D;
+}
+
+// q^ = RoPE_pos(RMSNorm(q_h) * g) for all heads into shared memory (bf16)
+__device__ void load_qhat(const AttendArgs& a, const uint16_t* qrow, int pos, uint16_t* qh,
+                          float* tmp) {
+  const int H = a.H, D = a.D, R = a.R;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int h = warp; h < H; h += nw) {
+    float ss = 0.f;
+    for (int d = lane; d < D; d += 32) {
+      const float x = bf2f(qrow[h * D + d]);
+      ss += x * x;
+    }
+    ss = warp_sum(ss);
+    const float rstd = rsqrtf(ss / (float)D + a.eps);
+    for (int d2 = lane; d2 < D / 2; d2 += 32) {
+      const int d = 2 * d2;
+      float x0 = bf2f(qrow[h * D + d]) * rstd * a.q_norm_g[d];
+      float x1 = bf2f(qrow[h * D + d + 1]) * rstd * a.q_norm_g[d + 1];
+      if (d >= D - R) {
+        float cs, sn;
+        rope_cos_sin(pos, (d - (D - R)) >> 1, R, a.rope_base, &cs, &sn);
+        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
+        x0 = y0;
+        x1 = y1;
+      }
+      qh[h * D + d] = f2bf(x0);
+      qh[h * D + d + 1] = f2bf(x1);
+    }
+  }
+  (void)tmp;
+}
+
+// normalise, de-rotate by -pos, store bf16: o[h][d] = acc[h][d] * inv[h]
+__device__ void finish_store(const AttendArgs& a, const float* acc, const float* inv, int pos,
+                             uint16_t* orow) {
+  const int H = a.H, D = a.D, R = a.R;
+  for (int e2 = threadIdx.x; e2 < H * D / 2; e2 += blockDim.x) {
+    const int h = (2 * e2) / D, d = (2 * e2) % D;
+    float x0 = acc[h * D + d] * inv[h];
+    float x1 = acc[h * D + d + 1] * inv[h];
+    if (d >= D - R) {
+      float cs, sn;
+      rope_cos_sin(pos, (d - (D - R)) >> 1, R, a.rope_base, &cs, &sn);
+      // rotation by -pos: (x cos + y sin, -x sin + y cos)
+      const float y0 = x0 * cs + x1 * sn, y1 = -x0 * sn + x1 * cs;
+      x0 = y0;
+      x1 = y1;
+    }
+    *reinterpret_cast<unsigned int*>(orow + h * D + d) = f2_to_bf2x2(x0, x1);
+  }
+}
+
+__global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs a) {
+  extern __shared__ __align__(16) unsigned char asm_raw[];
+  const int H = a.H, D = a.D;
+  float* acc = reinterpret_cast<float*>(asm_raw);          // [H*D]
+  float* kv = acc + H * D;                                  // [KT*D]
+  float* lg = kv + kAttKT * D;                              // [H*KT]
+  float* mrow = lg + H * kAttKT;                            // [H]
+  float* lrow = mrow + H;                                   // [H]
+  float* alpha = lrow + H;                                  // [H]
+  uint16_t* qh = reinterpret_cast<uint16_t*>(alpha + H);    // [H*D]
+
+  const int split = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
+  const int row = b * a.T_q + t;
+  const int pos = a.q_pos[row];
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  if (pos < 0) {
+    if (tid == 0 && split == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
+    return;
+  }
+  const int32_t* idx_row = a.sparse ? a.idx + (int64_t)row * a.k : nullptr;
+  const KeyList kl = key_list(a, b, t, pos, idx_row);
+  const int n_keys = kl.n_sel + kl.n_win;
+  const int per = (n_keys + a.n_splits - 1) / a.n_splits;
+  const int j0 = min(n_keys, split * per), j1 = min(n_keys, j0 + per);
+
+  load_qhat(a, a.q + (int64_t)row * H * D, pos, qh, nullptr);
+  for (int e = tid; e < H * D; e += blockDim.x) acc[e] = 0.f;
+  for (int h = tid; h < H; h += blockDim.x) { mrow[h] = -INFINITY; lrow[h] = 0.f; }
+  __syncthreads();
+
+  for (int jt = j0; jt < j1; jt += kAttKT) {
+    const int nk = min(kAttKT, j1 - jt);
+    // stage the K=V rows (rows that failed the bounds check become zeros
+    // with a -inf logit)
+    __shared__ int s_ok[kAttKT];
+    for (int jj = warp; jj < kAttKT; jj += nw) {
+      bool ok = false;
+      const uint16_t* src = jj < nk ? key_row(a, b, kl, idx_row, jt + jj, &ok) : nullptr;
+      if (jj < nk && !ok && lane == 0) raise_err(a.err, DS4A_DEV_BAD_INDEX);
+      for (int d = lane; d < D; d += 32) kv[jj * D + d] = (jj < nk && ok) ? bf2f(src[d]) : 0.f;
+      if (lane == 0) s_ok[jj] = (jj < nk && ok);
+    }
+    __syncthreads();
+    // logits: one warp per (head, key) pair
+    for (int pr = warp; pr < H * kAttKT; pr += nw) {
+      const int h = pr / kAttKT, jj = pr % kAttKT;
+      float dot = 0.f;
+      for (int d = lane; d < D; d += 32) dot = fmaf(bf2f(qh[h * D + d]), kv[jj * D + d], dot);
+      dot = warp_sum(dot);
+      if (lane == 0) lg[h * kAttKT + jj] = s_ok[jj] ? dot * a.scale : -INFINITY;
+    }
+    __syncthreads();
+    // online softmax
+    for (int h = tid; h < H; h += blockDim.x) {
+      float mx = mrow[h];
+      for (int jj = 0; jj < kAttKT; ++jj) mx = fmaxf(mx, lg[h * kAttKT + jj]);
+      const float al = (mrow[h] == -INFINITY) ? 0.f : __expf(mrow[h] - mx);
+      float ls = lrow[h] * al;
+      for (int jj = 0; jj < kAttKT; ++jj) {
+        const float z = lg[h * kAttKT + jj];
+        const float p = (z == -INFINITY) ? 0.f : __expf(z - mx);
+        lg[h * kAttKT + jj] = p;
+        ls += p;
+      }
+      mrow[h] = mx;
+      lrow[h] = ls;
+      alpha[h] = al;
+    }
+    __syncthreads();
+    for (int e = tid; e < H * D; e += blockDim.x) {
+      const int h = e / D, d = e % D;
+      float v = acc[e] * alpha[h];
+#pragma unroll
+      for (int jj = 0; jj < kAttKT; ++jj) v = fmaf(lg[h * kAttKT + jj], kv[jj * D + d], v);
+      acc[e] = v;
+    }
+    __syncthreads();
+  }
+
+  if (a.n_splits == 1) {
+    // finish: 1 / (sum + exp(sink - max)), de-rotate, store
+    for (int h = tid; h < H; h += blockDim.x) {
+      const float mx = mrow[h];
+      float den;
+      if (mx == -INFINITY) den = 0.f;  // no keys: output 0
+      else den = lrow[h] + __expf(a.sink[h] - mx);
+      alpha[h] = den > 0.f ? 1.f / den : 0.f;
+    }
+    __syncthreads();
+    finish_store(a, acc, alpha, pos, a.out + (int64_t)row * H * D);
+    return;
+  }
+  float* part = a.ws + ((int64_t)row * a.n_splits + split) * (2 * H + H * D);
+  for (int h = tid; h < H; h += blockDim.x) { part[h] = mrow[h]; part[H + h] = lrow[h]; }
+  for (int e = tid; e < H * D; e += blockDim.x) part[2 * H + e] = acc[e];
+}
+
+__global__ void __launch_bounds__(kAttThreads) attend_combine_kernel(AttendArgs a) {
+  extern __shared__ __align__(16) unsigned char cm_raw[];
+  const int H = a.H, D = a.D, S = a.n_splits;
+  float* acc = reinterpret_cast<float*>(cm_raw);  // [H*D]
+  float* scl = acc + H * D;                        // [S*H]
+  float* inv = scl + S * H;                        // [H]
+  const int t = blockIdx.x, b = blockIdx.y;
+  const int row = b * a.T_q + t;
+  const int pos = a.q_pos[row];
+  if (pos < 0) return;
+  const float* base = a.ws + (int64_t)row * S * (2 * H + H * D);
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, base[s * (2 * H + H * D) + h]);
+    float L = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float ms = base[s * (2 * H + H * D) + h];
+      const float e = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+      scl[s * H + h] = e;
+      L += base[s * (2 * H + H * D) + H + h] * e;
+    }
+    inv[h] = (M == -INFINITY) ? 0.f : 1.f / (L + __expf(a.sink[h] - M));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < H * D; e += blockDim.x) {
+    const int h = e / D;
+    float v = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float f = scl[s * H + h];
+      if (f != 0.f) v = fmaf(base[s * (2 * H + H * D) + 2 * H + e], f, v);
+    }
+    acc[e] = v;
+  }
+  __syncthreads();
+  finish_store(a, acc, inv, pos, a.out + (int64_t)row * H * D);
+}
+
+int attend_splits(int B, int T_q, int keys_max, int H, int D, size_t ws_bytes, size_t* need) {
+  const int rows = B * T_q;
+  int want = 1;
+  if (rows > 0 && rows < 2 * 148) {
+    want = (2 * 148 + rows - 1) / rows;
+    const int by_keys = (keys_max + 63) / 64;
+    want = min(want, max(1, by_keys));
+    want = min(want, 64);
+  }
+  const size_t per = (size_t)rows * (2 * H + (size_t)H * D) * sizeof(float);
+  if (need) *need = want > 1 ? per * want : 0;
+  if (want > 1 && per > 0 && ws_bytes < per * want) {
+    want = (int)(ws_bytes / per);
+    if (want < 2) want = 1;
+  }
+  return want;
+}
+
+cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
+  const int rows = a.B * a.T_q;
+  if (rows <= 0) return cudaSuccess;
+  const size_t smem = (size_t)(a.H * a.D + kAttKT * a.D + a.H * kAttKT + 3 * a.H) * sizeof(float) +
+                      (size_t)a.H * a.D * sizeof(uint16_t);
+  static unsigned long long attr_mask = 0;
+  set_smem_attr_once(attend_generic_kernel, 227 * 1024, &attr_mask, 0);
+  {
+    TraceScope tr("attend_generic", s);
+    attend_generic_kernel<<<dim3(a.n_splits, a.T_q, a.B), kAttThreads, smem, s>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || a.n_splits == 1) return e;
+  return launch_attend_combine(a, s);
+}
+
+cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s) {
+  const size_t smem = (size_t)(a.H * a.D + a.n_splits * a.H + a.H) * sizeof(float);
+  static unsigned long long attr_mask = 0;
+  set_smem_attr_once(attend_combine_kernel, 227 * 1024, &attr_mask, 0);
+  TraceScope tr("attend_combine", s);
+  attend_combine_kernel<<<dim3(a.T_q, a.B), kAttThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ds4a

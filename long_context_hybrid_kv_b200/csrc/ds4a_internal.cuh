@@ -1,0 +1,155 @@
+// Internal declarations shared by the ds4a CUDA sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ds4a.h"
+
+namespace ds4a {
+
+// ---------------------------------------------------------------------------
+// device error word (one per device, per loaded library).  It is a
+// __device__ variable of ds4a_api.cu; kernels get its device address in
+// their argument struct (err_word() looks it up once per device).
+// ---------------------------------------------------------------------------
+unsigned int* err_word();
+
+__device__ __forceinline__ void raise_err(unsigned int* w, unsigned int bits) { atomicOr(w, bits); }
+
+// ---------------------------------------------------------------------------
+// bf16 helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf2f(uint16_t u) { return __uint_as_float(((unsigned int)u) << 16); }
+
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  // round-to-nearest-even (inputs here are finite)
+  unsigned int b = __float_as_uint(f);
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return (uint16_t)(b >> 16);
+}
+
+__device__ __forceinline__ float2 bf2x2_to_f2(unsigned int w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ unsigned int f2_to_bf2x2(float a, float b) {
+  return (unsigned int)f2bf(a) | ((unsigned int)f2bf(b) << 16);
+}
+
+// Rotation angle pos * base^(-2j/R), formed in float64 so that positions up
+// to 2^20 and beyond keep their phase (float32 would lose ~0.03 rad there).
+__device__ __forceinline__ void rope_cos_sin(int pos, int j, int rope_dim, float base, float* c,
+                                             float* s) {
+  double theta = exp2(-(2.0 * j / (double)rope_dim) * log2((double)base));
+  double ang = (double)pos * theta;
+  double sd, cd;
+  sincos(ang, &sd, &cd);
+  *c = (float)cd;
+  *s = (float)sd;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// order-preserving map float -> uint32 (larger float -> larger key)
+__device__ __forceinline__ unsigned int f2key(float f) {
+  unsigned int b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key2f(unsigned int k) {
+  unsigned int b = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(b);
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device (bit `which`
+// of the per-device words in `mask` records that it was done; up to 8
+// kernels share one mask array of 64 devices).
+template <typename F>
+inline void set_smem_attr_once(F* f, int bytes, unsigned long long* mask, int which) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 8) dev = 0;
+  const unsigned long long bit = 1ull << (dev * 8 + which);
+  if (!(*mask & bit)) {
+    cudaFuncSetAttribute(reinterpret_cast<const void*>(f), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         bytes);
+    *mask |= bit;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launch trace
+// ---------------------------------------------------------------------------
+struct TraceScope {
+  const char* name;
+  cudaStream_t stream;
+  int slot;
+  TraceScope(const char* n, cudaStream_t s);
+  ~TraceScope();
+};
+
+// ---------------------------------------------------------------------------
+// kernels (launchers return cudaError_t of the launch)
+// ---------------------------------------------------------------------------
+struct CompressArgs {
+  int B, T_tok, tok_begin, c, m, rope_dim;
+  float rope_base, eps;
+  const uint16_t *ca, *cb, *za, *zb;
+  const float *bias_a, *bias_b, *norm_g;
+  int entry_begin, entry_end;
+  uint16_t* pool;
+  int64_t pool_bstride;
+  unsigned int* err;
+};
+cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
+
+struct IndexArgs {
+  int B, T_q, H, D, m, k, N_c;
+  const int32_t* q_pos;
+  const uint16_t *q, *w, *kidx;
+  int64_t k_bstride;
+  float* scores;  // workspace [B*T_q, N_c]
+  int32_t* idx_out;
+  float* score_out;
+  unsigned int* err;
+};
+cudaError_t launch_index_scores_generic(const IndexArgs& a, cudaStream_t s);
+bool index_scores_tc_supported(const IndexArgs& a);
+cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s);
+cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s);
+
+struct AttendArgs {
+  int B, T_q, H, D, R, W, m, k, N_c, win_cap, sparse;
+  float scale, rope_base, eps;
+  const int32_t* q_pos;
+  const uint16_t* q;
+  const float* q_norm_g;
+  const uint16_t* pool;
+  int64_t pool_bstride;
+  const int32_t* idx;
+  const uint16_t* win;
+  int64_t win_bstride;
+  const float* sink;
+  uint16_t* out;
+  float* ws;  // split partials
+  int n_splits;
+  int keys_max;  // upper bound of keys per query
+  unsigned int* err;
+};
+int attend_splits(int B, int T_q, int keys_max, int H, int D, size_t ws_bytes, size_t* need);
+cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s);
+bool attend_tc_supported(const AttendArgs& a);
+cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t s);
+cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s);
+
+}  // namespace ds4a

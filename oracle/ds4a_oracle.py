@@ -46,6 +46,14 @@ import numpy as np
 # --------------------------------------------------------------------------
 # storage helpers
 # --------------------------------------------------------------------------
+def store_bf16(x) -> np.ndarray:
+    """The ABI stores compressed entries as bfloat16: round (via float32,
+    then round-to-nearest-even) and return the bit patterns (uint16).  Used
+    by the oracle's own chain when one step's stored output feeds the next."""
+    b = np.ascontiguousarray(np.asarray(x, dtype=np.float32)).view(np.uint32)
+    return ((b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
+
+
 def widen(x) -> np.ndarray:
     """bfloat16 bit patterns (uint16) or float32 -> float64."""
     x = np.asarray(x)

@@ -129,7 +129,7 @@ int ds4a_compress(const ds4a_layer_cfg* cfg, int B, int T_tok, int tok_begin, in
     if (check_cfg(cfg) != DS4A_OK) return DS4A_EINVAL;
     if (cfg->rope_dim > c) return DS4A_EINVAL;
   }
-  if (pool_bstride < (int64_t)entry_end * c || (pool_bstride % 8) != 0) return DS4A_EINVAL;
+  if (pool_bstride < (int64_t)entry_end * c || (pool_bstride % 2) != 0) return DS4A_EINVAL;
   const int m = cfg->ratio;
   // every token the entries read must be in the streams
   const int64_t first_tok = (overlap && entry_begin >= 1) ? (int64_t)(entry_begin - 1) * m

@@ -168,9 +168,10 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
   const int NC = a.c / V;
   const int G = NC >= kCompressThreads ? 1 : kCompressThreads / NC;
   const size_t smem = (size_t)(3 * G * a.c + a.c) * sizeof(float);
-  static unsigned long long attr_mask = 0;
-  set_smem_attr_once(compress_kernel<8>, 200 * 1024, &attr_mask, 0);
-  set_smem_attr_once(compress_kernel<2>, 200 * 1024, &attr_mask, 1);
+  static int cache8[16], cache2[16];
+  cudaError_t e = V == 8 ? ensure_smem(compress_kernel<8>, (int)smem, cache8)
+                         : ensure_smem(compress_kernel<2>, (int)smem, cache2);
+  if (e != cudaSuccess) return e;
   TraceScope tr("compress", s);
   if (V == 8)
     compress_kernel<8><<<dim3(n, a.B), kCompressThreads, smem, s>>>(a);
@@ -227,8 +228,9 @@ cudaError_t launch_index_scores_generic(const IndexArgs& a, cudaStream_t s) {
   const int rows = a.B * a.T_q;
   if (rows <= 0 || a.N_c <= 0) return cudaSuccess;
   const size_t smem = (size_t)(a.H * a.D + a.H + kIdxKeys * (a.D + 1)) * sizeof(float);
-  static unsigned long long attr_mask = 0;
-  set_smem_attr_once(index_score_generic_kernel, 200 * 1024, &attr_mask, 0);
+  static int cache[16];
+  cudaError_t e = ensure_smem(index_score_generic_kernel, (int)smem, cache);
+  if (e != cudaSuccess) return e;
   TraceScope tr("index_score_generic", s);
   index_score_generic_kernel<<<dim3(rows, (a.N_c + kIdxKeys - 1) / kIdxKeys), kIdxKeys, smem, s>>>(a);
   return cudaGetLastError();
@@ -371,8 +373,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
 cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
   const int rows = a.B * a.T_q;
   if (rows <= 0) return cudaSuccess;
-  static unsigned long long attr_mask = 0;
-  set_smem_attr_once(topk_kernel, 64 * 1024, &attr_mask, 0);
+  static int cache[16];
+  cudaError_t e = ensure_smem(topk_kernel, (int)((size_t)a.k * sizeof(int)), cache);
+  if (e != cudaSuccess) return e;
   TraceScope tr("topk", s);
   topk_kernel<<<rows, kTopkThreads, (size_t)a.k * sizeof(int), s>>>(a);
   return cudaGetLastError();
@@ -641,8 +644,9 @@ cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   const size_t smem = (size_t)(a.H * a.D + kAttKT * a.D + a.H * kAttKT + 3 * a.H) * sizeof(float) +
                       (size_t)a.H * a.D * sizeof(uint16_t);
-  static unsigned long long attr_mask = 0;
-  set_smem_attr_once(attend_generic_kernel, 227 * 1024, &attr_mask, 0);
+  static int cache[16];
+  cudaError_t e0 = ensure_smem(attend_generic_kernel, (int)smem, cache);
+  if (e0 != cudaSuccess) return e0;
   {
     TraceScope tr("attend_generic", s);
     attend_generic_kernel<<<dim3(a.n_splits, a.T_q, a.B), kAttThreads, smem, s>>>(a);
@@ -654,8 +658,9 @@ cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)(a.H * a.D + a.n_splits * a.H + a.H) * sizeof(float);
-  static unsigned long long attr_mask = 0;
-  set_smem_attr_once(attend_combine_kernel, 227 * 1024, &attr_mask, 0);
+  static int cache[16];
+  cudaError_t e = ensure_smem(attend_combine_kernel, (int)smem, cache);
+  if (e != cudaSuccess) return e;
   TraceScope tr("attend_combine", s);
   attend_combine_kernel<<<dim3(a.T_q, a.B), kAttThreads, smem, s>>>(a);
   return cudaGetLastError();

@@ -72,19 +72,23 @@ __device__ __forceinline__ float key2f(unsigned int k) {
   return __uint_as_float(b);
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device (bit `which`
-// of the per-device words in `mask` records that it was done; up to 8
-// kernels share one mask array of 64 devices).
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device when it is below that (cache[dev] holds the value set so far; up to
+// 16 devices).  Returns the error of cudaFuncSetAttribute, if any.
 template <typename F>
-inline void set_smem_attr_once(F* f, int bytes, unsigned long long* mask, int which) {
+inline cudaError_t ensure_smem(F* f, int bytes, int* cache) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 8) dev = 0;
-  const unsigned long long bit = 1ull << (dev * 8 + which);
-  if (!(*mask & bit)) {
-    cudaFuncSetAttribute(reinterpret_cast<const void*>(f), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         bytes);
-    *mask |= bit;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) dev = 0;
+  if (cache[dev] >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(f),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();  // do not leave it for a later launch check
+    return e;
   }
+  cache[dev] = bytes;
+  return cudaSuccess;
 }
 
 // ---------------------------------------------------------------------------

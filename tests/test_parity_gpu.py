@@ -132,7 +132,8 @@ def _check_index(qi, wi, ki, qpos, gidx, gsc, cfg_py, n_c, rows=None):
         assert msg is None, f"row {(b, t)}: {msg}"
         sel = gidx[b, t][gidx[b, t] >= 0]
         if sel.size:
-            err = np.max(np.abs(gsc[b, t, : sel.size] - rs[sel]) / (np.abs(rs[sel]) + 1e-3 * np.abs(rs).max()))
+            den = np.abs(rs[sel]) + max(1e-3 * np.abs(rs).max(), 1e-12)
+            err = np.max(np.abs(gsc[b, t, : sel.size] - rs[sel]) / den)
             assert err < 1e-4, f"row {(b, t)} score error {err}"
         assert np.all(np.isneginf(gsc[b, t, sel.size:]))
 

@@ -142,6 +142,32 @@ int ds4a_index_topk(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_
                     int64_t k_bstride, int N_c, int32_t* idx_out, float* score_out, void* ws,
                     size_t ws_bytes, ds4a_stream stream);
 
+/*
+ * ds4a_index_topk_noalloc -- ds4a_index_topk for callers that cannot
+ * allocate device memory (engines that reserve all HBM for their caches at
+ * start-up, C plugin hosts that pass no allocator, decode loops that must
+ * avoid cudaMalloc/cudaFree's implicit synchronisation).  The pages have no
+ * counterpart: it is an interface choice of this library.
+ *
+ * Same arguments and result as ds4a_index_topk without the workspace: the
+ * score scratch is a device array inside the library, 2^21 floats (8 MiB),
+ * held by every GPU that loads the library until the process exits.
+ *   - B * T_q * N_c above 2097152 returns DS4A_ENOSPACE (use
+ *     ds4a_index_topk with a workspace instead).
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array: calls whose kernels
+ *     overlap on the GPU (other streams, other host threads) race.  The
+ *     array keeps the last call's contents; a call reads only scores it has
+ *     written itself, so nothing needs clearing.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+int ds4a_index_topk_noalloc(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                            const ds4a_bf16* q_idx, const ds4a_bf16* w_idx,
+                            const ds4a_bf16* k_idx, int64_t k_bstride, int N_c,
+                            int32_t* idx_out, float* score_out, ds4a_stream stream);
+
 /* Bytes of workspace the attend calls can use for these sizes (split over
  * more thread blocks when few queries are given).  Passing less (even 0)
  * is allowed: the work is then split less. */

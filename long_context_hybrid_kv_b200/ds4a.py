@@ -14,7 +14,7 @@ import os
 __all__ = [
     "DS4A_OK", "DS4A_EINVAL", "DS4A_EUNSUPPORTED", "DS4A_ECUDA", "DS4A_EDEVICE", "DS4A_ETIMEOUT",
     "DS4A_ENOSPACE", "Ds4aError", "LayerCfg", "layer_cfg", "lib", "LIB_PATH", "ds4a_compress",
-    "ds4a_index_topk_workspace", "ds4a_index_topk", "ds4a_attend_workspace", "ds4a_sparse_attend",
+    "ds4a_index_topk_workspace", "ds4a_index_topk", "ds4a_index_topk_noalloc", "ds4a_attend_workspace", "ds4a_sparse_attend",
     "ds4a_hca_attend", "ds4a_check", "ds4a_strerror", "ds4a_trace_enable", "ds4a_trace_read",
     "ds4a_version",
 ]
@@ -58,6 +58,7 @@ _SIGS = {
     "ds4a_compress": (_I, [_CFG, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I64, _P]),
     "ds4a_index_topk_workspace": (_SZ, [_CFG, _I, _I, _I]),
     "ds4a_index_topk": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
+    "ds4a_index_topk_noalloc": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _P]),
     "ds4a_attend_workspace": (_SZ, [_CFG, _I, _I, _I, _I]),
     "ds4a_sparse_attend": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _I, _I64, _P, _P, _P, _SZ, _P]),
     "ds4a_hca_attend": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _I, _I64, _P, _P, _P, _SZ, _P]),
@@ -150,6 +151,19 @@ def ds4a_index_topk(cfg: LayerCfg, q_pos, q_idx, w_idx, k_idx, N_c: int, idx_out
                                _ptr(k_idx), 0 if k_idx is None else k_idx.stride(0), N_c,
                                _ptr(idx_out), _ptr(score_out), _ptr(ws), ws_bytes, _stream(stream))
     _ok(rc, "ds4a_index_topk")
+
+
+def ds4a_index_topk_noalloc(cfg: LayerCfg, q_pos, q_idx, w_idx, k_idx, N_c: int, idx_out, *,
+                            score_out=None, stream=None):
+    """ds4a_index_topk without a workspace argument: the library's own
+    fixed device scratch (up to 2**21 scores) serves every call, for
+    callers that cannot allocate device memory."""
+    _bf16(q_idx, "q_idx"), _bf16(w_idx, "w_idx")
+    B, T_q = q_pos.shape
+    rc = lib().ds4a_index_topk_noalloc(ctypes.byref(cfg), B, T_q, _ptr(q_pos), _ptr(q_idx), _ptr(w_idx),
+                                       _ptr(k_idx), 0 if k_idx is None else k_idx.stride(0), N_c,
+                                       _ptr(idx_out), _ptr(score_out), _stream(stream))
+    _ok(rc, "ds4a_index_topk_noalloc")
 
 
 def ds4a_attend_workspace(cfg: LayerCfg, B: int, T_q: int, N_c: int, sparse: bool) -> int:

@@ -192,8 +192,11 @@ int ds4a_index_topk(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_
 size_t ds4a_attend_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c, int sparse) {
   if (check_cfg(cfg) != DS4A_OK || B <= 0 || T_q <= 0) return 0;
   const int keys_max = (sparse ? cfg->topk : (N_c > 0 ? N_c : 0)) + cfg->window;
+  AttendArgs probe{};
+  probe.H = cfg->n_heads; probe.D = cfg->head_dim; probe.R = cfg->rope_dim;
   size_t need = 0;
-  attend_splits(B, T_q, keys_max, cfg->n_heads, cfg->head_dim, (size_t)-1, &need);
+  attend_splits(B, T_q, keys_max, cfg->n_heads, cfg->head_dim, attend_tc_supported(probe), (size_t)-1,
+                &need);
   return need;
 }
 
@@ -231,10 +234,10 @@ static int attend_common(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_
   a.keys_max = (sparse ? cfg->topk : N_c) + cfg->window;
   a.err = err_word();
   if (!a.err) return DS4A_ECUDA;
-  a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, ws ? ws_bytes : 0, nullptr);
+  const bool tc = attend_tc_supported(a);
+  a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, tc, ws ? ws_bytes : 0, nullptr);
   cudaStream_t s = (cudaStream_t)stream;
-  if (attend_tc_supported(a)) return cuda_rc(launch_attend_tc(a, s));
-  return cuda_rc(launch_attend_generic(a, s));
+  return cuda_rc(tc ? launch_attend_tc(a, s) : launch_attend_generic(a, s));
 }
 
 int ds4a_sparse_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,

@@ -14,11 +14,12 @@ namespace ds4a {
 // eqs. 20-23): per channel, a softmax over the 2m (CSA) or m (HCA) logits
 // Z + B weights the matching C values; then RMSNorm * g and RoPE at i*m.
 // One thread block per (entry, sequence).  Thread t owns channels
-// [8*(t % NC), 8*(t % NC) + 8) (NC = c/8) and the terms g, g+G, ... of the
-// entry (g = t / NC, G = 256 / NC); the G partial softmaxes merge in shared
-// memory.  Loads are 16-byte vectors of 8 bf16.
+// [V*(t % NC), V*(t % NC) + V) (NC = c/V) and the terms g, g+G, ... of the
+// entry (g = t / NC, G = 512 / NC), four terms' loads in flight at a time;
+// the G partial softmaxes merge in shared memory.  Loads are 16-byte
+// vectors of 8 bf16 when c is a multiple of 8.
 // ===========================================================================
-constexpr int kCompressThreads = 256;
+constexpr int kCompressThreads = 512;
 
 template <int V>
 struct VecLoad;
@@ -74,27 +75,37 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
   for (int u = 0; u < V; ++u) { mx[u] = -INFINITY; l[u] = 0.f; acc[u] = 0.f; }
 
   if (g < G) {
-    for (int term = g; term < n_terms; term += G) {
-      const bool half_a = term < m;
-      const int r = half_a ? term : term - m;
-      const int tok = half_a ? i * m + r : (i - 1) * m + r;
-      const int64_t row = (int64_t)b * a.T_tok + (tok - a.tok_begin);
-      float vals[V], zs[V], bs[V];
-      VecLoad<V>::load((half_a ? a.ca : a.cb) + row * c + cc * V, vals);
-      VecLoad<V>::load((half_a ? a.za : a.zb) + row * c + cc * V, zs);
-      VecLoad<V>::load_f((half_a ? a.bias_a : a.bias_b) + (int64_t)r * c + cc * V, bs);
+    for (int t0 = g; t0 < n_terms; t0 += 4 * G) {
+      float vals[4][V], zs[4][V], bs[4][V];
 #pragma unroll
-      for (int q = 0; q < V; ++q) {
-        const float x = zs[q] + bs[q];
-        if (x > mx[q]) {
-          const float sc = __expf(mx[q] - x);
-          l[q] = l[q] * sc + 1.f;
-          acc[q] = acc[q] * sc + vals[q];
-          mx[q] = x;
-        } else {
-          const float e = __expf(x - mx[q]);
-          l[q] += e;
-          acc[q] += e * vals[q];
+      for (int u = 0; u < 4; ++u) {
+        const int term = t0 + u * G;
+        if (term < n_terms) {
+          const bool half_a = term < m;
+          const int r = half_a ? term : term - m;
+          const int tok = half_a ? i * m + r : (i - 1) * m + r;
+          const int64_t row = (int64_t)b * a.T_tok + (tok - a.tok_begin);
+          VecLoad<V>::load((half_a ? a.ca : a.cb) + row * c + cc * V, vals[u]);
+          VecLoad<V>::load((half_a ? a.za : a.zb) + row * c + cc * V, zs[u]);
+          VecLoad<V>::load_f((half_a ? a.bias_a : a.bias_b) + (int64_t)r * c + cc * V, bs[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (t0 + u * G >= n_terms) break;
+#pragma unroll
+        for (int q = 0; q < V; ++q) {
+          const float x = zs[u][q] + bs[u][q];
+          if (x > mx[q]) {
+            const float sc = __expf(mx[q] - x);
+            l[q] = l[q] * sc + 1.f;
+            acc[q] = acc[q] * sc + vals[u][q];
+            mx[q] = x;
+          } else {
+            const float e = __expf(x - mx[q]);
+            l[q] += e;
+            acc[q] += e * vals[u][q];
+          }
         }
       }
     }
@@ -274,9 +285,16 @@ __device__ __forceinline__ int block_excl_count(bool flag, int* s_warp, int* tot
   return r;
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
-  extern __shared__ int tsm[];
-  int* cand = tsm;  // [k]
+// kSmemKeys: the row's order-preserving keys are staged in shared memory
+// once (rows of up to kTopkSmemKeys entries); otherwise every pass reads
+// the scores from global memory (L2).
+constexpr int kTopkSmemKeys = 12288;
+
+template <int kThreadsT, bool kSmemKeys>
+__global__ void __launch_bounds__(kThreadsT) topk_kernel(IndexArgs a) {
+  extern __shared__ unsigned int tsm[];
+  int* cand = reinterpret_cast<int*>(tsm);            // [k]
+  unsigned int* keys = tsm + ((a.k + 3) & ~3);         // [n_vis] (kSmemKeys)
   __shared__ unsigned int hist[256];
   __shared__ int s_warp[65];
   __shared__ unsigned int s_digit;
@@ -291,6 +309,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
   int32_t* out = a.idx_out + (int64_t)row * k;
   float* so = a.score_out ? a.score_out + (int64_t)row * k : nullptr;
   const int tid = threadIdx.x;
+  if (pos < 0 && tid == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
 
   if (n_vis <= k) {
     for (int i = tid; i < k; i += blockDim.x) {
@@ -299,6 +318,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
     }
     return;
   }
+  if (kSmemKeys) {
+    for (int i = tid; i < n_vis; i += blockDim.x) keys[i] = f2key(sc[i]);
+    __syncthreads();
+  }
+  auto key_at = [&](int i) -> unsigned int { return kSmemKeys ? keys[i] : f2key(sc[i]); };
   unsigned int prefix = 0, mask = 0;
   int remaining = k;
   for (int pass = 0; pass < 4; ++pass) {
@@ -306,7 +330,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
     for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     for (int i = tid; i < n_vis; i += blockDim.x) {
-      const unsigned int u = f2key(sc[i]);
+      const unsigned int u = key_at(i);
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
     }
     __syncthreads();
@@ -346,14 +370,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
   if (tid == 0) s_cnt = 0;
   __syncthreads();
   for (int i = tid; i < n_vis; i += blockDim.x) {
-    if (f2key(sc[i]) > T) cand[atomicAdd(&s_cnt, 1)] = i;
+    if (key_at(i) > T) cand[atomicAdd(&s_cnt, 1)] = i;
   }
   __syncthreads();
   const int n_gt = k - need;
   int taken = 0;
   for (int base = 0; base < n_vis && taken < need; base += blockDim.x) {
     const int i = base + tid;
-    const bool eq = i < n_vis && f2key(sc[i]) == T;
+    const bool eq = i < n_vis && key_at(i) == T;
     int tot;
     const int r = block_excl_count(eq, s_warp, &tot);
     if (eq && taken + r < need) cand[n_gt + taken + r] = i;
@@ -373,11 +397,21 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
 cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
   const int rows = a.B * a.T_q;
   if (rows <= 0) return cudaSuccess;
+  const size_t cand_bytes = (size_t)((a.k + 3) & ~3) * sizeof(int);
+  if (a.N_c <= kTopkSmemKeys) {
+    const size_t smem = cand_bytes + (size_t)a.N_c * sizeof(unsigned int);
+    static int cache[16];
+    cudaError_t e = ensure_smem(topk_kernel<512, true>, (int)smem, cache);
+    if (e != cudaSuccess) return e;
+    TraceScope tr("topk_smem", s);
+    topk_kernel<512, true><<<rows, 512, smem, s>>>(a);
+    return cudaGetLastError();
+  }
   static int cache[16];
-  cudaError_t e = ensure_smem(topk_kernel, (int)((size_t)a.k * sizeof(int)), cache);
+  cudaError_t e = ensure_smem(topk_kernel<kTopkThreads, false>, (int)cand_bytes, cache);
   if (e != cudaSuccess) return e;
   TraceScope tr("topk", s);
-  topk_kernel<<<rows, kTopkThreads, (size_t)a.k * sizeof(int), s>>>(a);
+  topk_kernel<kTopkThreads, false><<<rows, kTopkThreads, cand_bytes, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -435,9 +469,17 @@ __device__ __forceinline__ const uint16_t* key_row(const AttendArgs& a, int b, c
   return a.win + (int64_t)b * a.win_bstride + (int64_t)(p % a.win_cap) * a.D;
 }
 
+// cos / sin of the R/2 rope pairs at position pos (float64 phase) into rt
+__device__ void rope_table(const AttendArgs& a, int pos, float2* rt) {
+  for (int j = threadIdx.x; j < a.R / 2; j += blockDim.x) {
+    float cs, sn;
+    rope_cos_sin(pos, j, a.R, a.rope_base, &cs, &sn);
+    rt[j] = make_float2(cs, sn);
+  }
+}
+
 // q^ = RoPE_pos(RMSNorm(q_h) * g) for all heads into shared memory (bf16)
-__device__ void load_qhat(const AttendArgs& a, const uint16_t* qrow, int pos, uint16_t* qh,
-                          float* tmp) {
+__device__ void load_qhat(const AttendArgs& a, const uint16_t* qrow, const float2* rt, uint16_t* qh) {
   const int H = a.H, D = a.D, R = a.R;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int h = warp; h < H; h += nw) {
@@ -453,9 +495,8 @@ __device__ void load_qhat(const AttendArgs& a, const uint16_t* qrow, int pos, ui
       float x0 = bf2f(qrow[h * D + d]) * rstd * a.q_norm_g[d];
       float x1 = bf2f(qrow[h * D + d + 1]) * rstd * a.q_norm_g[d + 1];
       if (d >= D - R) {
-        float cs, sn;
-        rope_cos_sin(pos, (d - (D - R)) >> 1, R, a.rope_base, &cs, &sn);
-        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
+        const float2 r = rt[(d - (D - R)) >> 1];
+        const float y0 = x0 * r.x - x1 * r.y, y1 = x0 * r.y + x1 * r.x;
         x0 = y0;
         x1 = y1;
       }
@@ -463,22 +504,20 @@ __device__ void load_qhat(const AttendArgs& a, const uint16_t* qrow, int pos, ui
       qh[h * D + d + 1] = f2bf(x1);
     }
   }
-  (void)tmp;
 }
 
 // normalise, de-rotate by -pos, store bf16: o[h][d] = acc[h][d] * inv[h]
-__device__ void finish_store(const AttendArgs& a, const float* acc, const float* inv, int pos,
-                             uint16_t* orow) {
+__device__ void finish_store(const AttendArgs& a, const float* acc, const float* inv,
+                             const float2* rt, uint16_t* orow) {
   const int H = a.H, D = a.D, R = a.R;
   for (int e2 = threadIdx.x; e2 < H * D / 2; e2 += blockDim.x) {
     const int h = (2 * e2) / D, d = (2 * e2) % D;
     float x0 = acc[h * D + d] * inv[h];
     float x1 = acc[h * D + d + 1] * inv[h];
     if (d >= D - R) {
-      float cs, sn;
-      rope_cos_sin(pos, (d - (D - R)) >> 1, R, a.rope_base, &cs, &sn);
       // rotation by -pos: (x cos + y sin, -x sin + y cos)
-      const float y0 = x0 * cs + x1 * sn, y1 = -x0 * sn + x1 * cs;
+      const float2 r = rt[(d - (D - R)) >> 1];
+      const float y0 = x0 * r.x + x1 * r.y, y1 = -x0 * r.y + x1 * r.x;
       x0 = y0;
       x1 = y1;
     }
@@ -495,7 +534,9 @@ __global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs 
   float* mrow = lg + H * kAttKT;                            // [H]
   float* lrow = mrow + H;                                   // [H]
   float* alpha = lrow + H;                                  // [H]
-  uint16_t* qh = reinterpret_cast<uint16_t*>(alpha + H);    // [H*D]
+  // [R/2] pairs; (H*D + KT*D + H*KT) is even, so rounding 3H up keeps 8 B
+  float2* rt = reinterpret_cast<float2*>(mrow + ((3 * H + 1) & ~1));
+  uint16_t* qh = reinterpret_cast<uint16_t*>(rt + a.R / 2 + 1);  // [H*D]
 
   const int split = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
   const int row = b * a.T_q + t;
@@ -512,7 +553,9 @@ __global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs 
   const int per = (n_keys + a.n_splits - 1) / a.n_splits;
   const int j0 = min(n_keys, split * per), j1 = min(n_keys, j0 + per);
 
-  load_qhat(a, a.q + (int64_t)row * H * D, pos, qh, nullptr);
+  rope_table(a, pos, rt);
+  __syncthreads();
+  load_qhat(a, a.q + (int64_t)row * H * D, rt, qh);
   for (int e = tid; e < H * D; e += blockDim.x) acc[e] = 0.f;
   for (int h = tid; h < H; h += blockDim.x) { mrow[h] = -INFINITY; lrow[h] = 0.f; }
   __syncthreads();
@@ -576,7 +619,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs 
       alpha[h] = den > 0.f ? 1.f / den : 0.f;
     }
     __syncthreads();
-    finish_store(a, acc, alpha, pos, a.out + (int64_t)row * H * D);
+    finish_store(a, acc, alpha, rt, a.out + (int64_t)row * H * D);
     return;
   }
   float* part = a.ws + ((int64_t)row * a.n_splits + split) * (2 * H + H * D);
@@ -584,47 +627,72 @@ __global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs 
   for (int e = tid; e < H * D; e += blockDim.x) part[2 * H + e] = acc[e];
 }
 
+// Merge of the key splits of one query: per head, M = max of the split
+// maxima, L = sum of l_s exp(m_s - M), o = sum acc_s exp(m_s - M) / (L +
+// exp(sink - M)); then the rope slice rotates back by -pos.  Thread block =
+// 8 heads of one query.
+constexpr int kCombHeads = 8;
+
 __global__ void __launch_bounds__(kAttThreads) attend_combine_kernel(AttendArgs a) {
   extern __shared__ __align__(16) unsigned char cm_raw[];
-  const int H = a.H, D = a.D, S = a.n_splits;
-  float* acc = reinterpret_cast<float*>(cm_raw);  // [H*D]
-  float* scl = acc + H * D;                        // [S*H]
-  float* inv = scl + S * H;                        // [H]
-  const int t = blockIdx.x, b = blockIdx.y;
+  const int H = a.H, D = a.D, S = a.n_splits, R = a.R;
+  float2* rt = reinterpret_cast<float2*>(cm_raw);          // [R/2]
+  float* scl = reinterpret_cast<float*>(rt + R / 2 + 1);    // [S * 8]
+  float* inv = scl + S * kCombHeads;                        // [8]
+  const int h0 = blockIdx.x * kCombHeads;
+  const int t = blockIdx.y, b = blockIdx.z;
   const int row = b * a.T_q + t;
   const int pos = a.q_pos[row];
   if (pos < 0) return;
-  const float* base = a.ws + (int64_t)row * S * (2 * H + H * D);
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+  const int64_t stride = 2 * H + (int64_t)H * D;
+  const float* base = a.ws + (int64_t)row * S * stride;
+  const int nh = min(kCombHeads, H - h0);
+  const int tid = threadIdx.x;
+  if (tid < nh) {
+    const int h = h0 + tid;
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, base[s * (2 * H + H * D) + h]);
+    for (int s = 0; s < S; ++s) M = fmaxf(M, base[s * stride + h]);
     float L = 0.f;
     for (int s = 0; s < S; ++s) {
-      const float ms = base[s * (2 * H + H * D) + h];
+      const float ms = base[s * stride + h];
       const float e = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-      scl[s * H + h] = e;
-      L += base[s * (2 * H + H * D) + H + h] * e;
+      scl[s * kCombHeads + tid] = e;
+      L += base[s * stride + H + h] * e;
     }
-    inv[h] = (M == -INFINITY) ? 0.f : 1.f / (L + __expf(a.sink[h] - M));
+    inv[tid] = (M == -INFINITY) ? 0.f : 1.f / (L + __expf(a.sink[h] - M));
   }
+  rope_table(a, pos, rt);
   __syncthreads();
-  for (int e = threadIdx.x; e < H * D; e += blockDim.x) {
-    const int h = e / D;
-    float v = 0.f;
+  uint16_t* orow = a.out + (int64_t)row * H * D;
+  for (int e2 = tid; e2 < nh * D / 2; e2 += blockDim.x) {
+    const int hl = (2 * e2) / D, d = (2 * e2) % D, h = h0 + hl;
+    float x0 = 0.f, x1 = 0.f;
     for (int s = 0; s < S; ++s) {
-      const float f = scl[s * H + h];
-      if (f != 0.f) v = fmaf(base[s * (2 * H + H * D) + 2 * H + e], f, v);
+      const float f = scl[s * kCombHeads + hl];
+      if (f == 0.f) continue;
+      const float2 v = *reinterpret_cast<const float2*>(base + s * stride + 2 * H + (int64_t)h * D + d);
+      x0 = fmaf(v.x, f, x0);
+      x1 = fmaf(v.y, f, x1);
     }
-    acc[e] = v;
+    x0 *= inv[hl];
+    x1 *= inv[hl];
+    if (d >= D - R) {
+      const float2 r = rt[(d - (D - R)) >> 1];
+      const float y0 = x0 * r.x + x1 * r.y, y1 = -x0 * r.y + x1 * r.x;
+      x0 = y0;
+      x1 = y1;
+    }
+    *reinterpret_cast<unsigned int*>(orow + (int64_t)h * D + d) = f2_to_bf2x2(x0, x1);
   }
-  __syncthreads();
-  finish_store(a, acc, inv, pos, a.out + (int64_t)row * H * D);
 }
 
-int attend_splits(int B, int T_q, int keys_max, int H, int D, size_t ws_bytes, size_t* need) {
+int attend_splits(int B, int T_q, int keys_max, int H, int D, bool tc, size_t ws_bytes,
+                  size_t* need) {
   const int rows = B * T_q;
   int want = 1;
-  if (rows > 0 && rows < 2 * 148) {
+  if (tc) {
+    want = attend_tc_splits(B, T_q, keys_max);
+  } else if (rows > 0 && rows < 2 * 148) {
     want = (2 * 148 + rows - 1) / rows;
     const int by_keys = (keys_max + 63) / 64;
     want = min(want, max(1, by_keys));
@@ -642,8 +710,8 @@ int attend_splits(int B, int T_q, int keys_max, int H, int D, size_t ws_bytes, s
 cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
   const int rows = a.B * a.T_q;
   if (rows <= 0) return cudaSuccess;
-  const size_t smem = (size_t)(a.H * a.D + kAttKT * a.D + a.H * kAttKT + 3 * a.H) * sizeof(float) +
-                      (size_t)a.H * a.D * sizeof(uint16_t);
+  const size_t smem = (size_t)(a.H * a.D + kAttKT * a.D + a.H * kAttKT + ((3 * a.H + 1) & ~1)) * sizeof(float) +
+                      (size_t)(a.R / 2 + 1) * sizeof(float2) + (size_t)a.H * a.D * sizeof(uint16_t);
   static int cache[16];
   cudaError_t e0 = ensure_smem(attend_generic_kernel, (int)smem, cache);
   if (e0 != cudaSuccess) return e0;
@@ -657,12 +725,13 @@ cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)(a.H * a.D + a.n_splits * a.H + a.H) * sizeof(float);
+  const size_t smem = (size_t)(a.R / 2 + 1) * sizeof(float2) +
+                      (size_t)(a.n_splits * kCombHeads + kCombHeads) * sizeof(float);
   static int cache[16];
   cudaError_t e = ensure_smem(attend_combine_kernel, (int)smem, cache);
   if (e != cudaSuccess) return e;
   TraceScope tr("attend_combine", s);
-  attend_combine_kernel<<<dim3(a.T_q, a.B), kAttThreads, smem, s>>>(a);
+  attend_combine_kernel<<<dim3((a.H + kCombHeads - 1) / kCombHeads, a.T_q, a.B), kAttThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,333 @@
-// Tensor-core (tcgen05) indexer score for the Flash shape (H_I = 64,
-// D_I = 128).
-#include "ds4a_internal.cuh"
+// Tensor-core (tcgen05) Lightning-Indexer score for the Flash shape
+// (64 indexer heads x 128): "DeepSeek-v4 Beyond Basics" 3.2.2 eq. 16,
+//   I[t][s] = sum_h w[t][h] * ReLU(q[t][h] . K[s]).
+// Per tile of 128 keys and a group of G queries of one sequence (G = 4 when
+// the sequence has several queries, else 1) one product
+//   D[key][g*64 + h] = K[key][:] . q[g][h][:]      (M = 128, N = 64 G, K = 128)
+// lands in tensor memory; the epilogue thread that owns a key row applies
+// the ReLU and the head weights in registers and writes the G scores.
+//
+// Thread block (192 threads, one per SM):
+//   warp 0     lane 0 streams K tiles with TMA (3-D map [B][N_c][128],
+//              128-byte swizzle, two 64-dim boxes per tile) into 4 stages,
+//              and the group's queries (2-D map over [B*T_q*64][128]);
+//   warp 1     TMEM allocation; lane 0 issues the MMAs (8 x K=16 per tile)
+//              into two accumulator buffers;
+//   warps 2-5  epilogue (they cover the four TMEM lane quarters).
+// Work: (query group, chunk of key tiles) pairs, taken round-robin by the
+// blocks; pairs past a group's visible entries are skipped.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "ds4a_tc.cuh"
 
 namespace ds4a {
-bool index_scores_tc_supported(const IndexArgs&) { return false; }
-cudaError_t launch_index_scores_tc(const IndexArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+using namespace tc;
+
+constexpr int kHI = 64;
+constexpr int kDI = 128;
+constexpr int kKT = 128;      // keys per tile
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kMaxG = 4;
+
+constexpr uint32_t kOffK = 0;                       // kStages x 2 blocks x 16 KB
+constexpr uint32_t kOffQ = kStages * 32768;         // 2 blocks x (G*64 rows x 128 B)
+constexpr uint32_t kOffW = kOffQ + 2 * kMaxG * 8192;  // [G*64] floats
+constexpr uint32_t kOffBar = kOffW + kMaxG * kHI * 4;
+constexpr uint32_t kOffMisc = kOffBar + 256;
+constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+
+enum Bar { kKFull = 0, kKEmpty = kKFull + kStages, kQFull = kKEmpty + kStages, kQEmpty, kAccFull0,
+           kAccFull1, kAccEmpty0, kAccEmpty1, kDrain, kNumBars };
+
+struct TcIndexParams {
+  IndexArgs a;
+  int G;               // queries per group
+  int groups_per_b;    // ceil(T_q / G)
+  int n_groups;
+  int chunk_tiles;     // key tiles per work pair
+  int chunks_per_group;
+  int n_pairs;
+};
+
+struct Pair {
+  int g, b, t0, nrows, tile0, tile1;  // tiles [tile0, tile1)
+  int n_vis[kMaxG];
+};
+
+__device__ __forceinline__ Pair make_pair(const TcIndexParams& p, int w) {
+  Pair q;
+  q.g = w / p.chunks_per_group;
+  const int chunk = w % p.chunks_per_group;
+  q.b = q.g / p.groups_per_b;
+  q.t0 = (q.g % p.groups_per_b) * p.G;
+  q.nrows = min(p.G, p.a.T_q - q.t0);
+  int vmax = 0;
+  for (int i = 0; i < kMaxG; ++i) {
+    int nv = 0;
+    if (i < q.nrows) {
+      const int pos = p.a.q_pos[q.b * p.a.T_q + q.t0 + i];
+      nv = pos < 0 ? 0 : min((pos + 1) / p.a.m, p.a.N_c);
+    }
+    q.n_vis[i] = nv;
+    vmax = max(vmax, nv);
+  }
+  const int tiles = (vmax + kKT - 1) / kKT;
+  q.tile0 = min(tiles, chunk * p.chunk_tiles);
+  q.tile1 = min(tiles, q.tile0 + p.chunk_tiles);
+  return q;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                    const TcIndexParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t k_base = sbase + kOffK, q_base = sbase + kOffQ;
+  float* w_s = reinterpret_cast<float*>(smem + kOffW);
+  const uint32_t bar0 = sbase + kOffBar;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc + 8);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = p.G;
+  const IndexArgs& a = p.a;
+  unsigned int* err = a.err;
+  const uint32_t q_bytes = (uint32_t)G * 64u * 256u;
+  const uint32_t q_blk = (uint32_t)G * 8192u;  // one 64-dim block of the group's queries
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kKFull + s), 1);
+      mbar_init(bar(kKEmpty + s), 1);
+    }
+    mbar_init(bar(kQFull), 1);
+    mbar_init(bar(kQEmpty), 1);
+    mbar_init(bar(kAccFull0), 1);
+    mbar_init(bar(kAccFull1), 1);
+    mbar_init(bar(kAccEmpty0), 128);
+    mbar_init(bar(kAccEmpty1), 128);
+    mbar_init(bar(kDrain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // =================== TMA producer ===================
+    if (lane == 0) {
+      uint32_t kt = 0, active = 0;
+      for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
+        const Pair q = make_pair(p, w);
+        if (q.tile1 <= q.tile0) continue;
+        if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
+        mbar_expect_tx(bar(kQFull), q_bytes);
+        const int qrow = (q.b * a.T_q + q.t0) * kHI;
+        tma_load_2d(q_base, &qmap, 0, qrow, bar(kQFull));
+        tma_load_2d(q_base + q_blk, &qmap, 64, qrow, bar(kQFull));
+        for (int tile = q.tile0; tile < q.tile1; ++tile, ++kt) {
+          const uint32_t s = kt % kStages;
+          if (kt >= (uint32_t)kStages)
+            mbar_wait(bar(kKEmpty + s), ((kt / kStages) - 1) & 1u, abort_flag, err);
+          mbar_expect_tx(bar(kKFull + s), 32768u);
+          const uint32_t dst = k_base + s * 32768u;
+          tma_load_3d(dst, &kmap, 0, tile * kKT, q.b, bar(kKFull + s));
+          tma_load_3d(dst + 16384u, &kmap, 64, tile * kKT, q.b, bar(kKFull + s));
+        }
+        ++active;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // =================== MMA issuer ===================
+    if (lane == 0) {
+      uint32_t kt = 0, at = 0, active = 0;
+      const uint32_t idesc = idesc_bf16(128, 64 * G, 0, 0);
+      for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
+        const Pair q = make_pair(p, w);
+        if (q.tile1 <= q.tile0) continue;
+        mbar_wait(bar(kQFull), active & 1u, abort_flag, err);
+        tc_fence_after();
+        for (int tile = q.tile0; tile < q.tile1; ++tile, ++kt, ++at) {
+          const uint32_t s = kt % kStages;
+          const uint32_t ab = at & 1u;
+          mbar_wait(bar(kKFull + s), (kt / kStages) & 1u, abort_flag, err);
+          if (at >= 2) mbar_wait(bar(kAccEmpty0 + ab), ((at >> 1) - 1) & 1u, abort_flag, err);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t blk = (uint32_t)(kk >> 2);
+            const uint32_t koff = (uint32_t)(kk & 3) * 32u;
+            const uint64_t ad = sdesc_sw128(k_base + s * 32768u + blk * 16384u + koff, 16, 1024);
+            const uint64_t bd = sdesc_sw128(q_base + blk * q_blk + koff, 16, 1024);
+            mma_bf16(tmem + ab * 256u, ad, bd, idesc, kk != 0);
+          }
+          mma_commit(bar(kKEmpty + s));
+          mma_commit(bar(kAccFull0 + ab));
+        }
+        mma_commit(bar(kQEmpty));
+        ++active;
+      }
+      mma_commit(bar(kDrain));
+      mbar_wait(bar(kDrain), 0, abort_flag, err);
+    }
+    __syncwarp();
+  } else {
+    // =================== epilogue ===================
+    const int et = tid - 64;                 // 0..127
+    const int quarter = warp & 3;            // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;       // key row within the tile
+    const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    uint32_t at = 0;
+    for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
+      const Pair q = make_pair(p, w);
+      if (q.tile1 <= q.tile0) continue;
+      named_bar(1, 128);  // everyone is done with the previous pair's weights
+      for (int e = et; e < G * kHI; e += 128) {
+        const int g = e / kHI;
+        w_s[e] = g < q.nrows ? bf2f(a.w[((int64_t)q.b * a.T_q + q.t0 + g) * kHI + (e % kHI)]) : 0.f;
+      }
+      named_bar(1, 128);
+      for (int tile = q.tile0; tile < q.tile1; ++tile, ++at) {
+        const uint32_t ab = at & 1u;
+        mbar_wait(bar(kAccFull0 + ab), (at >> 1) & 1u, abort_flag, err);
+        tc_fence_after();
+        float sc[kMaxG];
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) {
+          sc[g] = 0.f;
+          if (g < G) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              float v[32];
+              tmem_ld32(t_lane + ab * 256u + (uint32_t)(g * 64 + half * 32), v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) sc[g] = fmaf(w_s[g * kHI + half * 32 + i], fmaxf(v[i], 0.f), sc[g]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(kAccEmpty0 + ab));
+        const int s = tile * kKT + r;
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < q.nrows && s < q.n_vis[g])
+            a.scores[((int64_t)q.b * a.T_q + q.t0 + g) * a.N_c + s] = sc[g];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    else
+      (void)cudaGetLastError();
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool index_scores_tc_supported(const IndexArgs& a) {
+  // Flash indexer width; the batch stride of the key pool must be a multiple
+  // of 16 bytes for the tensor map
+  return a.H == kHI && a.D == kDI && (a.k_bstride % 8) == 0 && a.N_c >= kKT && get_encode() != nullptr;
+}
+
+cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s) {
+  const int rows = a.B * a.T_q;
+  if (rows <= 0 || a.N_c <= 0) return cudaSuccess;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+  if (!encode) return cudaErrorNotSupported;
+  TcIndexParams p;
+  p.a = a;
+  p.G = a.T_q >= kMaxG ? kMaxG : 1;
+  p.groups_per_b = (a.T_q + p.G - 1) / p.G;
+  p.n_groups = a.B * p.groups_per_b;
+  const int max_tiles = (a.N_c + kKT - 1) / kKT;
+  // about four rounds of pairs over the SMs, whole groups when they are many
+  const long long want_pairs = 148ll * 4;
+  int chunk = (int)((p.n_groups * (long long)max_tiles + want_pairs - 1) / want_pairs);
+  chunk = max(1, min(chunk, max_tiles));
+  p.chunk_tiles = chunk;
+  p.chunks_per_group = (max_tiles + chunk - 1) / chunk;
+  p.n_pairs = p.n_groups * p.chunks_per_group;
+
+  CUtensorMap kmap, qmap;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)kDI, (cuuint64_t)a.N_c, (cuuint64_t)a.B};
+    const cuuint64_t strides[2] = {(cuuint64_t)kDI * 2, (cuuint64_t)a.k_bstride * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kKT, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (encode(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(a.kidx), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)rows * kHI};
+    const cuuint64_t strides[1] = {(cuuint64_t)kDI * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)(p.G * kHI)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.q), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  static int cache[16];
+  cudaError_t e = ensure_smem(index_tc_kernel, (int)kSmemBytes, cache);
+  if (e != cudaSuccess) return e;
+  const int grid = min(p.n_pairs, 148);
+  TraceScope tr("index_score_tc", s);
+  index_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, qmap, p);
+  return cudaGetLastError();
+}
+
 }  // namespace ds4a

@@ -150,7 +150,10 @@ struct AttendArgs {
   int keys_max;  // upper bound of keys per query
   unsigned int* err;
 };
-int attend_splits(int B, int T_q, int keys_max, int H, int D, size_t ws_bytes, size_t* need);
+// Key splits per query (and the workspace they need) for the path that
+// serves these sizes; fewer when ws_bytes cannot hold the partials.
+int attend_splits(int B, int T_q, int keys_max, int H, int D, bool tc, size_t ws_bytes, size_t* need);
+int attend_tc_splits(int B, int T_q, int keys_max);
 cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s);
 bool attend_tc_supported(const AttendArgs& a);
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t s);

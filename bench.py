@@ -348,7 +348,8 @@ def time_steps(step, K, W, stream, flush, graph=False, barrier=None):
 
 def kernel_times(state, K, stream, flush):
     """Average device time per launch of every library kernel (launch trace,
-    CUDA events on the launch stream) over K steps."""
+    CUDA events on the launch stream) over K steps, each queued whole behind
+    a spin kernel so that the events time the GPU, not the host."""
     import torch
     import long_context_hybrid_kv_b200 as L
 
@@ -358,6 +359,9 @@ def kernel_times(state, K, stream, flush):
     with torch.cuda.stream(stream):
         for _ in range(K):
             flush()
+            # a ~1 ms spin ahead of the step lets the host queue every launch
+            # before the GPU reaches them, so no launch waits on the host
+            torch.cuda._sleep(2_000_000)
             L.ds4a_trace_enable(True)
             state.step()
             recs = L.ds4a_trace_read()

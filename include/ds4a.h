@@ -168,9 +168,11 @@ int ds4a_index_topk_noalloc(const ds4a_layer_cfg* cfg, int B, int T_q, const int
                             const ds4a_bf16* k_idx, int64_t k_bstride, int N_c,
                             int32_t* idx_out, float* score_out, ds4a_stream stream);
 
-/* Bytes of workspace the attend calls can use for these sizes (split over
- * more thread blocks when few queries are given).  Passing less (even 0)
- * is allowed: the work is then split less. */
+/* Bytes of workspace the attend calls can use for these sizes.  On the
+ * tensor-core path (64 heads x 512) it holds one prepared query (64 KiB)
+ * per query plus the partial results of key splits (used when few queries
+ * are given).  Passing less is allowed: the work is then split less, and
+ * below B * T_q * 64 KiB the CUDA-core path runs instead. */
 size_t ds4a_attend_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c, int sparse);
 
 /*

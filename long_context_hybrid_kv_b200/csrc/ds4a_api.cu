@@ -10,6 +10,11 @@ namespace ds4a {
 
 __device__ unsigned int g_err_word = 0;
 
+void fill_rope_theta(RopeTheta* r, int rope_dim, float base) {
+  for (int j = 0; j < kMaxRopePairs; ++j)
+    r->t[j] = (2 * j < rope_dim) ? pow((double)base, -2.0 * j / (double)rope_dim) / M_PI : 0.0;
+}
+
 unsigned int* err_word() {
   static unsigned int* addr[64] = {nullptr};
   int dev = 0;
@@ -145,6 +150,7 @@ int ds4a_compress(const ds4a_layer_cfg* cfg, int B, int T_tok, int tok_begin, in
   a.bias_a = bias_a; a.bias_b = bias_b; a.norm_g = norm_g;
   a.entry_begin = entry_begin; a.entry_end = entry_end;
   a.pool = pool; a.pool_bstride = pool_bstride;
+  fill_rope_theta(&a.rope, a.rope_dim, cfg->rope_base);
   a.err = err_word();
   if (!a.err) return DS4A_ECUDA;
   return cuda_rc(launch_compress(a, (cudaStream_t)stream));
@@ -232,12 +238,17 @@ static int attend_common(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_
   a.idx = idx; a.win = win; a.win_bstride = win_bstride; a.sink = sink; a.out = out;
   a.ws = reinterpret_cast<float*>(ws);
   a.keys_max = (sparse ? cfg->topk : N_c) + cfg->window;
+  fill_rope_theta(&a.rope, a.R, cfg->rope_base);
   a.err = err_word();
   if (!a.err) return DS4A_ECUDA;
-  const bool tc = attend_tc_supported(a);
-  a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, tc, ws ? ws_bytes : 0, nullptr);
+  const size_t have = ws ? ws_bytes : 0;
   cudaStream_t s = (cudaStream_t)stream;
-  return cuda_rc(tc ? launch_attend_tc(a, s) : launch_attend_generic(a, s));
+  if (attend_tc_supported(a)) {
+    a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, true, have, nullptr);
+    if (a.n_splits > 0) return cuda_rc(launch_attend_tc(a, s));
+  }
+  a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, false, have, nullptr);
+  return cuda_rc(launch_attend_generic(a, s));
 }
 
 int ds4a_sparse_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,

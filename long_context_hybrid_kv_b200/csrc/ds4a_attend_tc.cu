@@ -11,16 +11,22 @@
 // tile is read once from HBM (gathered rows: pool[idx] then the window) and
 // serves both products.
 //
-// Thread block (one per SM, 288 threads):
-//   warps 0-3  softmax + epilogue: thread = key row of S^T (lane), later
-//              dim row of O^T; online softmax with a lazy rescale (O^T is
-//              rescaled only when a head's running max grows by more than
-//              2^8), P^T to shared memory as bf16, final normalisation with
-//              the sink, de-rotation of the rope slice by -pos, stores.
-//   warp 4     TMEM allocation; lane 0 issues every tcgen05.mma / commit.
-//   warps 5-8  producers: q^ = RoPE(RMSNorm(q) * g) into shared memory, then
-//              the KV rows by cp.async, one 128-dim chunk (32 KB) at a time,
-//              each chunk released by the PV products that read it.
+// Thread block (one per SM, 416 threads):
+//   warps 0-7  softmax + epilogue: two warps per TMEM lane quarter, each
+//              with 32 of the 64 head columns; thread = key row of S^T,
+//              later dim row of O^T; online softmax with a lazy rescale
+//              (O^T is rescaled only when a head's running max grows by
+//              more than 2^8), P^T to shared memory as bf16, final
+//              normalisation with the sink, de-rotation of the rope slice
+//              by -pos, staged 16-byte stores.
+//   warp 8     TMEM allocation; lane 0 issues every tcgen05.mma / commit.
+//   warps 9-12 producers: q^ as one 64 KB bulk copy of the image that
+//              qhat_prep_kernel wrote, then the KV rows by cp.async, one
+//              128-dim chunk (32 KB) at a time, each chunk released by the
+//              PV products that read it.
+// qhat_prep_kernel computes q^ = RoPE_pos(RMSNorm(q) * g) for every query
+// (one warp per head, coalesced) straight into that shared-memory image
+// (K-major, 128-byte swizzle, 64 KB per query) in the workspace.
 // Work items are (query, key split) pairs taken round-robin by the blocks;
 // with one split the block writes the final bf16 output, otherwise the
 // float partials (max, sum, accumulator) the combine kernel merges.
@@ -34,10 +40,9 @@ using namespace tc;
 constexpr int kH = 64;
 constexpr int kD = 512;
 constexpr int kKT = 128;              // keys per tile
-constexpr int kThreads = 288;
-constexpr int kSG = 0;                // softmax warps 0-3
-constexpr int kMmaWarp = 4;
-constexpr int kPG0 = 160;             // first producer thread
+constexpr int kThreads = 416;
+constexpr int kMmaWarp = 8;
+constexpr int kPG0 = 288;             // first producer thread (warps 9-12)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 
@@ -136,7 +141,8 @@ __device__ __forceinline__ const uint16_t* key_ptr(const AttendArgs& a, const It
   return a.win + (int64_t)it.b * a.win_bstride + (int64_t)(p % a.win_cap) * kD;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, int n_items) {
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, int n_items,
+                                                                const uint8_t* qimg) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -158,16 +164,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
 
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bar(kQFull), 128);
+    mbar_init(bar(kQFull), 1);
     mbar_init(bar(kQEmpty), 1);
     for (int c = 0; c < 4; ++c) {
       mbar_init(bar(kKVFull0 + c), 128);
       mbar_init(bar(kKVEmpty0 + c), 1);
     }
     mbar_init(bar(kSFull), 1);
-    mbar_init(bar(kPFull), 128);
+    mbar_init(bar(kPFull), 256);
     mbar_init(bar(kPVDone), 1);
-    mbar_init(bar(kEpiDone), 128);
+    mbar_init(bar(kEpiDone), 256);
     mbar_init(bar(kDrain), 1);
     fence_barrier_init();
   }
@@ -181,87 +187,81 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
   const uint32_t tmem = *tmem_slot;
   unsigned int* err = a.err;
 
-  if (warp < 4) {
-    // =================== softmax + epilogue ===================
-    const int r = tid;  // key row of S^T / dim row of O^T within a chunk
-    const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
+  if (warp < 8) {
+    // =================== softmax + epilogue (8 warps) ===================
+    // warp w reads TMEM lane quarter w % 4 (its 32 key rows of S^T, later
+    // 32 dim rows of O^T) and the 32 head columns of half w / 4
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int r = 32 * q4 + lane;  // key row of S^T / dim row of O^T within a chunk
+    const int st = tid;            // 0..255
+    const int h0 = 32 * hf;
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
     const float scale2 = a.scale * kLog2e;
     uint32_t gt = 0, active = 0;
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       const Item it = make_item(a, w);
       const bool final_out = a.n_splits == 1;
-      if (it.pos < 0 && r == 0 && it.split == 0) raise_err(err, DS4A_DEV_BAD_POS);
+      if (it.pos < 0 && st == 0 && it.split == 0) raise_err(err, DS4A_DEV_BAD_POS);
       if (it.n_tiles == 0) {
         // no keys in this item: output 0, or an empty partial
         if (final_out) {
           if (it.pos >= 0)
-            for (int e = r; e < kH * kD / 8; e += 128)
+            for (int e = st; e < kH * kD / 8; e += 256)
               reinterpret_cast<uint4*>(a.out + (int64_t)it.row * kH * kD)[e] = make_uint4(0, 0, 0, 0);
         } else {
           float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
-          if (r < kH) {
-            part[r] = -INFINITY;
-            part[kH + r] = 0.f;
+          if (st < kH) {
+            part[st] = -INFINITY;
+            part[kH + st] = 0.f;
           }
-          for (int e = r; e < kH * kD; e += 128) part[2 * kH + e] = 0.f;
+          for (int e = st; e < kH * kD; e += 256) part[2 * kH + e] = 0.f;
         }
         continue;
       }
-      if (r < kH) mrun[r] = -INFINITY;
-      float lpart[64];
+      if (st < kH) mrun[st] = -INFINITY;
+      float lpart[32];
 #pragma unroll
-      for (int h = 0; h < 64; ++h) lpart[h] = 0.f;
-      named_bar(1, 128);
+      for (int i = 0; i < 32; ++i) lpart[i] = 0.f;
+      named_bar(1, 256);
       for (int tile = 0; tile < it.n_tiles; ++tile, ++gt) {
         const uint32_t sb = gt & 1u;
-        mbar_wait(bar(kSFull), gt & 1u, abort_flag, err);
-        tc_fence_after();
-        float z[64];
-        {
-          float v[32];
-          tmem_ld32(t_lane + sb * 64u, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) z[i] = v[i];
-          tmem_ld32(t_lane + sb * 64u + 32u, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) z[32 + i] = v[i];
-        }
+        // validity of this thread's key (an index load) before the wait
         const int j = it.j0 + tile * kKT + r;
         bool bad = false;
         const bool valid = key_ptr(a, it, j, &bad) != nullptr;
+        mbar_wait(bar(kSFull), gt & 1u, abort_flag, err);
+        tc_fence_after();
+        float z[32];
+        tmem_ld32(t_lane + sb * 64u + (uint32_t)h0, z);
+        tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < 64; ++h) z[h] = valid ? z[h] * scale2 : -INFINITY;
-        float m0, m1;
-        warp_reduce64<true>(z, m0, m1);
-        red[warp * 64 + 2 * lane] = m0;
-        red[warp * 64 + 2 * lane + 1] = m1;
-        if (r == 0) *any_rescale = 0;
-        named_bar(1, 128);
-        if (r < kH) {
-          const float mt = fmaxf(fmaxf(red[r], red[64 + r]), fmaxf(red[128 + r], red[192 + r]));
-          const float mo = mrun[r];
+        for (int i = 0; i < 32; ++i) z[i] = valid ? z[i] * scale2 : -INFINITY;
+        red[q4 * 64 + h0 + lane] = warp_reduce32<true>(z);
+        if (st == 0) *any_rescale = 0;
+        named_bar(1, 256);
+        if (st < kH) {
+          const float mt = fmaxf(fmaxf(red[st], red[64 + st]), fmaxf(red[128 + st], red[192 + st]));
+          const float mo = mrun[st];
           float al = 1.f;
           if (mt > mo + kRescaleLog2 || (mo == -INFINITY && mt != -INFINITY)) {
             al = (mo == -INFINITY) ? 0.f : exp2f(mo - mt);
-            mrun[r] = mt;
+            mrun[st] = mt;
             *any_rescale = 1;
           }
-          alpha_s[r] = al;
+          alpha_s[st] = al;
         }
-        named_bar(1, 128);
-        uint32_t pk[32];
+        named_bar(1, 256);
+        uint32_t pk[16];
 #pragma unroll
-        for (int h = 0; h < 64; h += 2) {
-          const float ma = mrun[h], mb = mrun[h + 1];
-          const float pa = (z[h] == -INFINITY || ma == -INFINITY) ? 0.f : exp2f(z[h] - ma);
-          const float pb = (z[h + 1] == -INFINITY || mb == -INFINITY) ? 0.f : exp2f(z[h + 1] - mb);
+        for (int i = 0; i < 32; i += 2) {
+          const float ma = mrun[h0 + i], mb = mrun[h0 + i + 1];
+          const float pa = (z[i] == -INFINITY || ma == -INFINITY) ? 0.f : ex2_approx(z[i] - ma);
+          const float pb = (z[i + 1] == -INFINITY || mb == -INFINITY) ? 0.f : ex2_approx(z[i + 1] - mb);
           const uint32_t w2 = f2_to_bf2x2(pa, pb);
-          pk[h >> 1] = w2;
+          pk[i >> 1] = w2;
           const float2 pr = bf2x2_to_f2(w2);
-          lpart[h] = lpart[h] * alpha_s[h] + pr.x;
-          lpart[h + 1] = lpart[h + 1] * alpha_s[h + 1] + pr.y;
+          lpart[i] = lpart[i] * alpha_s[h0 + i] + pr.x;
+          lpart[i + 1] = lpart[i + 1] * alpha_s[h0 + i + 1] + pr.y;
         }
         if (tile > 0) {
           // the previous tile's PV must be done before P^T and O^T change
@@ -270,25 +270,23 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
           if (*any_rescale) {
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
-#pragma unroll 1
-              for (int half = 0; half < 2; ++half) {
-                float v[32];
-                const uint32_t addr = t_lane + 128u + 64u * c + 32u * half;
-                tmem_ld32(addr, v);
-                tmem_ld_wait();
+              float v[32];
+              const uint32_t addr = t_lane + 128u + 64u * c + (uint32_t)h0;
+              tmem_ld32(addr, v);
+              tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= alpha_s[32 * half + i];
-                tmem_st32(addr, v);
-              }
+              for (int i = 0; i < 32; ++i) v[i] *= alpha_s[h0 + i];
+              tmem_st32(addr, v);
             }
             tmem_st_wait();
           }
         }
-        // P^T row r: 64 heads as bf16 (128 B), 128-byte swizzled
+        // P^T row r, heads h0 .. h0+31: 64 B = chunks 4 hf .. 4 hf + 3 of the
+        // 128-byte swizzled row
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16)
-          st_shared16(p_base + sw128(r, c16), pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2],
-                      pk[4 * c16 + 3]);
+        for (int cc = 0; cc < 4; ++cc)
+          st_shared16(p_base + sw128(r, 4 * hf + cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
+                      pk[4 * cc + 3]);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(bar(kPFull));
@@ -296,57 +294,60 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
       // ---------------- epilogue ----------------
       mbar_wait(bar(kPVDone), (gt - 1) & 1u, abort_flag, err);
       tc_fence_after();
-      {
-        float s0, s1;
-        warp_reduce64<false>(lpart, s0, s1);
-        red[warp * 64 + 2 * lane] = s0;
-        red[warp * 64 + 2 * lane + 1] = s1;
-      }
-      named_bar(1, 128);
-      if (r < kH) {
-        const float l = red[r] + red[64 + r] + red[128 + r] + red[192 + r];
-        const float m = mrun[r];
+      red[q4 * 64 + h0 + lane] = warp_reduce32<false>(lpart);
+      named_bar(1, 256);
+      if (st < kH) {
+        const float l = red[st] + red[64 + st] + red[128 + st] + red[192 + st];
+        const float m = mrun[st];
         if (final_out) {
-          const float den = (m == -INFINITY) ? 0.f : l + exp2f(a.sink[r] * kLog2e - m);
-          inv_s[r] = den > 0.f ? 1.f / den : 0.f;
+          const float den = (m == -INFINITY) ? 0.f : l + exp2f(a.sink[st] * kLog2e - m);
+          inv_s[st] = den > 0.f ? 1.f / den : 0.f;
         } else {
           float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
-          part[r] = (m == -INFINITY) ? -INFINITY : m * 0.6931471805599453f;  // natural-log units
-          part[kH + r] = l;
+          part[st] = (m == -INFINITY) ? -INFINITY : m * 0.6931471805599453f;  // natural-log units
+          part[kH + st] = l;
         }
       }
-      named_bar(1, 128);
+      named_bar(1, 256);
       float cs = 1.f, sn = 0.f;
       const int R = a.R;
+      // the final output goes out through the idle P^T buffer: [64 heads]
+      // [128 dims] bf16 per chunk, then 16-byte stores of whole rows
+      uint16_t* stage = reinterpret_cast<uint16_t*>(smem + kOffP);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         const int d = 128 * c + r;
         const bool rot = final_out && d >= kD - R;
-        if (rot) rope_cos_sin(it.pos, (d - (kD - R)) >> 1, R, a.rope_base, &cs, &sn);
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float v[32];
-          tmem_ld32(t_lane + 128u + 64u * c + 32u * half, v);
-          tmem_ld_wait();
-          if (final_out) {
-            uint16_t* orow = a.out + (int64_t)it.row * kH * kD;
+        if (rot) rope_cos_sin(it.pos, a.rope.t[(d - (kD - R)) >> 1], &cs, &sn);
+        float v[32];
+        tmem_ld32(t_lane + 128u + 64u * c + (uint32_t)h0, v);
+        tmem_ld_wait();
+        if (final_out) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int h = 32 * half + i;
-              float x = v[i] * inv_s[h];
-              const float y = __shfl_xor_sync(0xffffffffu, x, 1);
-              if (rot) {
-                // rotation by -pos: even dim (x, y) -> x cos + y sin; odd
-                // dim (y, x) -> -y sin + x cos
-                x = (d & 1) ? (x * cs - y * sn) : (x * cs + y * sn);
-              }
-              orow[h * kD + d] = f2bf(x);
+          for (int i = 0; i < 32; ++i) {
+            const int h = h0 + i;
+            float x = v[i] * inv_s[h];
+            const float y = __shfl_xor_sync(0xffffffffu, x, 1);
+            if (rot) {
+              // rotation by -pos: even dim (x, y) -> x cos + y sin; odd
+              // dim (y, x) -> -y sin + x cos
+              x = (d & 1) ? (x * cs - y * sn) : (x * cs + y * sn);
             }
-          } else {
-            float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) part[2 * kH + (32 * half + i) * kD + d] = v[i];
+            stage[h * 128 + r] = f2bf(x);
           }
+          named_bar(1, 256);
+          uint16_t* orow = a.out + (int64_t)it.row * kH * kD + 128 * c;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int e = i * 256 + st;  // 16-byte piece: head e / 16, dims (e % 16) * 8 ..
+            const int h = e >> 4, q8 = (e & 15) * 8;
+            *reinterpret_cast<uint4*>(orow + h * kD + q8) = *reinterpret_cast<const uint4*>(stage + h * 128 + q8);
+          }
+          named_bar(1, 256);
+        } else {
+          float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) part[2 * kH + (h0 + i) * kD + d] = v[i];
         }
       }
       tc_fence_before();
@@ -405,101 +406,48 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
   } else {
     // =================== producers ===================
     const int pt = tid - kPG0;  // 0..127
-    const int pw = pt >> 5;     // producer warp 0..3
     uint32_t gt = 0, active = 0;
-    // RMSNorm gain of this lane's 16 dims
-    float g[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      g[i] = a.q_norm_g[8 * lane + i];
-      g[8 + i] = a.q_norm_g[256 + 8 * lane + i];
-    }
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       const Item it = make_item(a, w);
       if (it.n_tiles == 0) continue;
-      // ---- q^ = RoPE_pos(RMSNorm(q) * g) into the K-major swizzled tile ----
-      if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
-      float qc[4], qs[4];  // cos/sin of this lane's rope pairs (dims 256+8l ..)
-#pragma unroll
-      for (int pr = 0; pr < 4; ++pr) {
-        qc[pr] = 1.f;
-        qs[pr] = 0.f;
-        const int d = 256 + 8 * lane + 2 * pr;
-        if (d >= kD - a.R) rope_cos_sin(it.pos, (d - (kD - a.R)) >> 1, a.R, a.rope_base, &qc[pr], &qs[pr]);
-      }
-      const uint16_t* qrow = a.q + (int64_t)it.row * kH * kD;
-#pragma unroll 1
-      for (int h8 = 0; h8 < 16; h8 += 8) {
-        // issue the 16 loads of 8 heads before using any of them
-        uint4 va[8], vb[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int h = pw * 16 + h8 + u;
-          va[u] = *reinterpret_cast<const uint4*>(qrow + h * kD + 8 * lane);
-          vb[u] = *reinterpret_cast<const uint4*>(qrow + h * kD + 256 + 8 * lane);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int h = pw * 16 + h8 + u;
-          float x[16];
-          const unsigned int wa[4] = {va[u].x, va[u].y, va[u].z, va[u].w};
-          const unsigned int wb[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 fa = bf2x2_to_f2(wa[q]), fb = bf2x2_to_f2(wb[q]);
-            x[2 * q] = fa.x;
-            x[2 * q + 1] = fa.y;
-            x[8 + 2 * q] = fb.x;
-            x[8 + 2 * q + 1] = fb.y;
-          }
-          float ss = 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) ss += x[i] * x[i];
-          ss = warp_sum(ss);
-          const float rstd = rsqrtf(ss / (float)kD + a.eps);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) x[i] = x[i] * rstd * g[i];
-#pragma unroll
-          for (int pr = 0; pr < 4; ++pr) {
-            const float x0 = x[8 + 2 * pr], x1 = x[8 + 2 * pr + 1];
-            x[8 + 2 * pr] = x0 * qc[pr] - x1 * qs[pr];
-            x[8 + 2 * pr + 1] = x0 * qs[pr] + x1 * qc[pr];
-          }
-          // dims 8l..8l+7 -> block l/8, chunk l%8; dims 256+8l.. -> block 4+l/8
-          const uint32_t cA = q_base + (uint32_t)(lane >> 3) * 8192u + sw128(h, lane & 7);
-          const uint32_t cB = q_base + (uint32_t)(4 + (lane >> 3)) * 8192u + sw128(h, lane & 7);
-          st_shared16(cA, f2_to_bf2x2(x[0], x[1]), f2_to_bf2x2(x[2], x[3]), f2_to_bf2x2(x[4], x[5]),
-                      f2_to_bf2x2(x[6], x[7]));
-          st_shared16(cB, f2_to_bf2x2(x[8], x[9]), f2_to_bf2x2(x[10], x[11]),
-                      f2_to_bf2x2(x[12], x[13]), f2_to_bf2x2(x[14], x[15]));
-        }
-      }
-      fence_async_smem();
-      mbar_arrive(bar(kQFull));
-      // ---- K=V tiles ----
-      for (int tile = 0; tile < it.n_tiles; ++tile, ++gt) {
-        named_bar(2, 128);  // every producer is done with the previous row pointers
-        {
-          bool bad = false;
-          const uint16_t* p = key_ptr(a, it, it.j0 + tile * kKT + pt, &bad);
-          if (bad) raise_err(err, DS4A_DEV_BAD_INDEX);
-          rowptr[pt] = p;
-        }
+      const int piece = pt & 15;  // 16-byte piece of the 256-byte chunk row
+      // row pointers of a tile (every producer is done with the previous ones)
+      auto set_rowptr = [&](int tile) {
         named_bar(2, 128);
-        const int piece = pt & 15;  // 16-byte piece of the 256-byte chunk row
+        bool bad = false;
+        const uint16_t* p = key_ptr(a, it, it.j0 + tile * kKT + pt, &bad);
+        if (bad) raise_err(err, DS4A_DEV_BAD_INDEX);
+        rowptr[pt] = p;
+        named_bar(2, 128);
+      };
+      // one 128-dim chunk of the tile: 128 rows x 256 B, 16 cp.async each
+      auto issue_chunk = [&](int c) {
+        if (gt > 0) mbar_wait(bar(kKVEmpty0 + c), (gt - 1) & 1u, abort_flag, err);
+        const uint32_t blk = kv_base + (uint32_t)(2 * c + (piece >> 3)) * 16384u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int row = (pt >> 4) + 8 * i;
+          const uint16_t* src = rowptr[row];
+          const uint32_t dst = blk + sw128(row, piece & 7);
+          if (src) cp_async16(dst, src + c * 128 + piece * 8);
+          else st_shared_zero16(dst);
+        }
+        cp_async_commit();
+      };
+      // ---- q^ (prepared by qhat_prep_kernel in the shared-memory image
+      // layout): one 64 KB bulk copy once the previous item's QK is done ----
+      if (pt == 0) {
+        if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
+        mbar_expect_tx(bar(kQFull), 65536u);
+        bulk_g2s(q_base, qimg + (size_t)it.row * 65536u, 65536u, bar(kQFull));
+      }
+      // ---- K=V tiles: each chunk goes out when the PV products of the
+      // previous tile have released it ----
+      for (int tile = 0; tile < it.n_tiles; ++tile, ++gt) {
+        set_rowptr(tile);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          if (gt > 0) mbar_wait(bar(kKVEmpty0 + c), (gt - 1) & 1u, abort_flag, err);
-          const uint32_t blk = kv_base + (uint32_t)(2 * c + (piece >> 3)) * 16384u;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int row = (pt >> 4) + 8 * i;
-            const uint16_t* src = rowptr[row];
-            const uint32_t dst = blk + sw128(row, piece & 7);
-            if (src) cp_async16(dst, src + c * 128 + piece * 8);
-            else st_shared_zero16(dst);
-          }
-          cp_async_commit();
+          issue_chunk(c);
           if (c > 0) {
             cp_async_wait<1>();
             fence_async_smem();
@@ -519,6 +467,66 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// q^ = RoPE_pos(RMSNorm(q_h) * g) for every query, written as the
+// shared-memory image attend_tc_kernel copies in: 8 blocks of 64 dims, each
+// [64 heads][128 B] with the 128-byte swizzle.  Block = (query, 8 heads),
+// warp = head, lane = dims 8l..8l+7 and 256+8l..256+8l+7.
+__global__ void __launch_bounds__(256) qhat_prep_kernel(AttendArgs a, uint8_t* qimg) {
+  __shared__ float2 rt[64];
+  const int row = blockIdx.x;
+  const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int pos = a.q_pos[row];
+  const int R = a.R;
+  for (int j = threadIdx.x; j < R / 2; j += blockDim.x) {
+    float cs, sn;
+    rope_cos_sin(pos < 0 ? 0 : pos, a.rope.t[j], &cs, &sn);
+    rt[j] = make_float2(cs, sn);
+  }
+  __syncthreads();
+  const uint16_t* qrow = a.q + (int64_t)row * kH * kD + h * kD;
+  const uint4 va = *reinterpret_cast<const uint4*>(qrow + 8 * lane);
+  const uint4 vb = *reinterpret_cast<const uint4*>(qrow + 256 + 8 * lane);
+  float x[16];
+  const unsigned int wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 fa = bf2x2_to_f2(wa[q]), fb = bf2x2_to_f2(wb[q]);
+    x[2 * q] = fa.x;
+    x[2 * q + 1] = fa.y;
+    x[8 + 2 * q] = fb.x;
+    x[8 + 2 * q + 1] = fb.y;
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) ss += x[i] * x[i];
+  ss = warp_sum(ss);
+  const float rstd = rsqrtf(ss / (float)kD + a.eps);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int d = i < 8 ? 8 * lane + i : 256 + 8 * lane + (i - 8);
+    x[i] = x[i] * rstd * a.q_norm_g[d];
+  }
+#pragma unroll
+  for (int pr = 0; pr < 8; ++pr) {
+    const int i = 2 * pr;
+    const int d = i < 8 ? 8 * lane + i : 256 + 8 * lane + (i - 8);
+    if (d >= kD - R) {
+      const float2 t = rt[(d - (kD - R)) >> 1];
+      const float x0 = x[i], x1 = x[i + 1];
+      x[i] = x0 * t.x - x1 * t.y;
+      x[i + 1] = x0 * t.y + x1 * t.x;
+    }
+  }
+  uint8_t* img = qimg + (size_t)row * 65536u;
+  const uint32_t offA = (uint32_t)(lane >> 3) * 8192u + sw128(h, lane & 7);
+  const uint32_t offB = (uint32_t)(4 + (lane >> 3)) * 8192u + sw128(h, lane & 7);
+  *reinterpret_cast<uint4*>(img + offA) = make_uint4(f2_to_bf2x2(x[0], x[1]), f2_to_bf2x2(x[2], x[3]),
+                                                     f2_to_bf2x2(x[4], x[5]), f2_to_bf2x2(x[6], x[7]));
+  *reinterpret_cast<uint4*>(img + offB) = make_uint4(f2_to_bf2x2(x[8], x[9]), f2_to_bf2x2(x[10], x[11]),
+                                                     f2_to_bf2x2(x[12], x[13]), f2_to_bf2x2(x[14], x[15]));
 }
 
 }  // namespace
@@ -541,14 +549,23 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   AttendArgs a = a0;
   const int rows = a.B * a.T_q;
   if (rows <= 0) return cudaSuccess;
+  // workspace: [rows x 64 KB q^ images][split partials]
+  uint8_t* qimg = reinterpret_cast<uint8_t*>(a.ws);
+  a.ws = reinterpret_cast<float*>(qimg + (size_t)rows * 65536u);
   static int cache[16];
   cudaError_t e = ensure_smem(attend_tc_kernel, (int)kSmemBytes, cache);
+  if (e != cudaSuccess) return e;
+  {
+    TraceScope tr("qhat_prep", s);
+    qhat_prep_kernel<<<dim3(rows, kH / 8), 256, 0, s>>>(a, qimg);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n_items = rows * a.n_splits;
   const int grid = min(n_items, 148);
   {
     TraceScope tr("attend_tc", s);
-    attend_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a, n_items);
+    attend_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a, n_items, qimg);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess || a.n_splits == 1) return e;

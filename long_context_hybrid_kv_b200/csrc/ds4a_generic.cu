@@ -1,8 +1,9 @@
 // Shape-generic CUDA kernels of the ds4a path: the KV compressor, the
-// indexer score (CUDA-core form), the top-k selector, the split attention
-// (CUDA-core form) and its combine.  They serve every shape the ABI accepts
-// (the toy widths included); the Flash-0731 shapes take the tensor-core
-// kernels of ds4a_index_tc.cu / ds4a_attend_tc.cu where those apply.
+// indexer score (CUDA-core form), the split attention (CUDA-core form) and
+// its combine (the top-k selector is in ds4a_topk.cu).  They serve every
+// shape the ABI accepts (the toy widths included); the Flash-0731 shapes
+// take the tensor-core kernels of ds4a_index_tc.cu / ds4a_attend_tc.cu
+// where those apply.
 #include "ds4a_internal.cuh"
 
 #include <float.h>
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
     float x1 = s_v[ch + 1] * rstd * a.norm_g[ch + 1];
     if (ch >= c - R) {
       float cs, sn;
-      rope_cos_sin(pos, (ch - (c - R)) >> 1, R, a.rope_base, &cs, &sn);
+      rope_cos_sin(pos, a.rope.t[(ch - (c - R)) >> 1], &cs, &sn);
       const float y0 = x0 * cs - x1 * sn;
       const float y1 = x0 * sn + x1 * cs;
       x0 = y0;
@@ -248,174 +249,6 @@ cudaError_t launch_index_scores_generic(const IndexArgs& a, cudaStream_t s) {
 }
 
 // ===========================================================================
-// Top-k selector ("DeepSeek-v4 Beyond Basics" 3.2.2 eq. 17; "Phase 1
-// Module 1" "Top-k selects"): keep the k highest of the n_vis visible scores,
-// ties to the lower index; indices ascending, -1 padded.
-// One thread block per query row.  A 4-pass 8-bit radix select on the
-// order-preserving uint32 image of the scores finds the k-th largest key T
-// and how many of the entries equal to T are needed; entries above T are
-// appended in any order, the needed ties are taken in index order (the scan
-// stops once it has enough), and each kept index is placed at its rank.
-// ===========================================================================
-constexpr int kTopkThreads = 1024;
-
-__device__ __forceinline__ int block_excl_count(bool flag, int* s_warp, int* total) {
-  // exclusive prefix count of flag over the block, in thread order
-  const unsigned int ballot = __ballot_sync(0xffffffffu, flag);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int in_warp = __popc(ballot & ((1u << lane) - 1u));
-  if (lane == 0) s_warp[warp] = __popc(ballot);
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = blockDim.x >> 5;
-    int v = lane < nw ? s_warp[lane] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += n;
-    }
-    if (lane < nw) s_warp[32 + lane] = incl - v;
-    if (lane == 31) s_warp[64] = incl;
-  }
-  __syncthreads();
-  const int r = s_warp[32 + warp] + in_warp;
-  *total = s_warp[64];
-  __syncthreads();
-  return r;
-}
-
-// kSmemKeys: the row's order-preserving keys are staged in shared memory
-// once (rows of up to kTopkSmemKeys entries); otherwise every pass reads
-// the scores from global memory (L2).
-constexpr int kTopkSmemKeys = 12288;
-
-template <int kThreadsT, bool kSmemKeys>
-__global__ void __launch_bounds__(kThreadsT) topk_kernel(IndexArgs a) {
-  extern __shared__ unsigned int tsm[];
-  int* cand = reinterpret_cast<int*>(tsm);            // [k]
-  unsigned int* keys = tsm + ((a.k + 3) & ~3);         // [n_vis] (kSmemKeys)
-  __shared__ unsigned int hist[256];
-  __shared__ int s_warp[65];
-  __shared__ unsigned int s_digit;
-  __shared__ int s_above;
-  __shared__ int s_cnt;
-
-  const int row = blockIdx.x;
-  const int k = a.k;
-  const int pos = a.q_pos[row];
-  const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
-  const float* sc = a.scores + (int64_t)row * a.N_c;
-  int32_t* out = a.idx_out + (int64_t)row * k;
-  float* so = a.score_out ? a.score_out + (int64_t)row * k : nullptr;
-  const int tid = threadIdx.x;
-  if (pos < 0 && tid == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
-
-  if (n_vis <= k) {
-    for (int i = tid; i < k; i += blockDim.x) {
-      out[i] = i < n_vis ? i : -1;
-      if (so) so[i] = i < n_vis ? sc[i] : -INFINITY;
-    }
-    return;
-  }
-  if (kSmemKeys) {
-    for (int i = tid; i < n_vis; i += blockDim.x) keys[i] = f2key(sc[i]);
-    __syncthreads();
-  }
-  auto key_at = [&](int i) -> unsigned int { return kSmemKeys ? keys[i] : f2key(sc[i]); };
-  unsigned int prefix = 0, mask = 0;
-  int remaining = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < n_vis; i += blockDim.x) {
-      const unsigned int u = key_at(i);
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
-    }
-    __syncthreads();
-    if (tid < 32) {
-      // lane l holds digits 255-8l .. 248-8l (descending)
-      int cnt[8], sum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { cnt[j] = (int)hist[255 - 8 * tid - j]; sum += cnt[j]; }
-      int incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (tid >= o) incl += n;
-      }
-      const int excl = incl - sum;
-      if (excl < remaining && incl >= remaining) {
-        int above = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (above + cnt[j] >= remaining) {
-            s_digit = 255u - 8u * tid - j;
-            s_above = above;
-            break;
-          }
-          above += cnt[j];
-        }
-      }
-    }
-    __syncthreads();
-    prefix |= s_digit << shift;
-    mask |= 255u << shift;
-    remaining -= s_above;
-    __syncthreads();
-  }
-  const unsigned int T = prefix;
-  const int need = remaining;  // ties (== T) to keep, >= 1
-  if (tid == 0) s_cnt = 0;
-  __syncthreads();
-  for (int i = tid; i < n_vis; i += blockDim.x) {
-    if (key_at(i) > T) cand[atomicAdd(&s_cnt, 1)] = i;
-  }
-  __syncthreads();
-  const int n_gt = k - need;
-  int taken = 0;
-  for (int base = 0; base < n_vis && taken < need; base += blockDim.x) {
-    const int i = base + tid;
-    const bool eq = i < n_vis && key_at(i) == T;
-    int tot;
-    const int r = block_excl_count(eq, s_warp, &tot);
-    if (eq && taken + r < need) cand[n_gt + taken + r] = i;
-    taken += tot;
-  }
-  __syncthreads();
-  // place each kept index at its rank (number of kept indices below it)
-  for (int j = tid; j < k; j += blockDim.x) {
-    const int v = cand[j];
-    int rank = 0;
-    for (int q = 0; q < k; ++q) rank += cand[q] < v;
-    out[rank] = v;
-    if (so) so[rank] = sc[v];
-  }
-}
-
-cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
-  const int rows = a.B * a.T_q;
-  if (rows <= 0) return cudaSuccess;
-  const size_t cand_bytes = (size_t)((a.k + 3) & ~3) * sizeof(int);
-  if (a.N_c <= kTopkSmemKeys) {
-    const size_t smem = cand_bytes + (size_t)a.N_c * sizeof(unsigned int);
-    static int cache[16];
-    cudaError_t e = ensure_smem(topk_kernel<512, true>, (int)smem, cache);
-    if (e != cudaSuccess) return e;
-    TraceScope tr("topk_smem", s);
-    topk_kernel<512, true><<<rows, 512, smem, s>>>(a);
-    return cudaGetLastError();
-  }
-  static int cache[16];
-  cudaError_t e = ensure_smem(topk_kernel<kTopkThreads, false>, (int)cand_bytes, cache);
-  if (e != cudaSuccess) return e;
-  TraceScope tr("topk", s);
-  topk_kernel<kTopkThreads, false><<<rows, kTopkThreads, cand_bytes, s>>>(a);
-  return cudaGetLastError();
-}
-
-// ===========================================================================
 // Attention, CUDA-core form ("DeepSeek-v4 Beyond Basics" 3.2.2 eq. 19,
 // 3.3 eqs. 24-27; "DeepSeek V4 Inside" sink and window examples).
 // Thread block = (split, query, sequence).  The query's key list is the
@@ -473,7 +306,7 @@ __device__ __forceinline__ const uint16_t* key_row(const AttendArgs& a, int b, c
 __device__ void rope_table(const AttendArgs& a, int pos, float2* rt) {
   for (int j = threadIdx.x; j < a.R / 2; j += blockDim.x) {
     float cs, sn;
-    rope_cos_sin(pos, j, a.R, a.rope_base, &cs, &sn);
+    rope_cos_sin(pos, a.rope.t[j], &cs, &sn);
     rt[j] = make_float2(cs, sn);
   }
 }
@@ -689,16 +522,28 @@ __global__ void __launch_bounds__(kAttThreads) attend_combine_kernel(AttendArgs 
 int attend_splits(int B, int T_q, int keys_max, int H, int D, bool tc, size_t ws_bytes,
                   size_t* need) {
   const int rows = B * T_q;
-  int want = 1;
+  const size_t per = (size_t)rows * (2 * H + (size_t)H * D) * sizeof(float);
   if (tc) {
-    want = attend_tc_splits(B, T_q, keys_max);
-  } else if (rows > 0 && rows < 2 * 148) {
+    // the tensor-core path keeps one 64 KB prepared q^ per query in front
+    // of the split partials; without room for those it cannot run (0)
+    const size_t qimg = (size_t)rows * 65536u;
+    int want = attend_tc_splits(B, T_q, keys_max);
+    if (need) *need = qimg + (want > 1 ? per * want : 0);
+    if (ws_bytes < qimg) return 0;
+    const size_t avail = ws_bytes - qimg;
+    if (want > 1 && per > 0 && avail < per * want) {
+      want = (int)(avail / per);
+      if (want < 2) want = 1;
+    }
+    return want;
+  }
+  int want = 1;
+  if (rows > 0 && rows < 2 * 148) {
     want = (2 * 148 + rows - 1) / rows;
     const int by_keys = (keys_max + 63) / 64;
     want = min(want, max(1, by_keys));
     want = min(want, 64);
   }
-  const size_t per = (size_t)rows * (2 * H + (size_t)H * D) * sizeof(float);
   if (need) *need = want > 1 ? per * want : 0;
   if (want > 1 && per > 0 && ws_bytes < per * want) {
     want = (int)(ws_bytes / per);

@@ -38,16 +38,21 @@ __device__ __forceinline__ unsigned int f2_to_bf2x2(float a, float b) {
   return (unsigned int)f2bf(a) | ((unsigned int)f2bf(b) << 16);
 }
 
-// Rotation angle pos * base^(-2j/R), formed in float64 so that positions up
-// to 2^20 and beyond keep their phase (float32 would lose ~0.03 rad there).
-__device__ __forceinline__ void rope_cos_sin(int pos, int j, int rope_dim, float base, float* c,
-                                             float* s) {
-  double theta = exp2(-(2.0 * j / (double)rope_dim) * log2((double)base));
-  double ang = (double)pos * theta;
-  double sd, cd;
-  sincos(ang, &sd, &cd);
-  *c = (float)cd;
-  *s = (float)sd;
+// RoPE frequencies theta_j = base^(-2j/R), j < R/2, divided by pi and
+// formed in float64 on the host once per call (float32 would lose ~0.03 rad
+// of phase at positions near 2^20).
+constexpr int kMaxRopePairs = 256;
+struct RopeTheta {
+  double t[kMaxRopePairs];
+};
+void fill_rope_theta(RopeTheta* r, int rope_dim, float base);
+
+// cos / sin of pos * theta_j: one float64 product, an exact reduction of the
+// angle (in units of pi) into [-1, 1], then float32 sincospif.
+__device__ __forceinline__ void rope_cos_sin(int pos, double theta_over_pi, float* c, float* s) {
+  double t = (double)pos * theta_over_pi;
+  t -= 2.0 * rint(0.5 * t);
+  sincospif((float)t, s, c);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -114,6 +119,7 @@ struct CompressArgs {
   uint16_t* pool;
   int64_t pool_bstride;
   unsigned int* err;
+  RopeTheta rope;
 };
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
 
@@ -149,6 +155,7 @@ struct AttendArgs {
   int n_splits;
   int keys_max;  // upper bound of keys per query
   unsigned int* err;
+  RopeTheta rope;
 };
 // Key splits per query (and the workspace they need) for the path that
 // serves these sizes; fewer when ws_bytes cannot hold the partials.

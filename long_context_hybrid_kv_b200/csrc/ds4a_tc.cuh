@@ -196,6 +196,27 @@ __device__ __forceinline__ void st_shared16(uint32_t dst, uint32_t a, uint32_t b
                : "memory");
 }
 
+// bulk copy global -> shared (no tensor map, no multicast): bytes a multiple
+// of 16, both addresses 16-byte aligned; completes as transaction bytes on
+// the mbarrier
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// 2^x with the hardware approximation (about 2 ulp; the softmax weights are
+// rounded to bf16 right after)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 128-byte swizzle inside a 1024-byte atom: 16-byte chunk c of row r
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
   return row * 128u + (((chunk ^ row) & 7u) << 4);
@@ -254,6 +275,54 @@ __device__ __forceinline__ void warp_reduce64(const float (&v)[64], float& r0, f
   }
   r0 = e[0];
   r1 = e[1];
+}
+
+// Reduce 32 values per lane over the 32 lanes of a warp; afterwards lane l
+// holds the result of entry l (31 shuffles).
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce32(const float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+  float a[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const bool up = lane & 16;
+    const float send = up ? v[i] : v[i + 16];
+    const float keep = up ? v[i + 16] : v[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 16);
+    a[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+  float b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool up = lane & 8;
+    const float send = up ? a[i] : a[i + 8];
+    const float keep = up ? a[i + 8] : a[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 8);
+    b[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+  float c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool up = lane & 4;
+    const float send = up ? b[i] : b[i + 4];
+    const float keep = up ? b[i + 4] : b[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 4);
+    c[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+  float d[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool up = lane & 2;
+    const float send = up ? c[i] : c[i + 2];
+    const float keep = up ? c[i + 2] : c[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 2);
+    d[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+  const bool up = lane & 1;
+  const float send = up ? d[0] : d[1];
+  const float keep = up ? d[1] : d[0];
+  const float got = __shfl_xor_sync(0xffffffffu, send, 1);
+  return kMax ? fmaxf(keep, got) : keep + got;
 }
 
 }  // namespace tc

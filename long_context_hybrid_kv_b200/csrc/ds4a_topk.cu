@@ -1,0 +1,346 @@
+// Top-k selector of the Lightning indexer ("DeepSeek-v4 Beyond Basics"
+// 3.2.2 eq. 17; "Phase 1 Module 1" "Top-k selects", "only kicks in once
+// there are more than 512 rows"): keep the k highest of a row's n_vis
+// visible scores, ties to the lower index; write the kept indices
+// ascending, padded with -1 when n_vis <= k.
+//
+// Scores become order-preserving uint32 keys.  A 4-pass 8-bit radix select
+// finds the k-th largest key T and how many entries equal to T are needed;
+// an ordered compaction then walks the row in index order and keeps every
+// key above T and the first `need` keys equal to T, so the output comes out
+// ascending without a sort.
+//   topk_smem_kernel     one thread block per row, the row's keys staged in
+//                        shared memory once (rows up to 12288 entries)
+//   topk_cluster_kernel  one 8-block cluster per row (rows up to 262144):
+//                        each block stages a slice; histograms and the
+//                        compaction offsets are summed over the cluster
+//                        through distributed shared memory
+//   topk_global_kernel   one block per row, every pass reading the scores
+//                        from global memory (any length)
+#include <cooperative_groups.h>
+
+#include "ds4a_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace ds4a {
+namespace {
+
+constexpr int kSmemRowMax = 12288;
+constexpr int kCluster = 8;
+constexpr int kClusterSlice = 32768;
+constexpr int kClusterThreads = 1024;
+
+// inclusive scan of v over the block (thread order); *total = block sum.
+// s_warp: >= 33 ints of shared memory.  Every thread must call it.
+__device__ __forceinline__ int block_incl_scan(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += n;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    if (lane < nw) s_warp[lane] = w;  // inclusive warp prefix
+    if (lane == 31) s_warp[32] = w;
+  }
+  __syncthreads();
+  const int r = x + (warp > 0 ? s_warp[warp - 1] : 0);
+  *total = s_warp[32];
+  __syncthreads();
+  return r;
+}
+
+// Digit of this pass: the bin holding the remaining-th largest key.
+// hist: 256 counts; returns the digit and the count of keys in higher bins.
+__device__ __forceinline__ void find_digit(const unsigned int* hist, int remaining, unsigned int* s_digit,
+                                           int* s_above) {
+  const int lane = threadIdx.x;
+  if (lane >= 32) return;
+  int cnt[8], sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    cnt[j] = (int)hist[255 - 8 * lane - j];
+    sum += cnt[j];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  const int excl = incl - sum;
+  if (excl < remaining && incl >= remaining) {
+    int above = excl;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (above + cnt[j] >= remaining) {
+        *s_digit = 255u - 8u * lane - j;
+        *s_above = above;
+        break;
+      }
+      above += cnt[j];
+    }
+  }
+}
+
+__device__ __forceinline__ void write_identity(const IndexArgs& a, int n_vis, const float* sc, int32_t* out,
+                                               float* so) {
+  for (int i = threadIdx.x; i < a.k; i += blockDim.x) {
+    out[i] = i < n_vis ? i : -1;
+    if (so) so[i] = i < n_vis ? sc[i] : -INFINITY;
+  }
+}
+
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
+  extern __shared__ unsigned int keys[];  // [n_vis]
+  __shared__ unsigned int hist[256];
+  __shared__ int s_warp[33];
+  __shared__ unsigned int s_digit;
+  __shared__ int s_above;
+  const int row = blockIdx.x, tid = threadIdx.x;
+  const int pos = a.q_pos[row];
+  const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
+  const float* sc = a.scores + (int64_t)row * a.N_c;
+  int32_t* out = a.idx_out + (int64_t)row * a.k;
+  float* so = a.score_out ? a.score_out + (int64_t)row * a.k : nullptr;
+  if (pos < 0 && tid == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
+  if (n_vis <= a.k) {
+    write_identity(a, n_vis, sc, out, so);
+    return;
+  }
+  for (int i = tid; i < n_vis; i += blockDim.x) keys[i] = f2key(sc[i]);
+  unsigned int prefix = 0, mask = 0;
+  int remaining = a.k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n_vis; i += blockDim.x) {
+      const unsigned int u = keys[i];
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    find_digit(hist, remaining, &s_digit, &s_above);
+    __syncthreads();
+    prefix |= s_digit << shift;
+    mask |= 255u << shift;
+    remaining -= s_above;
+  }
+  const unsigned int T = prefix;
+  const int need = remaining;
+  // ordered compaction: thread t walks keys [t*run, t*run + run)
+  const int run = (n_vis + blockDim.x - 1) / blockDim.x;
+  const int i0 = min(n_vis, tid * run), i1 = min(n_vis, i0 + run);
+  int gt = 0, eq = 0;
+  for (int i = i0; i < i1; ++i) {
+    const unsigned int u = keys[i];
+    gt += u > T;
+    eq += u == T;
+  }
+  int tot;
+  const int eq_before = block_incl_scan(eq, s_warp, &tot) - eq;
+  const int take_eq = max(0, min(eq, need - eq_before));
+  const int sel_before = block_incl_scan(gt + take_eq, s_warp, &tot) - (gt + take_eq);
+  int o = sel_before, tr = eq_before;
+  for (int i = i0; i < i1; ++i) {
+    const unsigned int u = keys[i];
+    bool keep = u > T;
+    if (u == T) keep = tr++ < need;
+    if (keep) {
+      out[o] = i;
+      if (so) so[o] = sc[i];
+      ++o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThreads)
+    topk_cluster_kernel(IndexArgs a) {
+  extern __shared__ unsigned int keys[];  // [kClusterSlice]
+  __shared__ unsigned int hist[256];
+  __shared__ unsigned int hist_all[256];
+  __shared__ int s_warp[33];
+  __shared__ int s_tot[2];  // this block's tie count, kept count
+  __shared__ unsigned int s_digit;
+  __shared__ int s_above;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int row = blockIdx.x / kCluster, tid = threadIdx.x;
+  const int pos = a.q_pos[row];
+  const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
+  const float* sc = a.scores + (int64_t)row * a.N_c;
+  int32_t* out = a.idx_out + (int64_t)row * a.k;
+  float* so = a.score_out ? a.score_out + (int64_t)row * a.k : nullptr;
+  if (n_vis <= a.k) {  // the same branch in every block of the cluster
+    if (rank == 0) {
+      if (pos < 0 && tid == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
+      write_identity(a, n_vis, sc, out, so);
+    }
+    return;
+  }
+  const int slice = (n_vis + kCluster - 1) / kCluster;
+  const int lo = min(n_vis, rank * slice), hi = min(n_vis, lo + slice);
+  const int n = hi - lo;
+  for (int i = tid; i < n; i += blockDim.x) keys[i] = f2key(sc[lo + i]);
+  unsigned int prefix = 0, mask = 0;
+  int remaining = a.k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += blockDim.x) {
+      const unsigned int u = keys[i];
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    }
+    cl.sync();  // every block's histogram is complete
+    if (tid < 256) {
+      unsigned int s = 0;
+#pragma unroll
+      for (int r = 0; r < kCluster; ++r) s += cl.map_shared_rank(hist, r)[tid];
+      hist_all[tid] = s;
+    }
+    __syncthreads();
+    find_digit(hist_all, remaining, &s_digit, &s_above);
+    cl.sync();  // peers are done reading this block's histogram
+    prefix |= s_digit << shift;
+    mask |= 255u << shift;
+    remaining -= s_above;
+  }
+  const unsigned int T = prefix;
+  const int need = remaining;
+  // ordered compaction across the cluster: block r holds indices
+  // [lo, hi), so the ties and kept entries of lower ranks come first
+  const int run = (n + blockDim.x - 1) / blockDim.x;
+  const int i0 = min(n, tid * run), i1 = min(n, i0 + run);
+  int gt = 0, eq = 0;
+  for (int i = i0; i < i1; ++i) {
+    const unsigned int u = keys[i];
+    gt += u > T;
+    eq += u == T;
+  }
+  int eq_tot;
+  const int eq_local = block_incl_scan(eq, s_warp, &eq_tot) - eq;
+  if (tid == 0) s_tot[0] = eq_tot;
+  cl.sync();
+  int eq_base = 0;
+  for (int r = 0; r < rank; ++r) eq_base += cl.map_shared_rank(s_tot, r)[0];
+  const int eq_before = eq_base + eq_local;
+  const int take_eq = max(0, min(eq, need - eq_before));
+  int sel_tot;
+  const int sel_local = block_incl_scan(gt + take_eq, s_warp, &sel_tot) - (gt + take_eq);
+  if (tid == 0) s_tot[1] = sel_tot;
+  cl.sync();
+  int sel_base = 0;
+  for (int r = 0; r < rank; ++r) sel_base += cl.map_shared_rank(s_tot, r)[1];
+  int o = sel_base + sel_local, tr = eq_before;
+  for (int i = i0; i < i1; ++i) {
+    const unsigned int u = keys[i];
+    bool keep = u > T;
+    if (u == T) keep = tr++ < need;
+    if (keep) {
+      out[o] = lo + i;
+      if (so) so[o] = sc[lo + i];
+      ++o;
+    }
+  }
+  cl.sync();  // no block leaves while a peer may still read its shared memory
+}
+
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) topk_global_kernel(IndexArgs a) {
+  __shared__ unsigned int hist[256];
+  __shared__ int s_warp[33];
+  __shared__ unsigned int s_digit;
+  __shared__ int s_above;
+  const int row = blockIdx.x, tid = threadIdx.x;
+  const int pos = a.q_pos[row];
+  const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
+  const float* sc = a.scores + (int64_t)row * a.N_c;
+  int32_t* out = a.idx_out + (int64_t)row * a.k;
+  float* so = a.score_out ? a.score_out + (int64_t)row * a.k : nullptr;
+  if (pos < 0 && tid == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
+  if (n_vis <= a.k) {
+    write_identity(a, n_vis, sc, out, so);
+    return;
+  }
+  unsigned int prefix = 0, mask = 0;
+  int remaining = a.k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n_vis; i += blockDim.x) {
+      const unsigned int u = f2key(sc[i]);
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    find_digit(hist, remaining, &s_digit, &s_above);
+    __syncthreads();
+    prefix |= s_digit << shift;
+    mask |= 255u << shift;
+    remaining -= s_above;
+  }
+  const unsigned int T = prefix;
+  const int need = remaining;
+  // ordered compaction in chunks of blockDim (coalesced reads)
+  int out_base = 0, eq_base = 0;
+  for (int base = 0; base < n_vis; base += blockDim.x) {
+    const int i = base + tid;
+    const unsigned int u = i < n_vis ? f2key(sc[i]) : 0u;
+    const int eq = (i < n_vis && u == T) ? 1 : 0;
+    int eq_tot;
+    const int eq_before = eq_base + block_incl_scan(eq, s_warp, &eq_tot) - eq;
+    const int keep = (i < n_vis && (u > T || (eq && eq_before < need))) ? 1 : 0;
+    int keep_tot;
+    const int o = out_base + block_incl_scan(keep, s_warp, &keep_tot) - keep;
+    if (keep) {
+      out[o] = i;
+      if (so) so[o] = sc[i];
+    }
+    out_base += keep_tot;
+    eq_base += eq_tot;
+    if (out_base >= a.k) break;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
+  const int rows = a.B * a.T_q;
+  if (rows <= 0) return cudaSuccess;
+  if (a.N_c <= kSmemRowMax) {
+    const size_t smem = (size_t)max(1, a.N_c) * sizeof(unsigned int);
+    static int cache[16];
+    cudaError_t e = ensure_smem(topk_smem_kernel, (int)smem, cache);
+    if (e != cudaSuccess) return e;
+    TraceScope tr("topk_smem", s);
+    topk_smem_kernel<<<rows, 512, smem, s>>>(a);
+    return cudaGetLastError();
+  }
+  if (a.N_c <= kCluster * kClusterSlice) {
+    const size_t smem = (size_t)kClusterSlice * sizeof(unsigned int);
+    static int cache[16];
+    cudaError_t e = ensure_smem(topk_cluster_kernel, (int)smem, cache);
+    if (e != cudaSuccess) return e;
+    TraceScope tr("topk_cluster", s);
+    topk_cluster_kernel<<<rows * kCluster, kClusterThreads, smem, s>>>(a);
+    return cudaGetLastError();
+  }
+  TraceScope tr("topk_global", s);
+  topk_global_kernel<<<rows, 1024, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ds4a

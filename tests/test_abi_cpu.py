@@ -134,8 +134,11 @@ def test_workspace_queries():
     assert L.ds4a_index_topk_workspace(cfg, 1, 1, 0) == 0
     # few queries: split over more blocks -> partials need workspace
     assert L.ds4a_attend_workspace(cfg, 1, 1, 2048, True) > 0
-    # many queries: one block each, no workspace
-    assert L.ds4a_attend_workspace(cfg, 1, 16384, 4096, True) == 0
+    # many queries on the tensor-core path: one prepared query (64 KiB) each,
+    # no split partials
+    assert L.ds4a_attend_workspace(cfg, 1, 16384, 4096, True) == 16384 * 65536
+    # the CUDA-core path (another head width) needs none for many queries
+    assert L.ds4a_attend_workspace(flash_cfg(head_dim=256, rope_dim=32), 1, 16384, 4096, True) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

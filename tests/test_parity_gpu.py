@@ -160,6 +160,26 @@ def test_index_topk_ties_take_lower_index():
     assert np.array_equal(gidx[0, 0], np.arange(FLASH.topk))
 
 
+def test_index_topk_large_rows_cluster_path():
+    # rows above the shared-memory size take the 8-block cluster selector:
+    # random keys (checked against the oracle) and all-equal keys (ties)
+    n_c = 50000
+    pos = [4 * n_c - 1, 4 * 20000 - 1, 4 * 12289 - 1]
+    qi, wi, ki, qpos, gidx, gsc = _index_case(2, pos, n_c, FLASH, "clus")
+    _check_index(qi, wi, ki, qpos, gidx, gsc, FLASH, n_c)
+    row = nb("clus.tie", (1, 1, FLASH.idx_dim))
+    ki = np.repeat(row, n_c, axis=1)
+    qi, wi, ki, qpos, gidx, gsc = _index_case(1, [4 * n_c - 1], n_c, FLASH, "clustie", ki=ki)
+    assert np.array_equal(gidx[0, 0], np.arange(FLASH.topk))
+
+
+def test_index_topk_beyond_cluster_rows():
+    # longer than the cluster selector's 262144: the global-memory selector
+    n_c = 262144 + 1000
+    qi, wi, ki, qpos, gidx, gsc = _index_case(1, [4 * n_c - 1], n_c, FLASH, "huge")
+    _check_index(qi, wi, ki, qpos, gidx, gsc, FLASH, n_c)
+
+
 def test_index_topk_prefill_rows():
     # causal prefill over 4096 tokens (1024 entries), sampled rows
     T = 4096
@@ -181,7 +201,7 @@ def test_index_topk_toy():
 # ---------------------------------------------------------------------------
 # attention
 # ---------------------------------------------------------------------------
-def _attend_case(name, cfg_py, B, positions, n_c, sparse, win_cap, use_ws=True, idx=None):
+def _attend_case(name, cfg_py, B, positions, n_c, sparse, win_cap, use_ws=True, idx=None, ws_bytes=None):
     Tq = len(positions)
     H, D = cfg_py.n_heads, cfg_py.head_dim
     q = nb(f"{name}.q", (B, Tq, H, D))
@@ -192,7 +212,10 @@ def _attend_case(name, cfg_py, B, positions, n_c, sparse, win_cap, use_ws=True, 
     qpos = np.tile(np.asarray(positions, np.int32), (B, 1))
     cfg = L.layer_cfg(cfg_py)
     out = torch.empty((B, Tq, H, D), dtype=torch.bfloat16, device="cuda")
-    ws = ws_f32(L.ds4a_attend_workspace(cfg, B, Tq, n_c, sparse)) if use_ws else None
+    if ws_bytes is not None:
+        ws = ws_f32(ws_bytes)
+    else:
+        ws = ws_f32(L.ds4a_attend_workspace(cfg, B, Tq, n_c, sparse)) if use_ws else None
     if sparse:
         if idx is None:
             n_vis = np.minimum((qpos + 1) // cfg_py.ratio, n_c)
@@ -221,6 +244,25 @@ def test_sparse_attend_flash(use_ws):
 @pytest.mark.parametrize("use_ws", [True, False], ids=["split", "nosplit"])
 def test_hca_attend_flash(use_ws):
     _attend_case("hc", HCA, 2, [126, 127, 5119, 6000], 40, False, 128, use_ws)
+
+
+def test_attend_tensor_core_without_splits():
+    # workspace for the prepared queries only: the tensor-core path with one
+    # split per query (final output written by the attention kernel)
+    pos = [0, 5, 127, 300, 3999]
+    names = kernels_used(lambda: _attend_case("tc1", FLASH, 2, pos, 1000, True, 128, ws_bytes=2 * 5 * 65536))
+    assert "attend_tc" in names and "attend_combine" not in names, names
+    names = kernels_used(lambda: _attend_case("tc1h", HCA, 2, [126, 5119], 40, False, 128, ws_bytes=2 * 2 * 65536))
+    assert "attend_tc" in names and "attend_combine" not in names, names
+
+
+def test_attend_paths_used():
+    # Flash shapes with the recommended workspace take the tensor-core
+    # kernels; without a workspace the CUDA-core kernel runs
+    names = kernels_used(lambda: _attend_case("path", FLASH, 1, [3999], 1000, True, 128))
+    assert "qhat_prep" in names and "attend_tc" in names, names
+    names = kernels_used(lambda: _attend_case("path0", FLASH, 1, [3999], 1000, True, 128, use_ws=False))
+    assert names == ["attend_generic"], names
 
 
 def test_swa_only_layer():
@@ -405,8 +447,9 @@ def _tensor_core_path_active():
     z = torch.ones(512, device="cuda")
     idx = torch.full((1, 1, 512), -1, dtype=torch.int32, device="cuda")
     win = torch.zeros((1, 128, 512), dtype=torch.bfloat16, device="cuda")
+    ws = ws_f32(L.ds4a_attend_workspace(cfg, 1, 1, 0, True))
     names = kernels_used(lambda: L.ds4a_sparse_attend(cfg, i32([[10]]), q, z, None, 0, idx, win, 128,
-                                                      z[:64], out))
+                                                      z[:64], out, ws))
     return any("tc" in n for n in names)
 
 

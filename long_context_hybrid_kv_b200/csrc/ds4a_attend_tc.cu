@@ -157,7 +157,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
   float* mrun = reinterpret_cast<float*>(smem + kOffMrun);
   float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);
   float* inv_s = reinterpret_cast<float*>(smem + kOffInv);
-  int* any_rescale = reinterpret_cast<int*>(smem + kOffMisc + 16);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -186,6 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   unsigned int* err = a.err;
+  pdl_trigger();
+  pdl_wait();
 
   if (warp < 8) {
     // =================== softmax + epilogue (8 warps) ===================
@@ -234,23 +235,34 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
         float z[32];
         tmem_ld32(t_lane + sb * 64u + (uint32_t)h0, z);
         tmem_ld_wait();
+        bool over = false;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] = valid ? z[i] * scale2 : -INFINITY;
-        red[q4 * 64 + h0 + lane] = warp_reduce32<true>(z);
-        if (st == 0) *any_rescale = 0;
-        named_bar(1, 256);
-        if (st < kH) {
-          const float mt = fmaxf(fmaxf(red[st], red[64 + st]), fmaxf(red[128 + st], red[192 + st]));
-          const float mo = mrun[st];
-          float al = 1.f;
-          if (mt > mo + kRescaleLog2 || (mo == -INFINITY && mt != -INFINITY)) {
-            al = (mo == -INFINITY) ? 0.f : exp2f(mo - mt);
-            mrun[st] = mt;
-            *any_rescale = 1;
-          }
-          alpha_s[st] = al;
+        for (int i = 0; i < 32; ++i) {
+          z[i] = valid ? z[i] * scale2 : -INFINITY;
+          const float mr = mrun[h0 + i];
+          over |= z[i] > mr + kRescaleLog2 || (mr == -INFINITY && z[i] != -INFINITY);
         }
-        named_bar(1, 256);
+        // the running reference moves (and O^T is rescaled) only when some
+        // head's logit passes it by more than 2^8: one barrier-reduction
+        // decides whether the tile maximum is needed at all
+        const bool rescale = bar_or(1, 256, over);
+        if (rescale) {
+          red[q4 * 64 + h0 + lane] = warp_reduce32<true>(z);
+          named_bar(1, 256);
+          if (st < kH) {
+            const float mt = fmaxf(fmaxf(red[st], red[64 + st]), fmaxf(red[128 + st], red[192 + st]));
+            const float mo = mrun[st];
+            float al = 1.f;
+            if (mt > mo + kRescaleLog2 || (mo == -INFINITY && mt != -INFINITY)) {
+              al = (mo == -INFINITY) ? 0.f : exp2f(mo - mt);
+              mrun[st] = mt;
+            }
+            alpha_s[st] = al;
+          }
+          named_bar(1, 256);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) lpart[i] *= alpha_s[h0 + i];
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -260,14 +272,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
           const uint32_t w2 = f2_to_bf2x2(pa, pb);
           pk[i >> 1] = w2;
           const float2 pr = bf2x2_to_f2(w2);
-          lpart[i] = lpart[i] * alpha_s[h0 + i] + pr.x;
-          lpart[i + 1] = lpart[i + 1] * alpha_s[h0 + i + 1] + pr.y;
+          lpart[i] += pr.x;
+          lpart[i + 1] += pr.y;
         }
         if (tile > 0) {
           // the previous tile's PV must be done before P^T and O^T change
           mbar_wait(bar(kPVDone), (gt - 1) & 1u, abort_flag, err);
           tc_fence_after();
-          if (*any_rescale) {
+          if (rescale) {
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float v[32];
@@ -356,6 +368,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
     }
   } else if (warp == kMmaWarp) {
     // =================== MMA issuer ===================
+    // Descriptors are built once; every product adds a compile-time offset
+    // (the start-address field holds addr >> 4 and stays below 2^14), so the
+    // issue loop is an add and the MMA per step.
+    const uint64_t qk_a0 = sdesc_sw128(kv_base, 16, 1024);
+    const uint64_t qk_b0 = sdesc_sw128(q_base, 16, 1024);
+    const uint64_t pv_a0 = sdesc_sw128(kv_base, 16384, 1024);
+    const uint64_t pv_b0 = sdesc_sw128(p_base, 16384, 1024);
     uint32_t gt = 0, active = 0;
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       const Item it = make_item(a, w);
@@ -364,7 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
         mbar_wait(bar(kQFull), active & 1u, abort_flag, err);
         tc_fence_after();
         for (int tile = 0; tile < it.n_tiles; ++tile, ++gt) {
-          const uint32_t sb = gt & 1u;
+          const uint32_t d_s = tmem + (gt & 1u) * 64u;
+#pragma unroll
           for (int c = 0; c < 4; ++c) {
             mbar_wait(bar(kKVFull0 + c), gt & 1u, abort_flag, err);
             tc_fence_after();
@@ -372,9 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t blk = 2u * c + (kk >> 2);
               const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-              const uint64_t ad = sdesc_sw128(kv_base + blk * 16384u + koff, 16, 1024);
-              const uint64_t bd = sdesc_sw128(q_base + blk * 8192u + koff, 16, 1024);
-              mma_bf16(tmem + sb * 64u, ad, bd, kIdescQK, (c | kk) != 0);
+              mma_bf16(d_s, qk_a0 + ((blk * 16384u + koff) >> 4), qk_b0 + ((blk * 8192u + koff) >> 4),
+                       kIdescQK, (c | kk) != 0 ? 1u : 0u);
             }
           }
           mma_commit(bar(kSFull));
@@ -382,13 +401,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
           mbar_wait(bar(kPFull), gt & 1u, abort_flag, err);
           if (tile == 0 && active > 0) mbar_wait(bar(kEpiDone), (active - 1) & 1u, abort_flag, err);
           tc_fence_after();
+          const uint32_t acc0 = tile == 0 ? 0u : 1u;
+#pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t ad = sdesc_sw128(kv_base + 2u * c * 16384u + kk * 2048u, 16384, 1024);
-              const uint64_t bd = sdesc_sw128(p_base + kk * 2048u, 16384, 1024);
-              mma_bf16(tmem + 128u + 64u * c, ad, bd, kIdescPV, !(tile == 0 && kk == 0));
-            }
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16(tmem + 128u + 64u * c, pv_a0 + ((2u * c * 16384u + kk * 2048u) >> 4),
+                       pv_b0 + ((kk * 2048u) >> 4), kIdescPV, kk == 0 ? acc0 : 1u);
             mma_commit(bar(kKVEmpty0 + c));
           }
           mma_commit(bar(kPVDone));
@@ -420,7 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
         rowptr[pt] = p;
         named_bar(2, 128);
       };
-      // one 128-dim chunk of the tile: 128 rows x 256 B, 16 cp.async each
+      // one 128-dim chunk of the tile: 128 rows x 256 B, 16 cp.async each;
+      // rows past the key list or with a bad index are zero-filled
       auto issue_chunk = [&](int c) {
         if (gt > 0) mbar_wait(bar(kKVEmpty0 + c), (gt - 1) & 1u, abort_flag, err);
         const uint32_t blk = kv_base + (uint32_t)(2 * c + (piece >> 3)) * 16384u;
@@ -443,6 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
       }
       // ---- K=V tiles: each chunk goes out when the PV products of the
       // previous tile have released it ----
+      // Two chunks stay in flight: chunk c goes out, then chunk c-1 is
+      // retired (a deeper queue over-subscribes L2 across the SMs).
       for (int tile = 0; tile < it.n_tiles; ++tile, ++gt) {
         set_rowptr(tile);
 #pragma unroll 1
@@ -460,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
       }
       ++active;
     }
-    cp_async_wait<0>();
+    cp_async_wait<0>();  // nothing of this block is in flight at exit
   }
 
   tc_fence_before();
@@ -478,6 +500,8 @@ __global__ void __launch_bounds__(256) qhat_prep_kernel(AttendArgs a, uint8_t* q
   const int row = blockIdx.x;
   const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();
   const int pos = a.q_pos[row];
   const int R = a.R;
   for (int j = threadIdx.x; j < R / 2; j += blockDim.x) {
@@ -557,17 +581,16 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   {
     TraceScope tr("qhat_prep", s);
-    qhat_prep_kernel<<<dim3(rows, kH / 8), 256, 0, s>>>(a, qimg);
+    e = launch_pdl(qhat_prep_kernel, dim3(rows, kH / 8), dim3(256), 0, s, a, qimg);
   }
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n_items = rows * a.n_splits;
   const int grid = min(n_items, 148);
   {
     TraceScope tr("attend_tc", s);
-    attend_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a, n_items, qimg);
+    e = launch_pdl(attend_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, a, n_items,
+                   static_cast<const uint8_t*>(qimg));
   }
-  e = cudaGetLastError();
   if (e != cudaSuccess || a.n_splits == 1) return e;
   return launch_attend_combine(a, s);
 }

@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
   const int b = blockIdx.y;
   const bool overlap = a.cb != nullptr;
   const int n_terms = (overlap && i >= 1) ? 2 * m : m;
+  pdl_trigger();
+  pdl_wait();
 
   float mx[V], l[V], acc[V];
 #pragma unroll
@@ -185,11 +187,8 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
                          : ensure_smem(compress_kernel<2>, (int)smem, cache2);
   if (e != cudaSuccess) return e;
   TraceScope tr("compress", s);
-  if (V == 8)
-    compress_kernel<8><<<dim3(n, a.B), kCompressThreads, smem, s>>>(a);
-  else
-    compress_kernel<2><<<dim3(n, a.B), kCompressThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return V == 8 ? launch_pdl(compress_kernel<8>, dim3(n, a.B), dim3(kCompressThreads), smem, s, a)
+                : launch_pdl(compress_kernel<2>, dim3(n, a.B), dim3(kCompressThreads), smem, s, a);
 }
 
 // ===========================================================================
@@ -207,6 +206,8 @@ __global__ void __launch_bounds__(kIdxKeys) index_score_generic_kernel(IndexArgs
   float* qs = ism;              // [H * D]
   float* wsum = qs + H * D;     // [H]
   float* kt = wsum + H;         // [128 * (D + 1)]
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x;
   const int b = row / a.T_q;
   const int pos = a.q_pos[row];
@@ -244,8 +245,8 @@ cudaError_t launch_index_scores_generic(const IndexArgs& a, cudaStream_t s) {
   cudaError_t e = ensure_smem(index_score_generic_kernel, (int)smem, cache);
   if (e != cudaSuccess) return e;
   TraceScope tr("index_score_generic", s);
-  index_score_generic_kernel<<<dim3(rows, (a.N_c + kIdxKeys - 1) / kIdxKeys), kIdxKeys, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(index_score_generic_kernel, dim3(rows, (a.N_c + kIdxKeys - 1) / kIdxKeys), dim3(kIdxKeys),
+                    smem, s, a);
 }
 
 // ===========================================================================
@@ -373,6 +374,8 @@ __global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs 
 
   const int split = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
   const int row = b * a.T_q + t;
+  pdl_trigger();
+  pdl_wait();
   const int pos = a.q_pos[row];
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
@@ -475,6 +478,8 @@ __global__ void __launch_bounds__(kAttThreads) attend_combine_kernel(AttendArgs 
   const int h0 = blockIdx.x * kCombHeads;
   const int t = blockIdx.y, b = blockIdx.z;
   const int row = b * a.T_q + t;
+  pdl_trigger();
+  pdl_wait();
   const int pos = a.q_pos[row];
   if (pos < 0) return;
   const int64_t stride = 2 * H + (int64_t)H * D;
@@ -562,7 +567,8 @@ cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
   if (e0 != cudaSuccess) return e0;
   {
     TraceScope tr("attend_generic", s);
-    attend_generic_kernel<<<dim3(a.n_splits, a.T_q, a.B), kAttThreads, smem, s>>>(a);
+    cudaError_t e1 = launch_pdl(attend_generic_kernel, dim3(a.n_splits, a.T_q, a.B), dim3(kAttThreads), smem, s, a);
+    if (e1 != cudaSuccess) return e1;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.n_splits == 1) return e;
@@ -576,8 +582,8 @@ cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s) {
   cudaError_t e = ensure_smem(attend_combine_kernel, (int)smem, cache);
   if (e != cudaSuccess) return e;
   TraceScope tr("attend_combine", s);
-  attend_combine_kernel<<<dim3((a.H + kCombHeads - 1) / kCombHeads, a.T_q, a.B), kAttThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(attend_combine_kernel, dim3((a.H + kCombHeads - 1) / kCombHeads, a.T_q, a.B),
+                    dim3(kAttThreads), smem, s, a);
 }
 
 }  // namespace ds4a

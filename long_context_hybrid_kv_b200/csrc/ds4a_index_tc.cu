@@ -142,6 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     // =================== TMA producer ===================
@@ -173,6 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kt = 0, at = 0, active = 0;
       const uint32_t idesc = idesc_bf16(128, 64 * G, 0, 0);
+      const uint64_t k_desc0 = sdesc_sw128(k_base, 16, 1024);
+      const uint64_t q_desc0 = sdesc_sw128(q_base, 16, 1024);
       for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
         const Pair q = make_pair(p, w);
         if (q.tile1 <= q.tile0) continue;
@@ -184,13 +188,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(kKFull + s), (kt / kStages) & 1u, abort_flag, err);
           if (at >= 2) mbar_wait(bar(kAccEmpty0 + ab), ((at >> 1) - 1) & 1u, abort_flag, err);
           tc_fence_after();
+          const uint64_t a0 = k_desc0 + ((s * 32768u) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t blk = (uint32_t)(kk >> 2);
             const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-            const uint64_t ad = sdesc_sw128(k_base + s * 32768u + blk * 16384u + koff, 16, 1024);
-            const uint64_t bd = sdesc_sw128(q_base + blk * q_blk + koff, 16, 1024);
-            mma_bf16(tmem + ab * 256u, ad, bd, idesc, kk != 0);
+            mma_bf16(tmem + ab * 256u, a0 + ((blk * 16384u + koff) >> 4), q_desc0 + ((blk * q_blk + koff) >> 4),
+                     idesc, kk != 0 ? 1u : 0u);
           }
           mma_commit(bar(kKEmpty + s));
           mma_commit(bar(kAccFull0 + ab));
@@ -321,8 +325,7 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int grid = min(p.n_pairs, 148);
   TraceScope tr("index_score_tc", s);
-  index_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(kmap, qmap, p);
-  return cudaGetLastError();
+  return launch_pdl(index_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, kmap, qmap, p);
 }
 
 }  // namespace ds4a

@@ -97,6 +97,32 @@ inline cudaError_t ensure_smem(F* f, int bytes, int* cache) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: every library kernel is launched with
+// programmatic stream serialisation, lets its successor start once all of its
+// own blocks are running (pdl_trigger), and waits for its predecessor's
+// memory (pdl_wait) before touching global memory.  Every kernel waits, so
+// the ordering is transitive along the stream.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// ---------------------------------------------------------------------------
 // launch trace
 // ---------------------------------------------------------------------------
 struct TraceScope {

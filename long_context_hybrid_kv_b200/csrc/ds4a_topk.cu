@@ -109,6 +109,8 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
   __shared__ unsigned int s_digit;
   __shared__ int s_above;
   const int row = blockIdx.x, tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   const int pos = a.q_pos[row];
   const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
   const float* sc = a.scores + (int64_t)row * a.N_c;
@@ -178,6 +180,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
   const int row = blockIdx.x / kCluster, tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   const int pos = a.q_pos[row];
   const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
   const float* sc = a.scores + (int64_t)row * a.N_c;
@@ -265,6 +269,8 @@ __global__ void __launch_bounds__(1024) topk_global_kernel(IndexArgs a) {
   __shared__ unsigned int s_digit;
   __shared__ int s_above;
   const int row = blockIdx.x, tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   const int pos = a.q_pos[row];
   const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
   const float* sc = a.scores + (int64_t)row * a.N_c;
@@ -326,8 +332,7 @@ cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
     cudaError_t e = ensure_smem(topk_smem_kernel, (int)smem, cache);
     if (e != cudaSuccess) return e;
     TraceScope tr("topk_smem", s);
-    topk_smem_kernel<<<rows, 512, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(topk_smem_kernel, dim3(rows), dim3(512), smem, s, a);
   }
   if (a.N_c <= kCluster * kClusterSlice) {
     const size_t smem = (size_t)kClusterSlice * sizeof(unsigned int);
@@ -335,12 +340,10 @@ cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
     cudaError_t e = ensure_smem(topk_cluster_kernel, (int)smem, cache);
     if (e != cudaSuccess) return e;
     TraceScope tr("topk_cluster", s);
-    topk_cluster_kernel<<<rows * kCluster, kClusterThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(topk_cluster_kernel, dim3(rows * kCluster), dim3(kClusterThreads), smem, s, a);
   }
   TraceScope tr("topk_global", s);
-  topk_global_kernel<<<rows, 1024, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(topk_global_kernel, dim3(rows), dim3(1024), 0, s, a);
 }
 
 }  // namespace ds4a

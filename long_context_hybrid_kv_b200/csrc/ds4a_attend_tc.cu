@@ -79,8 +79,30 @@ __device__ __forceinline__ Item make_item(const AttendArgs& a, int w) {
   it.row = w / a.n_splits;
   it.split = w % a.n_splits;
   it.b = it.row / a.T_q;
-  it.pos = a.q_pos[it.row];
   it.idx_row = a.sparse ? a.idx + (int64_t)it.row * a.k : nullptr;
+  // the index loads go out together with the position load: building an
+  // item costs one memory round trip
+  int n_sel = 0;
+  if (a.sparse) {
+    // selected entries come first (ascending, -1 padded): count them with
+    // independent loads, 16 per lane in flight
+    const int lane = threadIdx.x & 31;
+    int cnt = 0;
+    for (int base = 0; base < a.k; base += 512) {
+      int v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int j = base + 32 * u + lane;
+        v[u] = j < a.k ? it.idx_row[j] : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) cnt += v[u] >= 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    n_sel = cnt;
+  }
+  it.pos = a.q_pos[it.row];
   if (it.pos < 0) {
     it.n_sel = 0;
     it.win_start = 0;
@@ -88,28 +110,7 @@ __device__ __forceinline__ Item make_item(const AttendArgs& a, int w) {
     it.n_tiles = 0;
     return it;
   }
-  int n_sel;
-  if (a.sparse) {
-    // selected entries come first (ascending, -1 padded): count them with
-    // independent loads, 8 per lane in flight
-    const int lane = threadIdx.x & 31;
-    int cnt = 0;
-    for (int base = 0; base < a.k; base += 256) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = base + 32 * u + lane;
-        v[u] = j < a.k ? it.idx_row[j] : -1;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) cnt += v[u] >= 0;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    n_sel = cnt;
-  } else {
-    n_sel = min((it.pos + 1) / a.m, a.N_c);
-  }
+  if (!a.sparse) n_sel = min((it.pos + 1) / a.m, a.N_c);
   it.n_sel = n_sel;
   it.win_start = max(0, it.pos - a.W + 1);
   const int n_win = a.W > 0 ? it.pos - it.win_start + 1 : 0;

@@ -467,60 +467,77 @@ __global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs 
 // maxima, L = sum of l_s exp(m_s - M), o = sum acc_s exp(m_s - M) / (L +
 // exp(sink - M)); then the rope slice rotates back by -pos.  Thread block =
 // 8 heads of one query.
-constexpr int kCombHeads = 8;
+constexpr int kCombThreads = 256;
 
-__global__ void __launch_bounds__(kAttThreads) attend_combine_kernel(AttendArgs a) {
-  extern __shared__ __align__(16) unsigned char cm_raw[];
+// One block per (head, query row), one thread per pair of output dims.
+// Every thread merges the splits itself, eight at a time with all their
+// loads (max, sum, two accumulator values) in flight together: the split
+// maxima and sums are the same addresses for the whole block (broadcast),
+// so no shared memory or block barrier is needed and a decode-sized merge
+// costs one memory round trip.  The sink enters the denominator as in the
+// split-free kernels; the rope slice is de-rotated by -pos at the end.
+__global__ void __launch_bounds__(kCombThreads) attend_combine_kernel(AttendArgs a) {
   const int H = a.H, D = a.D, S = a.n_splits, R = a.R;
-  float2* rt = reinterpret_cast<float2*>(cm_raw);          // [R/2]
-  float* scl = reinterpret_cast<float*>(rt + R / 2 + 1);    // [S * 8]
-  float* inv = scl + S * kCombHeads;                        // [8]
-  const int h0 = blockIdx.x * kCombHeads;
-  const int t = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
   const int row = b * a.T_q + t;
   pdl_trigger();
   pdl_wait();
   const int pos = a.q_pos[row];
-  if (pos < 0) return;
+  const float sink = a.sink[h];
   const int64_t stride = 2 * H + (int64_t)H * D;
   const float* base = a.ws + (int64_t)row * S * stride;
-  const int nh = min(kCombHeads, H - h0);
-  const int tid = threadIdx.x;
-  if (tid < nh) {
-    const int h = h0 + tid;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, base[s * stride + h]);
-    float L = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float ms = base[s * stride + h];
-      const float e = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-      scl[s * kCombHeads + tid] = e;
-      L += base[s * stride + H + h] * e;
+  uint16_t* orow = a.out + ((int64_t)row * H + h) * D;
+  for (int d2 = threadIdx.x; d2 < D / 2; d2 += kCombThreads) {
+    const int d = 2 * d2;
+    float M = -INFINITY, L = 0.f, x0 = 0.f, x1 = 0.f;
+    for (int s0 = 0; s0 < S; s0 += 8) {
+      float ms[8], ls[8];
+      float2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        ms[u] = -INFINITY;
+        ls[u] = 0.f;
+        v[u] = make_float2(0.f, 0.f);
+        if (s0 + u < S) {
+          const float* p = base + (int64_t)(s0 + u) * stride;
+          ms[u] = p[h];
+          ls[u] = p[H + h];
+          v[u] = *reinterpret_cast<const float2*>(p + 2 * H + (int64_t)h * D + d);
+        }
+      }
+      float mc = M;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mc = fmaxf(mc, ms[u]);
+      if (mc == -INFINITY) continue;
+      const float sc = __expf(M - mc);  // 0 while nothing was merged
+      L *= sc;
+      x0 *= sc;
+      x1 *= sc;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        // a split with no visible key has max -inf: its accumulator is
+        // never read into the sum
+        if (ms[u] != -INFINITY) {
+          const float e = __expf(ms[u] - mc);
+          L = fmaf(ls[u], e, L);
+          x0 = fmaf(v[u].x, e, x0);
+          x1 = fmaf(v[u].y, e, x1);
+        }
+      }
+      M = mc;
     }
-    inv[tid] = (M == -INFINITY) ? 0.f : 1.f / (L + __expf(a.sink[h] - M));
-  }
-  rope_table(a, pos, rt);
-  __syncthreads();
-  uint16_t* orow = a.out + (int64_t)row * H * D;
-  for (int e2 = tid; e2 < nh * D / 2; e2 += blockDim.x) {
-    const int hl = (2 * e2) / D, d = (2 * e2) % D, h = h0 + hl;
-    float x0 = 0.f, x1 = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float f = scl[s * kCombHeads + hl];
-      if (f == 0.f) continue;
-      const float2 v = *reinterpret_cast<const float2*>(base + s * stride + 2 * H + (int64_t)h * D + d);
-      x0 = fmaf(v.x, f, x0);
-      x1 = fmaf(v.y, f, x1);
-    }
-    x0 *= inv[hl];
-    x1 *= inv[hl];
+    if (pos < 0) return;
+    const float inv = (M == -INFINITY) ? 0.f : 1.f / (L + __expf(sink - M));
+    x0 *= inv;
+    x1 *= inv;
     if (d >= D - R) {
-      const float2 r = rt[(d - (D - R)) >> 1];
-      const float y0 = x0 * r.x + x1 * r.y, y1 = -x0 * r.y + x1 * r.x;
+      float c, sn;
+      rope_cos_sin(pos, a.rope.t[(d - (D - R)) >> 1], &c, &sn);
+      const float y0 = x0 * c + x1 * sn, y1 = -x0 * sn + x1 * c;
       x0 = y0;
       x1 = y1;
     }
-    *reinterpret_cast<unsigned int*>(orow + (int64_t)h * D + d) = f2_to_bf2x2(x0, x1);
+    *reinterpret_cast<unsigned int*>(orow + d) = f2_to_bf2x2(x0, x1);
   }
 }
 
@@ -576,14 +593,8 @@ cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)(a.R / 2 + 1) * sizeof(float2) +
-                      (size_t)(a.n_splits * kCombHeads + kCombHeads) * sizeof(float);
-  static int cache[16];
-  cudaError_t e = ensure_smem(attend_combine_kernel, (int)smem, cache);
-  if (e != cudaSuccess) return e;
   TraceScope tr("attend_combine", s);
-  return launch_pdl(attend_combine_kernel, dim3((a.H + kCombHeads - 1) / kCombHeads, a.T_q, a.B),
-                    dim3(kAttThreads), smem, s, a);
+  return launch_pdl(attend_combine_kernel, dim3(a.H, a.T_q, a.B), dim3(kCombThreads), 0, s, a);
 }
 
 }  // namespace ds4a

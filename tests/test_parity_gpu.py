@@ -201,7 +201,10 @@ def test_index_topk_toy():
 # ---------------------------------------------------------------------------
 # attention
 # ---------------------------------------------------------------------------
-def _attend_case(name, cfg_py, B, positions, n_c, sparse, win_cap, use_ws=True, idx=None, ws_bytes=None):
+def _attend_case(name, cfg_py, B, positions, n_c, sparse, win_cap, use_ws=True, idx=None, ws_bytes=None,
+                 pool_pad=0):
+    """One attend call against the oracle.  pool_pad > 0 lays the pool's
+    sequences out pool_pad elements further apart than [N_c, D] rows."""
     Tq = len(positions)
     H, D = cfg_py.n_heads, cfg_py.head_dim
     q = nb(f"{name}.q", (B, Tq, H, D))
@@ -216,15 +219,21 @@ def _attend_case(name, cfg_py, B, positions, n_c, sparse, win_cap, use_ws=True, 
         ws = ws_f32(ws_bytes)
     else:
         ws = ws_f32(L.ds4a_attend_workspace(cfg, B, Tq, n_c, sparse)) if use_ws else None
+    pool_d = bf(pool)
+    if pool_pad:
+        rows = pool.shape[1] * D
+        flat = torch.zeros(B * (rows + pool_pad), dtype=torch.bfloat16, device="cuda")
+        pool_d = flat.as_strided(tuple(pool.shape), (rows + pool_pad, D, 1))
+        pool_d.copy_(bf(pool))
     if sparse:
         if idx is None:
             n_vis = np.minimum((qpos + 1) // cfg_py.ratio, n_c)
             idx = host.random_subset_idx(SEED, f"{name}.idx", n_vis.ravel(), cfg_py.topk).reshape(B, Tq, -1)
-        L.ds4a_sparse_attend(cfg, i32(qpos), bf(q), f32(g), bf(pool), n_c, i32(idx), bf(win), win_cap, f32(sink),
+        L.ds4a_sparse_attend(cfg, i32(qpos), bf(q), f32(g), pool_d, n_c, i32(idx), bf(win), win_cap, f32(sink),
                              out, ws)
         ref = O.csa_attend_batch(q, g, pool, idx, win, win_cap, sink, qpos, cfg_py)
     else:
-        L.ds4a_hca_attend(cfg, i32(qpos), bf(q), f32(g), bf(pool), n_c, bf(win), win_cap, f32(sink), out, ws)
+        L.ds4a_hca_attend(cfg, i32(qpos), bf(q), f32(g), pool_d, n_c, bf(win), win_cap, f32(sink), out, ws)
         ref = O.hca_attend_batch(q, g, pool, n_c, win, win_cap, sink, qpos, cfg_py)
     check_ok()
     got = f64(out)
@@ -260,9 +269,20 @@ def test_attend_paths_used():
     # Flash shapes with the recommended workspace take the tensor-core
     # kernels; without a workspace the CUDA-core kernel runs
     names = kernels_used(lambda: _attend_case("path", FLASH, 1, [3999], 1000, True, 128))
-    assert "qhat_prep" in names and "attend_tc" in names, names
+    assert names == ["qhat_prep", "attend_tc", "attend_combine"], names
     names = kernels_used(lambda: _attend_case("path0", FLASH, 1, [3999], 1000, True, 128, use_ws=False))
     assert names == ["attend_generic"], names
+
+
+def test_attend_many_splits_and_empty_splits():
+    # 1093 visible HCA entries + 128 window keys = 10 tiles, split ten ways;
+    # beside it a query whose keys fill two tiles leaves eight splits empty
+    names = kernels_used(lambda: _attend_case("many", HCA, 1, [140000], 1100, False, 128))
+    assert names == ["qhat_prep", "attend_tc", "attend_combine"], names
+    _attend_case("two", HCA, 1, [130, 140000], 1100, False, 128)
+    # the CUDA-core path with a pool whose sequences are not a whole number
+    # of rows apart
+    _attend_case("gen", FLASH, 2, [0, 5, 127, 300, 3999], 1000, True, 128, use_ws=False, pool_pad=8)
 
 
 def test_swa_only_layer():

@@ -142,6 +142,11 @@ __device__ __forceinline__ const uint16_t* key_ptr(const AttendArgs& a, const It
   return a.win + (int64_t)it.b * a.win_bstride + (int64_t)(p % a.win_cap) * kD;
 }
 
+// kCompact: the issue loops (MMAs, gathers) stay rolled.  A decode block
+// runs each of them once with its code fetched cold, and the rolled loop is
+// a few cache lines instead of a few hundred instructions; a prefill block
+// runs them per tile with the code warm and keeps them unrolled.
+template <bool kCompact>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, int n_items,
                                                                 const uint8_t* qimg) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -385,11 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
         tc_fence_after();
         for (int tile = 0; tile < it.n_tiles; ++tile, ++gt) {
           const uint32_t d_s = tmem + (gt & 1u) * 64u;
-#pragma unroll
+#pragma unroll(kCompact ? 1 : 4)
           for (int c = 0; c < 4; ++c) {
             mbar_wait(bar(kKVFull0 + c), gt & 1u, abort_flag, err);
             tc_fence_after();
-#pragma unroll
+#pragma unroll(kCompact ? 2 : 8)
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t blk = 2u * c + (kk >> 2);
               const uint32_t koff = (uint32_t)(kk & 3) * 32u;
@@ -403,9 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
           if (tile == 0 && active > 0) mbar_wait(bar(kEpiDone), (active - 1) & 1u, abort_flag, err);
           tc_fence_after();
           const uint32_t acc0 = tile == 0 ? 0u : 1u;
-#pragma unroll
+#pragma unroll(kCompact ? 1 : 4)
           for (int c = 0; c < 4; ++c) {
-#pragma unroll
+#pragma unroll(kCompact ? 2 : 8)
             for (int kk = 0; kk < 8; ++kk)
               mma_bf16(tmem + 128u + 64u * c, pv_a0 + ((2u * c * 16384u + kk * 2048u) >> 4),
                        pv_b0 + ((kk * 2048u) >> 4), kIdescPV, kk == 0 ? acc0 : 1u);
@@ -445,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
       auto issue_chunk = [&](int c) {
         if (gt > 0) mbar_wait(bar(kKVEmpty0 + c), (gt - 1) & 1u, abort_flag, err);
         const uint32_t blk = kv_base + (uint32_t)(2 * c + (piece >> 3)) * 16384u;
-#pragma unroll
+#pragma unroll(kCompact ? 4 : 16)
         for (int i = 0; i < 16; ++i) {
           const int row = (pt >> 4) + 8 * i;
           const uint16_t* src = rowptr[row];
@@ -577,20 +582,23 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   // workspace: [rows x 64 KB q^ images][split partials]
   uint8_t* qimg = reinterpret_cast<uint8_t*>(a.ws);
   a.ws = reinterpret_cast<float*>(qimg + (size_t)rows * 65536u);
-  static int cache[16];
-  cudaError_t e = ensure_smem(attend_tc_kernel, (int)kSmemBytes, cache);
+  const int n_items = rows * a.n_splits;
+  const bool compact = n_items <= 148;  // every block takes at most one item
+  static int cache[16], cache_c[16];
+  cudaError_t e = compact ? ensure_smem(attend_tc_kernel<true>, (int)kSmemBytes, cache_c)
+                          : ensure_smem(attend_tc_kernel<false>, (int)kSmemBytes, cache);
   if (e != cudaSuccess) return e;
   {
     TraceScope tr("qhat_prep", s);
     e = launch_pdl(qhat_prep_kernel, dim3(rows, kH / 8), dim3(256), 0, s, a, qimg);
   }
   if (e != cudaSuccess) return e;
-  const int n_items = rows * a.n_splits;
   const int grid = min(n_items, 148);
   {
     TraceScope tr("attend_tc", s);
-    e = launch_pdl(attend_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, a, n_items,
-                   static_cast<const uint8_t*>(qimg));
+    const uint8_t* qi = qimg;
+    e = compact ? launch_pdl(attend_tc_kernel<true>, dim3(grid), dim3(kThreads), kSmemBytes, s, a, n_items, qi)
+                : launch_pdl(attend_tc_kernel<false>, dim3(grid), dim3(kThreads), kSmemBytes, s, a, n_items, qi);
   }
   if (e != cudaSuccess || a.n_splits == 1) return e;
   return launch_attend_combine(a, s);

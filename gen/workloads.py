@@ -80,6 +80,8 @@ WORKLOADS = {
     3: Workload(3, "hca_decode_b32_ctx128k", "hca_decode", 32, 131071, None, FLASH_HCA, 0, 1024),
     4: Workload(4, "csa_prefill_b1_t16k", "csa_prefill", 1, 16383, FLASH_CSA, None, 4096, 0),
     5: Workload(5, "mix_decode_b8_ctx1m", "mix_decode", 8, 1048575, FLASH_CSA, FLASH_HCA, 262144, 8192),
+    # a 4096-token prefill, small enough for multi-pass profiler captures
+    6: Workload(6, "csa_prefill_b1_t4k", "csa_prefill", 1, 4095, FLASH_CSA, None, 1024, 0),
 }
 
 

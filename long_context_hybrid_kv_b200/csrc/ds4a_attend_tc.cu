@@ -146,8 +146,20 @@ __device__ __forceinline__ const uint16_t* key_ptr(const AttendArgs& a, const It
 // runs each of them once with its code fetched cold, and the rolled loop is
 // a few cache lines instead of a few hundred instructions; a prefill block
 // runs them per tile with the code warm and keeps them unrolled.
+// omap: the output as rows of 512 bf16 ([B*T_q*64][512], box 128 dims x
+// 64 heads), written by TMA stores from the idle P^T buffer.
+// kvmap: the pool as rows of 512 bf16 (box 64 dims x 128 rows, 128-byte
+// swizzle) for the dense key ranges of HCA: a tile of 128 consecutive pool
+// entries comes in as eight TMA tile loads instead of 2048 gathered
+// 16-byte copies (pool_rows_b = rows per sequence; dense = 0: not used).
+struct DenseKV {
+  int dense;
+  int64_t pool_rows_b;
+};
+
 template <bool kCompact>
-__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, int n_items,
+__global__ void __launch_bounds__(kThreads, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap omap, const __grid_constant__ CUtensorMap kvmap, DenseKV dkv, AttendArgs a, int n_items,
                                                                 const uint8_t* qimg) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -312,6 +324,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
       // ---------------- epilogue ----------------
       mbar_wait(bar(kPVDone), (gt - 1) & 1u, abort_flag, err);
       tc_fence_after();
+      if (warp == 0 && w + (int)gridDim.x < n_items) {
+        // the next item's position and indices into L1 while this one's
+        // output goes out (its make_item then hits L1)
+        const int rn = (w + (int)gridDim.x) / a.n_splits;
+        if (lane < 16 && a.sparse && 32 * lane < a.k) prefetch_l1(a.idx + (int64_t)rn * a.k + 32 * lane);
+        if (lane == 16) prefetch_l1(a.q_pos + rn);
+      }
       red[q4 * 64 + h0 + lane] = warp_reduce32<false>(lpart);
       named_bar(1, 256);
       if (st < kH) {
@@ -329,9 +348,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
       named_bar(1, 256);
       float cs = 1.f, sn = 0.f;
       const int R = a.R;
-      // the final output goes out through the idle P^T buffer: [64 heads]
-      // [128 dims] bf16 per chunk, then 16-byte stores of whole rows
-      uint16_t* stage = reinterpret_cast<uint16_t*>(smem + kOffP);
+      // the final output goes out through the idle P^T buffer (16 KiB): per
+      // chunk [64 heads][128 dims] bf16, sent by one TMA store; split
+      // partials go straight to the workspace (coalesced 128-byte rows)
+      unsigned int* stage = reinterpret_cast<unsigned int*>(smem + kOffP);
+      const bool odd = r & 1;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         const int d = 128 * c + r;
@@ -341,25 +362,29 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
         tmem_ld32(t_lane + 128u + 64u * c + (uint32_t)h0, v);
         tmem_ld_wait();
         if (final_out) {
+          // lanes r and r^1 hold dims d and d^1: one exchange per head pair
+          // gives the even lane both dims of the even head and the odd lane
+          // both dims of the odd head, so each lane rotates its pair (rope
+          // slice, by -pos) and writes one 4-byte word
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int h = h0 + i;
-            float x = v[i] * inv_s[h];
-            const float y = __shfl_xor_sync(0xffffffffu, x, 1);
+          for (int i = 0; i < 32; i += 2) {
+            const float got = __shfl_xor_sync(0xffffffffu, odd ? v[i] : v[i + 1], 1);
+            const int h = h0 + i + (odd ? 1 : 0);
+            const float s = inv_s[h];
+            float x0 = (odd ? got : v[i]) * s, x1 = (odd ? v[i + 1] : got) * s;
             if (rot) {
-              // rotation by -pos: even dim (x, y) -> x cos + y sin; odd
-              // dim (y, x) -> -y sin + x cos
-              x = (d & 1) ? (x * cs - y * sn) : (x * cs + y * sn);
+              const float y0 = x0 * cs + x1 * sn, y1 = -x0 * sn + x1 * cs;
+              x0 = y0;
+              x1 = y1;
             }
-            stage[h * 128 + r] = f2bf(x);
+            stage[h * 64 + (r >> 1)] = f2_to_bf2x2(x0, x1);
           }
+          fence_async_smem();
           named_bar(1, 256);
-          uint16_t* orow = a.out + (int64_t)it.row * kH * kD + 128 * c;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int e = i * 256 + st;  // 16-byte piece: head e / 16, dims (e % 16) * 8 ..
-            const int h = e >> 4, q8 = (e & 15) * 8;
-            *reinterpret_cast<uint4*>(orow + h * kD + q8) = *reinterpret_cast<const uint4*>(stage + h * 128 + q8);
+          if (st == 0) {
+            tma_store_2d(&omap, p_base, 128 * c, it.row * kH);
+            bulk_commit();
+            bulk_wait_read();  // the buffer is free again
           }
           named_bar(1, 256);
         } else {
@@ -432,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
     // =================== producers ===================
     const int pt = tid - kPG0;  // 0..127
     uint32_t gt = 0, active = 0;
+    bool tma_used = false;
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       const Item it = make_item(a, w);
       if (it.n_tiles == 0) continue;
@@ -472,6 +498,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
       // Two chunks stay in flight: chunk c goes out, then chunk c-1 is
       // retired (a deeper queue over-subscribes L2 across the SMs).
       for (int tile = 0; tile < it.n_tiles; ++tile, ++gt) {
+        const int s0 = it.j0 + tile * kKT;
+        if (dkv.dense && !a.sparse && s0 + kKT <= it.n_sel) {
+          // 128 consecutive pool entries: one thread arms each chunk's
+          // barrier with its bytes and starts two TMA tile loads, the
+          // others arrive
+          const int y = (int)(it.b * dkv.pool_rows_b + s0);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            if (gt > 0) mbar_wait(bar(kKVEmpty0 + c), (gt - 1) & 1u, abort_flag, err);
+            if (pt == 0) {
+              mbar_expect_tx(bar(kKVFull0 + c), 32768u);
+              tma_load_2d(kv_base + (uint32_t)(2 * c) * 16384u, &kvmap, 128 * c, y, bar(kKVFull0 + c));
+              tma_load_2d(kv_base + (uint32_t)(2 * c + 1) * 16384u, &kvmap, 128 * c + 64, y, bar(kKVFull0 + c));
+              tma_used = true;
+            } else {
+              mbar_arrive(bar(kKVFull0 + c));
+            }
+          }
+          continue;
+        }
         set_rowptr(tile);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -489,8 +535,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendArgs a, in
       ++active;
     }
     cp_async_wait<0>();  // nothing of this block is in flight at exit
+    if (pt == 0 && tma_used)
+      for (int c = 0; c < 4; ++c) mbar_drain(bar(kKVFull0 + c), (gt - 1) & 1u);
   }
 
+  if (tid == 0) bulk_wait_all();  // the output stores have landed
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -593,12 +642,46 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
     e = launch_pdl(qhat_prep_kernel, dim3(rows, kH / 8), dim3(256), 0, s, a, qimg);
   }
   if (e != cudaSuccess) return e;
+  CUtensorMap omap;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+  if (!encode) return cudaErrorNotSupported;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows * kH};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {128, (cuuint32_t)kH};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  // HCA keys are consecutive pool entries: a row view of the pool for TMA
+  // tile loads (when the sequences are a whole number of rows apart)
+  CUtensorMap kvmap;
+  memset(&kvmap, 0, sizeof(kvmap));
+  DenseKV dkv;
+  dkv.dense = 0;
+  dkv.pool_rows_b = a.B > 1 ? a.pool_bstride / kD : 0;
+  const int64_t pool_rows = (int64_t)(a.B - 1) * dkv.pool_rows_b + a.N_c;
+  if (!a.sparse && a.N_c >= kKT && (a.B == 1 || a.pool_bstride % kD == 0) && pool_rows < INT32_MAX) {
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)pool_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kKT};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&kvmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.pool), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    dkv.dense = 1;
+  }
   const int grid = min(n_items, 148);
   {
     TraceScope tr("attend_tc", s);
     const uint8_t* qi = qimg;
-    e = compact ? launch_pdl(attend_tc_kernel<true>, dim3(grid), dim3(kThreads), kSmemBytes, s, a, n_items, qi)
-                : launch_pdl(attend_tc_kernel<false>, dim3(grid), dim3(kThreads), kSmemBytes, s, a, n_items, qi);
+    e = compact ? launch_pdl(attend_tc_kernel<true>, dim3(grid), dim3(kThreads), kSmemBytes, s, omap, kvmap,
+                             dkv, a, n_items, qi)
+                : launch_pdl(attend_tc_kernel<false>, dim3(grid), dim3(kThreads), kSmemBytes, s, omap, kvmap,
+                             dkv, a, n_items, qi);
   }
   if (e != cudaSuccess || a.n_splits == 1) return e;
   return launch_attend_combine(a, s);

@@ -21,6 +21,7 @@ namespace ds4a {
 // vectors of 8 bf16 when c is a multiple of 8.
 // ===========================================================================
 constexpr int kCompressThreads = 512;
+constexpr float kLog2eC = 1.4426950408889634f;
 
 template <int V>
 struct VecLoad;
@@ -98,17 +99,19 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
         if (t0 + u * G >= n_terms) break;
 #pragma unroll
         for (int q = 0; q < V; ++q) {
-          const float x = zs[u][q] + bs[u][q];
-          if (x > mx[q]) {
-            const float sc = __expf(mx[q] - x);
-            l[q] = l[q] * sc + 1.f;
-            acc[q] = acc[q] * sc + vals[u][q];
+          // log2 units; the reference moves only when a logit passes it by
+          // more than 2^8 (always for the first term), so the common step
+          // is one exp2 and two FMAs
+          const float x = (zs[u][q] + bs[u][q]) * kLog2eC;
+          if (x > mx[q] + 8.f) {
+            const float sc = ex2_approx(mx[q] - x);  // 0 while empty
+            l[q] *= sc;
+            acc[q] *= sc;
             mx[q] = x;
-          } else {
-            const float e = __expf(x - mx[q]);
-            l[q] += e;
-            acc[q] += e * vals[u][q];
           }
+          const float e = ex2_approx(x - mx[q]);
+          l[q] += e;
+          acc[q] = fmaf(e, vals[u][q], acc[q]);
         }
       }
     }
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
     for (int gg = 0; gg < G; ++gg) {
       const float mm = s_m[gg * c + ch];
       if (mm == -INFINITY) continue;
-      const float e = __expf(mm - M);
+      const float e = ex2_approx(mm - M);
       Ls += s_l[gg * c + ch] * e;
       A += s_a[gg * c + ch] * e;
     }

@@ -23,19 +23,22 @@ __device__ __forceinline__ void raise_err(unsigned int* w, unsigned int bits) { 
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf2f(uint16_t u) { return __uint_as_float(((unsigned int)u) << 16); }
 
+// round-to-nearest-even conversions (one cvt instruction each)
 __device__ __forceinline__ uint16_t f2bf(float f) {
-  // round-to-nearest-even (inputs here are finite)
-  unsigned int b = __float_as_uint(f);
-  b += 0x7FFFu + ((b >> 16) & 1u);
-  return (uint16_t)(b >> 16);
+  uint16_t u;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(u) : "f"(f));
+  return u;
 }
 
 __device__ __forceinline__ float2 bf2x2_to_f2(unsigned int w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
+// a in the low half, b in the high half
 __device__ __forceinline__ unsigned int f2_to_bf2x2(float a, float b) {
-  return (unsigned int)f2bf(a) | ((unsigned int)f2bf(b) << 16);
+  unsigned int u;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(b), "f"(a));
+  return u;
 }
 
 // RoPE frequencies theta_j = base^(-2j/R), j < R/2, divided by pi and
@@ -68,6 +71,13 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // order-preserving map float -> uint32 (larger float -> larger key)
+// 2^x with the hardware approximation (about 2 ulp)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ unsigned int f2key(float f) {
   unsigned int b = __float_as_uint(f);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);

@@ -4,9 +4,16 @@
 // bf16 inputs, fp32 accumulators), commits, proxy fences and cp.async.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "ds4a_internal.cuh"
 
 namespace ds4a {
+
+// the driver's cuTensorMapEncodeTiled (null when unavailable)
+PFN_cuTensorMapEncodeTiled_v12000 get_encode();
+
 namespace tc {
 
 // A bounded wait gives up after this many SM cycles (about 2 s at 1.9 GHz),
@@ -57,6 +64,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       }
     }
   }
+}
+
+// Wait, with the same bound but regardless of the abort flag, for a phase
+// that this thread's async copies complete: a block never exits with copies
+// into its shared memory still in flight.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return;
 }
 
 __device__ __forceinline__ void fence_barrier_init() {
@@ -226,13 +242,45 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
                : "memory");
 }
 
-// 2^x with the hardware approximation (about 2 ulp; the softmax weights are
-// rounded to bf16 right after)
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
+// TMA loads of a box (tiled mode, no multicast) into this block's shared
+// memory; complete as transaction bytes on the mbarrier.  x * element size
+// must be a multiple of 16.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
 }
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// TMA store of a shared-memory box (tensor map without swizzle) to global
+// memory at non-negative coordinates whose x * element size is a multiple
+// of 16; the bulk group completes when the data has been read (wait_read)
+// or written (wait_all).
+__device__ __forceinline__ void tma_store_2d(const void* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// hint: bring the 128-byte line holding p into this SM's L1
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 
 // 128-byte swizzle inside a 1024-byte atom: 16-byte chunk c of row r
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {

@@ -14,7 +14,9 @@
 //   topk_cluster_kernel  one 8-block cluster per row (rows up to 262144):
 //                        each block stages a slice; histograms and the
 //                        compaction offsets are summed over the cluster
-//                        through distributed shared memory
+//                        through distributed shared memory; a first select
+//                        over the per-thread maxima gives a floor below
+//                        which the main select need not count
 //   topk_global_kernel   one block per row, every pass reading the scores
 //                        from global memory (any length)
 #include <cooperative_groups.h>
@@ -93,6 +95,13 @@ __device__ __forceinline__ void find_digit(const unsigned int* hist, int remaini
   }
 }
 
+// Shared-memory slot of key i: XOR-swizzled inside each group of 32 so that
+// both the strided passes (thread t reads i = t + j * blockDim) and the
+// ordered walks (thread t reads its own run i = t * run + j) are free of
+// bank conflicts (a plain layout put a run's 32 threads in one bank).  The
+// array is sized to whole groups of 32.
+__device__ __forceinline__ int kpos(int i) { return i ^ ((i >> 5) & 31); }
+
 __device__ __forceinline__ void write_identity(const IndexArgs& a, int n_vis, const float* sc, int32_t* out,
                                                float* so) {
   for (int i = threadIdx.x; i < a.k; i += blockDim.x) {
@@ -121,7 +130,7 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
     write_identity(a, n_vis, sc, out, so);
     return;
   }
-  for (int i = tid; i < n_vis; i += blockDim.x) keys[i] = f2key(sc[i]);
+  for (int i = tid; i < n_vis; i += blockDim.x) keys[kpos(i)] = f2key(sc[i]);
   unsigned int prefix = 0, mask = 0;
   int remaining = a.k;
   for (int pass = 0; pass < 4; ++pass) {
@@ -129,7 +138,7 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
     for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     for (int i = tid; i < n_vis; i += blockDim.x) {
-      const unsigned int u = keys[i];
+      const unsigned int u = keys[kpos(i)];
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
     }
     __syncthreads();
@@ -146,7 +155,7 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
   const int i0 = min(n_vis, tid * run), i1 = min(n_vis, i0 + run);
   int gt = 0, eq = 0;
   for (int i = i0; i < i1; ++i) {
-    const unsigned int u = keys[i];
+    const unsigned int u = keys[kpos(i)];
     gt += u > T;
     eq += u == T;
   }
@@ -156,7 +165,7 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
   const int sel_before = block_incl_scan(gt + take_eq, s_warp, &tot) - (gt + take_eq);
   int o = sel_before, tr = eq_before;
   for (int i = i0; i < i1; ++i) {
-    const unsigned int u = keys[i];
+    const unsigned int u = keys[kpos(i)];
     bool keep = u > T;
     if (u == T) keep = tr++ < need;
     if (keep) {
@@ -177,6 +186,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   __shared__ int s_tot[2];  // this block's tie count, kept count
   __shared__ unsigned int s_digit;
   __shared__ int s_above;
+  __shared__ unsigned int tmaxs[kClusterThreads];
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
   const int row = blockIdx.x / kCluster, tid = threadIdx.x;
@@ -197,31 +207,57 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   const int slice = (n_vis + kCluster - 1) / kCluster;
   const int lo = min(n_vis, rank * slice), hi = min(n_vis, lo + slice);
   const int n = hi - lo;
-  for (int i = tid; i < n; i += blockDim.x) keys[i] = f2key(sc[lo + i]);
-  unsigned int prefix = 0, mask = 0;
-  int remaining = a.k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < n; i += blockDim.x) {
-      const unsigned int u = keys[i];
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
-    }
-    cl.sync();  // every block's histogram is complete
-    if (tid < 256) {
-      unsigned int s = 0;
-#pragma unroll
-      for (int r = 0; r < kCluster; ++r) s += cl.map_shared_rank(hist, r)[tid];
-      hist_all[tid] = s;
-    }
-    __syncthreads();
-    find_digit(hist_all, remaining, &s_digit, &s_above);
-    cl.sync();  // peers are done reading this block's histogram
-    prefix |= s_digit << shift;
-    mask |= 255u << shift;
-    remaining -= s_above;
+  // stage the slice; thread t's keys are t, t + 1024, ...: keep their max
+  unsigned int tmax = 0u;
+  for (int i = tid; i < n; i += blockDim.x) {
+    const unsigned int u = f2key(sc[lo + i]);
+    keys[kpos(i)] = u;
+    tmax = max(tmax, u);
   }
+  tmaxs[tid] = tmax;
+  // Radix select over the cluster (k-th largest of vals[0..nv) in every
+  // block, counting only values >= floor): the key T and how many of the
+  // values equal to T are needed.
+  auto cluster_select = [&](const unsigned int* vals, bool swz, int nv, unsigned int floor, unsigned int* T_out,
+                            int* need_out) {
+    unsigned int prefix = 0, mask = 0;
+    int remaining = a.k;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < nv; i += blockDim.x) {
+        const unsigned int u = vals[swz ? kpos(i) : i];
+        if (u >= floor && (u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      }
+      cl.sync();  // every block's histogram is complete
+      if (tid < 256) {
+        unsigned int sum = 0;
+#pragma unroll
+        for (int r = 0; r < kCluster; ++r) sum += cl.map_shared_rank(hist, r)[tid];
+        hist_all[tid] = sum;
+      }
+      __syncthreads();
+      find_digit(hist_all, remaining, &s_digit, &s_above);
+      cl.sync();  // peers are done reading this block's histogram
+      prefix |= s_digit << shift;
+      mask |= 255u << shift;
+      remaining -= s_above;
+    }
+    *T_out = prefix;
+    *need_out = remaining;
+  };
+  // The k-th largest of the cluster's 8192 per-thread maxima is a floor
+  // with at least k keys at or above it (each of those k threads holds
+  // one), so the k-th largest key is at or above it too and the select over
+  // the keys can skip everything below: its histogram passes then count
+  // about a thousand keys instead of the whole row.
+  unsigned int floor_key;
+  int unused;
+  cluster_select(tmaxs, false, (int)blockDim.x, 0u, &floor_key, &unused);
+  unsigned int prefix;
+  int remaining;
+  cluster_select(keys, true, n, floor_key, &prefix, &remaining);
   const unsigned int T = prefix;
   const int need = remaining;
   // ordered compaction across the cluster: block r holds indices
@@ -230,7 +266,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   const int i0 = min(n, tid * run), i1 = min(n, i0 + run);
   int gt = 0, eq = 0;
   for (int i = i0; i < i1; ++i) {
-    const unsigned int u = keys[i];
+    const unsigned int u = keys[kpos(i)];
     gt += u > T;
     eq += u == T;
   }
@@ -250,7 +286,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   for (int r = 0; r < rank; ++r) sel_base += cl.map_shared_rank(s_tot, r)[1];
   int o = sel_base + sel_local, tr = eq_before;
   for (int i = i0; i < i1; ++i) {
-    const unsigned int u = keys[i];
+    const unsigned int u = keys[kpos(i)];
     bool keep = u > T;
     if (u == T) keep = tr++ < need;
     if (keep) {
@@ -327,7 +363,7 @@ cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
   const int rows = a.B * a.T_q;
   if (rows <= 0) return cudaSuccess;
   if (a.N_c <= kSmemRowMax) {
-    const size_t smem = (size_t)max(1, a.N_c) * sizeof(unsigned int);
+    const size_t smem = (size_t)((max(1, a.N_c) + 31) & ~31) * sizeof(unsigned int);
     static int cache[16];
     cudaError_t e = ensure_smem(topk_smem_kernel, (int)smem, cache);
     if (e != cudaSuccess) return e;

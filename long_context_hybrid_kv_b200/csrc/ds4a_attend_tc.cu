@@ -57,7 +57,8 @@ constexpr uint32_t kOffRed = kOffRowPtr + 1024;     // [4][64] floats
 constexpr uint32_t kOffMrun = kOffRed + 1024;       // [64]
 constexpr uint32_t kOffAlpha = kOffMrun + 256;      // [64]
 constexpr uint32_t kOffInv = kOffAlpha + 256;       // [64]
-constexpr uint32_t kSmemBytes = kOffInv + 256 + 1024;  // + alignment slack
+constexpr uint32_t kOffSink = kOffInv + 256;        // [64] sink * log2(e)
+constexpr uint32_t kSmemBytes = kOffSink + 256 + 1024;  // + alignment slack
 
 enum Bar {
   kQFull = 0, kQEmpty, kKVFull0, kKVFull1, kKVFull2, kKVFull3, kKVEmpty0, kKVEmpty1, kKVEmpty2,
@@ -67,6 +68,8 @@ enum Bar {
 constexpr uint32_t kIdescQK = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 64, 1, 1);
 
+// Key slots of an item: its selected (or, for HCA, visible) entries, then
+// the window rows.
 struct Item {
   int row, split, b, pos;
   int n_sel, win_start, j0, j1, n_tiles;
@@ -142,6 +145,7 @@ __device__ __forceinline__ const uint16_t* key_ptr(const AttendArgs& a, const It
   return a.win + (int64_t)it.b * a.win_bstride + (int64_t)(p % a.win_cap) * kD;
 }
 
+
 // kCompact: the issue loops (MMAs, gathers) stay rolled.  A decode block
 // runs each of them once with its code fetched cold, and the rolled loop is
 // a few cache lines instead of a few hundred instructions; a prefill block
@@ -175,13 +179,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* mrun = reinterpret_cast<float*>(smem + kOffMrun);
   float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);
   float* inv_s = reinterpret_cast<float*>(smem + kOffInv);
+  float* sink_s = reinterpret_cast<float*>(smem + kOffSink);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bar(kQFull), 1);
+    // decode-sized launches (kCompact): the softmax warps prepare q^ in the
+    // kernel and all 256 arrive; otherwise one bulk copy of the prepared
+    // image arrives with its bytes
+    mbar_init(bar(kQFull), kCompact ? 256 : 1);
     mbar_init(bar(kQEmpty), 1);
     for (int c = 0; c < 4; ++c) {
       mbar_init(bar(kKVFull0 + c), 128);
@@ -216,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h0 = 32 * hf;
     const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
     const float scale2 = a.scale * kLog2e;
+    if (st < kH) sink_s[st] = a.sink[st] * kLog2e;  // read by the epilogues (after a named barrier)
     uint32_t gt = 0, active = 0;
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       const Item it = make_item(a, w);
@@ -236,6 +245,77 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = st; e < kH * kD; e += 256) part[2 * kH + e] = 0.f;
         }
         continue;
+      }
+      if (kCompact) {
+        // q^ = RoPE_pos(RMSNorm(q) * g) of this block's (only) query,
+        // straight into the operand layout while the K=V rows are on their
+        // way: warp w takes heads w, w + 8, ..., four heads' rows in flight
+        // per round; lane l holds dims 8l..8l+7 and 256+8l..256+8l+7
+        const uint16_t* qrow = a.q + (int64_t)it.row * kH * kD;
+        float rc[4], rs[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          rc[u] = 1.f;
+          rs[u] = 0.f;
+          const int d = 256 + 8 * lane + 2 * u;
+          if (d >= kD - a.R) rope_cos_sin(it.pos, a.rope.t[(d - (kD - a.R)) >> 1], &rc[u], &rs[u]);
+        }
+        const float4 g0 = *reinterpret_cast<const float4*>(a.q_norm_g + 8 * lane);
+        const float4 g1 = *reinterpret_cast<const float4*>(a.q_norm_g + 8 * lane + 4);
+        const float4 g2 = *reinterpret_cast<const float4*>(a.q_norm_g + 256 + 8 * lane);
+        const float4 g3 = *reinterpret_cast<const float4*>(a.q_norm_g + 256 + 8 * lane + 4);
+        const float g[16] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w,
+                             g2.x, g2.y, g2.z, g2.w, g3.x, g3.y, g3.z, g3.w};
+        const uint32_t offA = (uint32_t)(lane >> 3) * 8192u, offB = (uint32_t)(4 + (lane >> 3)) * 8192u;
+#pragma unroll 1
+        for (int h4 = warp; h4 < kH; h4 += 32) {
+          uint4 va[4], vb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint16_t* hp = qrow + (h4 + 8 * u) * kD;
+            va[u] = *reinterpret_cast<const uint4*>(hp + 8 * lane);
+            vb[u] = *reinterpret_cast<const uint4*>(hp + 256 + 8 * lane);
+          }
+          float ss[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const unsigned int wv[8] = {va[u].x, va[u].y, va[u].z, va[u].w, vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+            float acc = 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float2 f = bf2x2_to_f2(wv[q]);
+              acc = fmaf(f.x, f.x, fmaf(f.y, f.y, acc));
+            }
+            ss[u] = acc;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int h = h4 + 8 * u;
+            const float rstd = rsqrtf(ss[u] / (float)kD + a.eps);
+            const unsigned int wv[8] = {va[u].x, va[u].y, va[u].z, va[u].w, vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+            uint32_t pq[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float2 f = bf2x2_to_f2(wv[q]);
+              float x0 = f.x * rstd * g[2 * q], x1 = f.y * rstd * g[2 * q + 1];
+              if (q >= 4) {
+                const float y0 = x0 * rc[q - 4] - x1 * rs[q - 4], y1 = x0 * rs[q - 4] + x1 * rc[q - 4];
+                x0 = y0;
+                x1 = y1;
+              }
+              pq[q] = f2_to_bf2x2(x0, x1);
+            }
+            const uint32_t sw = sw128((uint32_t)h, (uint32_t)(lane & 7));
+            st_shared16(q_base + offA + sw, pq[0], pq[1], pq[2], pq[3]);
+            st_shared16(q_base + offB + sw, pq[4], pq[5], pq[6], pq[7]);
+          }
+        }
+        fence_async_smem();
+        mbar_arrive(bar(kQFull));
       }
       if (st < kH) mrun[st] = -INFINITY;
       float lpart[32];
@@ -337,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l = red[st] + red[64 + st] + red[128 + st] + red[192 + st];
         const float m = mrun[st];
         if (final_out) {
-          const float den = (m == -INFINITY) ? 0.f : l + exp2f(a.sink[st] * kLog2e - m);
+          const float den = (m == -INFINITY) ? 0.f : l + exp2f(sink_s[st] - m);
           inv_s[st] = den > 0.f ? 1.f / den : 0.f;
         } else {
           float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
@@ -488,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // ---- q^ (prepared by qhat_prep_kernel in the shared-memory image
       // layout): one 64 KB bulk copy once the previous item's QK is done ----
-      if (pt == 0) {
+      if (!kCompact && pt == 0) {
         if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
         mbar_expect_tx(bar(kQFull), 65536u);
         bulk_g2s(q_base, qimg + (size_t)it.row * 65536u, 65536u, bar(kQFull));
@@ -637,11 +717,12 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   cudaError_t e = compact ? ensure_smem(attend_tc_kernel<true>, (int)kSmemBytes, cache_c)
                           : ensure_smem(attend_tc_kernel<false>, (int)kSmemBytes, cache);
   if (e != cudaSuccess) return e;
-  {
+  if (!compact) {
+    // decode-sized launches prepare q^ inside the attention kernel
     TraceScope tr("qhat_prep", s);
     e = launch_pdl(qhat_prep_kernel, dim3(rows, kH / 8), dim3(256), 0, s, a, qimg);
+    if (e != cudaSuccess) return e;
   }
-  if (e != cudaSuccess) return e;
   CUtensorMap omap;
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
   if (!encode) return cudaErrorNotSupported;

@@ -269,7 +269,7 @@ def test_attend_paths_used():
     # Flash shapes with the recommended workspace take the tensor-core
     # kernels; without a workspace the CUDA-core kernel runs
     names = kernels_used(lambda: _attend_case("path", FLASH, 1, [3999], 1000, True, 128))
-    assert names == ["qhat_prep", "attend_tc", "attend_combine"], names
+    assert names == ["attend_tc", "attend_combine"], names  # decode-sized: q^ inside the kernel
     names = kernels_used(lambda: _attend_case("path0", FLASH, 1, [3999], 1000, True, 128, use_ws=False))
     assert names == ["attend_generic"], names
 
@@ -278,11 +278,26 @@ def test_attend_many_splits_and_empty_splits():
     # 1093 visible HCA entries + 128 window keys = 10 tiles, split ten ways;
     # beside it a query whose keys fill two tiles leaves eight splits empty
     names = kernels_used(lambda: _attend_case("many", HCA, 1, [140000], 1100, False, 128))
-    assert names == ["qhat_prep", "attend_tc", "attend_combine"], names
+    assert names == ["attend_tc", "attend_combine"], names
     _attend_case("two", HCA, 1, [130, 140000], 1100, False, 128)
     # the CUDA-core path with a pool whose sequences are not a whole number
     # of rows apart
     _attend_case("gen", FLASH, 2, [0, 5, 127, 300, 3999], 1000, True, 128, use_ws=False, pool_pad=8)
+
+
+def test_attend_prefill_sized_launches():
+    # more than 148 queries: the prefill form of the kernel (work items
+    # round-robin over the blocks, selected rows gathered by TMA gather4 in
+    # groups of four slots, padding slots masked); positions cover empty,
+    # partial and full windows and selected counts that are not multiples
+    # of four
+    pos = sorted(set([0, 1, 2, 3, 5, 6, 7, 126, 127, 128, 129, 130, 131] + list(range(200, 3999, 23))))
+    assert len(pos) > 148
+    _attend_case("pf", FLASH, 1, pos, 1000, True, 4096)
+    # HCA over consecutive pool entries (whole tiles by TMA tile loads) in
+    # the prefill form
+    hpos = list(range(16383, 16383 + 160 * 131, 131))
+    _attend_case("pfh", HCA, 1, hpos, 300, False, 512)
 
 
 def test_swa_only_layer():

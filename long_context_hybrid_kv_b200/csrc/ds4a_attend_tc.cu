@@ -628,15 +628,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // q^ = RoPE_pos(RMSNorm(q_h) * g) for every query, written as the
 // shared-memory image attend_tc_kernel copies in: 8 blocks of 64 dims, each
-// [64 heads][128 B] with the 128-byte swizzle.  Block = (query, 8 heads),
-// warp = head, lane = dims 8l..8l+7 and 256+8l..256+8l+7.
+// [64 heads][128 B] with the 128-byte swizzle.  Block = (query, 16 heads),
+// warp = two heads, lane = dims 8l..8l+7 and 256+8l..256+8l+7.
 __global__ void __launch_bounds__(256) qhat_prep_kernel(AttendArgs a, uint8_t* qimg) {
   __shared__ float2 rt[64];
   const int row = blockIdx.x;
-  const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
   pdl_wait();
+  // every load goes out before any of them is used: the two heads' rows
+  // (heads 16 y + w and 16 y + 8 + w), this lane's gains, the position
+  const uint16_t* qrow = a.q + (int64_t)row * kH * kD;
+  uint4 v[2][2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int h = blockIdx.y * 16 + 8 * u + warp;
+    v[u][0] = *reinterpret_cast<const uint4*>(qrow + h * kD + 8 * lane);
+    v[u][1] = *reinterpret_cast<const uint4*>(qrow + h * kD + 256 + 8 * lane);
+  }
+  float g[16];
+  {
+    const float4 g0 = *reinterpret_cast<const float4*>(a.q_norm_g + 8 * lane);
+    const float4 g1 = *reinterpret_cast<const float4*>(a.q_norm_g + 8 * lane + 4);
+    const float4 g2 = *reinterpret_cast<const float4*>(a.q_norm_g + 256 + 8 * lane);
+    const float4 g3 = *reinterpret_cast<const float4*>(a.q_norm_g + 256 + 8 * lane + 4);
+    const float t[16] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w, g2.x, g2.y, g2.z, g2.w, g3.x, g3.y, g3.z, g3.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) g[i] = t[i];
+  }
   const int pos = a.q_pos[row];
   const int R = a.R;
   for (int j = threadIdx.x; j < R / 2; j += blockDim.x) {
@@ -645,47 +664,46 @@ __global__ void __launch_bounds__(256) qhat_prep_kernel(AttendArgs a, uint8_t* q
     rt[j] = make_float2(cs, sn);
   }
   __syncthreads();
-  const uint16_t* qrow = a.q + (int64_t)row * kH * kD + h * kD;
-  const uint4 va = *reinterpret_cast<const uint4*>(qrow + 8 * lane);
-  const uint4 vb = *reinterpret_cast<const uint4*>(qrow + 256 + 8 * lane);
-  float x[16];
-  const unsigned int wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float2 fa = bf2x2_to_f2(wa[q]), fb = bf2x2_to_f2(wb[q]);
-    x[2 * q] = fa.x;
-    x[2 * q + 1] = fa.y;
-    x[8 + 2 * q] = fb.x;
-    x[8 + 2 * q + 1] = fb.y;
-  }
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) ss += x[i] * x[i];
-  ss = warp_sum(ss);
-  const float rstd = rsqrtf(ss / (float)kD + a.eps);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int d = i < 8 ? 8 * lane + i : 256 + 8 * lane + (i - 8);
-    x[i] = x[i] * rstd * a.q_norm_g[d];
-  }
-#pragma unroll
-  for (int pr = 0; pr < 8; ++pr) {
-    const int i = 2 * pr;
-    const int d = i < 8 ? 8 * lane + i : 256 + 8 * lane + (i - 8);
-    if (d >= kD - R) {
-      const float2 t = rt[(d - (kD - R)) >> 1];
-      const float x0 = x[i], x1 = x[i + 1];
-      x[i] = x0 * t.x - x1 * t.y;
-      x[i + 1] = x0 * t.y + x1 * t.x;
-    }
-  }
   uint8_t* img = qimg + (size_t)row * 65536u;
-  const uint32_t offA = (uint32_t)(lane >> 3) * 8192u + sw128(h, lane & 7);
-  const uint32_t offB = (uint32_t)(4 + (lane >> 3)) * 8192u + sw128(h, lane & 7);
-  *reinterpret_cast<uint4*>(img + offA) = make_uint4(f2_to_bf2x2(x[0], x[1]), f2_to_bf2x2(x[2], x[3]),
-                                                     f2_to_bf2x2(x[4], x[5]), f2_to_bf2x2(x[6], x[7]));
-  *reinterpret_cast<uint4*>(img + offB) = make_uint4(f2_to_bf2x2(x[8], x[9]), f2_to_bf2x2(x[10], x[11]),
-                                                     f2_to_bf2x2(x[12], x[13]), f2_to_bf2x2(x[14], x[15]));
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int h = blockIdx.y * 16 + 8 * u + warp;
+    float x[16];
+    const unsigned int wa[4] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w};
+    const unsigned int wb[4] = {v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 fa = bf2x2_to_f2(wa[q]), fb = bf2x2_to_f2(wb[q]);
+      x[2 * q] = fa.x;
+      x[2 * q + 1] = fa.y;
+      x[8 + 2 * q] = fb.x;
+      x[8 + 2 * q + 1] = fb.y;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ss += x[i] * x[i];
+    ss = warp_sum(ss);
+    const float rstd = rsqrtf(ss / (float)kD + a.eps);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = x[i] * rstd * g[i];
+#pragma unroll
+    for (int pr = 0; pr < 8; ++pr) {
+      const int i = 2 * pr;
+      const int d = i < 8 ? 8 * lane + i : 256 + 8 * lane + (i - 8);
+      if (d >= kD - R) {
+        const float2 t = rt[(d - (kD - R)) >> 1];
+        const float x0 = x[i], x1 = x[i + 1];
+        x[i] = x0 * t.x - x1 * t.y;
+        x[i + 1] = x0 * t.y + x1 * t.x;
+      }
+    }
+    const uint32_t offA = (uint32_t)(lane >> 3) * 8192u + sw128(h, lane & 7);
+    const uint32_t offB = (uint32_t)(4 + (lane >> 3)) * 8192u + sw128(h, lane & 7);
+    *reinterpret_cast<uint4*>(img + offA) = make_uint4(f2_to_bf2x2(x[0], x[1]), f2_to_bf2x2(x[2], x[3]),
+                                                       f2_to_bf2x2(x[4], x[5]), f2_to_bf2x2(x[6], x[7]));
+    *reinterpret_cast<uint4*>(img + offB) = make_uint4(f2_to_bf2x2(x[8], x[9]), f2_to_bf2x2(x[10], x[11]),
+                                                       f2_to_bf2x2(x[12], x[13]), f2_to_bf2x2(x[14], x[15]));
+  }
 }
 
 }  // namespace
@@ -720,7 +738,7 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   if (!compact) {
     // decode-sized launches prepare q^ inside the attention kernel
     TraceScope tr("qhat_prep", s);
-    e = launch_pdl(qhat_prep_kernel, dim3(rows, kH / 8), dim3(256), 0, s, a, qimg);
+    e = launch_pdl(qhat_prep_kernel, dim3(rows, kH / 16), dim3(256), 0, s, a, qimg);
     if (e != cudaSuccess) return e;
   }
   CUtensorMap omap;

@@ -58,7 +58,8 @@ constexpr uint32_t kOffMrun = kOffRed + 1024;       // [64]
 constexpr uint32_t kOffAlpha = kOffMrun + 256;      // [64]
 constexpr uint32_t kOffInv = kOffAlpha + 256;       // [64]
 constexpr uint32_t kOffSink = kOffInv + 256;        // [64] sink * log2(e)
-constexpr uint32_t kSmemBytes = kOffSink + 256 + 1024;  // + alignment slack
+constexpr uint32_t kOffNext = kOffSink + 256;       // the softmax warps' next work item
+constexpr uint32_t kSmemBytes = kOffNext + 64 + 1024;  // + alignment slack
 
 enum Bar {
   kQFull = 0, kQEmpty, kKVFull0, kKVFull1, kKVFull2, kKVFull3, kKVEmpty0, kKVEmpty1, kKVEmpty2,
@@ -225,9 +226,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
     const float scale2 = a.scale * kLog2e;
     if (st < kH) sink_s[st] = a.sink[st] * kLog2e;  // read by the epilogues (after a named barrier)
+    // Warp 0 builds the next work item during the current item's last tile
+    // (its loads overlap the wait for S^T) and leaves it in shared memory;
+    // every softmax thread picks it up after the epilogue's last barrier.
+    Item* s_next = reinterpret_cast<Item*>(smem + kOffNext);
     uint32_t gt = 0, active = 0;
+    Item it;
+    if (!kCompact && (int)blockIdx.x < n_items) it = make_item(a, blockIdx.x);
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
-      const Item it = make_item(a, w);
+      const int wn = w + (int)gridDim.x;
+      if (kCompact) it = make_item(a, w);  // one item per block
+      else if (w != (int)blockIdx.x) it = *s_next;
       const bool final_out = a.n_splits == 1;
       if (it.pos < 0 && st == 0 && it.split == 0) raise_err(err, DS4A_DEV_BAD_POS);
       if (it.n_tiles == 0) {
@@ -243,6 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             part[kH + st] = 0.f;
           }
           for (int e = st; e < kH * kD; e += 256) part[2 * kH + e] = 0.f;
+        }
+        if (!kCompact && wn < n_items) {
+          named_bar(1, 256);  // every softmax thread has read *s_next
+          if (warp == 0) {
+            const Item nx = make_item(a, wn);
+            if (lane == 0) *s_next = nx;
+          }
+          named_bar(1, 256);
         }
         continue;
       }
@@ -324,6 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(1, 256);
       for (int tile = 0; tile < it.n_tiles; ++tile, ++gt) {
         const uint32_t sb = gt & 1u;
+        if (!kCompact && tile == it.n_tiles - 1 && warp == 0 && wn < n_items) {
+          const Item nx = make_item(a, wn);
+          if (lane == 0) *s_next = nx;
+        }
         // validity of this thread's key (an index load) before the wait
         const int j = it.j0 + tile * kKT + r;
         bool bad = false;
@@ -334,11 +355,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(t_lane + sb * 64u + (uint32_t)h0, z);
         tmem_ld_wait();
         bool over = false;
+        const float4* mrun4 = reinterpret_cast<const float4*>(mrun + h0);  // broadcast, 16 B per read
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          z[i] = valid ? z[i] * scale2 : -INFINITY;
-          const float mr = mrun[h0 + i];
-          over |= z[i] > mr + kRescaleLog2 || (mr == -INFINITY && z[i] != -INFINITY);
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 m4 = mrun4[i4];
+          const float mr4[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = 4 * i4 + u;
+            z[i] = valid ? z[i] * scale2 : -INFINITY;
+            const float mr = mr4[u];
+            over |= z[i] > mr + kRescaleLog2 || (mr == -INFINITY && z[i] != -INFINITY);
+          }
         }
         // the running reference moves (and O^T is rescaled) only when some
         // head's logit passes it by more than 2^8: one barrier-reduction
@@ -358,13 +386,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             alpha_s[st] = al;
           }
           named_bar(1, 256);
+          const float4* al4 = reinterpret_cast<const float4*>(alpha_s + h0);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) lpart[i] *= alpha_s[h0 + i];
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 a4 = al4[i4];
+            lpart[4 * i4] *= a4.x;
+            lpart[4 * i4 + 1] *= a4.y;
+            lpart[4 * i4 + 2] *= a4.z;
+            lpart[4 * i4 + 3] *= a4.w;
+          }
         }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float ma = mrun[h0 + i], mb = mrun[h0 + i + 1];
+          const float2 m2 = reinterpret_cast<const float2*>(mrun + h0)[i >> 1];
+          const float ma = m2.x, mb = m2.y;
           const float pa = (z[i] == -INFINITY || ma == -INFINITY) ? 0.f : ex2_approx(z[i] - ma);
           const float pb = (z[i + 1] == -INFINITY || mb == -INFINITY) ? 0.f : ex2_approx(z[i + 1] - mb);
           const uint32_t w2 = f2_to_bf2x2(pa, pb);
@@ -476,6 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(kEpiDone));
       ++active;
+      if (!kCompact && wn < n_items) named_bar(1, 256);  // *s_next is written
     }
   } else if (warp == kMmaWarp) {
     // =================== MMA issuer ===================

@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs 
 constexpr int kCombThreads = 256;
 
 // One block per (head, query row), one thread per pair of output dims.
-// Every thread merges the splits itself, eight at a time with all their
+// Every thread merges the splits itself, four at a time with all their
 // loads (max, sum, two accumulator values) in flight together: the split
 // maxima and sums are the same addresses for the whole block (broadcast),
 // so no shared memory or block barrier is needed and a decode-sized merge
@@ -493,11 +493,11 @@ __global__ void __launch_bounds__(kCombThreads) attend_combine_kernel(AttendArgs
   for (int d2 = threadIdx.x; d2 < D / 2; d2 += kCombThreads) {
     const int d = 2 * d2;
     float M = -INFINITY, L = 0.f, x0 = 0.f, x1 = 0.f;
-    for (int s0 = 0; s0 < S; s0 += 8) {
-      float ms[8], ls[8];
-      float2 v[8];
+    for (int s0 = 0; s0 < S; s0 += 4) {
+      float ms[4], ls[4];
+      float2 v[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 4; ++u) {
         ms[u] = -INFINITY;
         ls[u] = 0.f;
         v[u] = make_float2(0.f, 0.f);
@@ -510,14 +510,14 @@ __global__ void __launch_bounds__(kCombThreads) attend_combine_kernel(AttendArgs
       }
       float mc = M;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mc = fmaxf(mc, ms[u]);
+      for (int u = 0; u < 4; ++u) mc = fmaxf(mc, ms[u]);
       if (mc == -INFINITY) continue;
       const float sc = __expf(M - mc);  // 0 while nothing was merged
       L *= sc;
       x0 *= sc;
       x1 *= sc;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 4; ++u) {
         // a split with no visible key has max -inf: its accumulator is
         // never read into the sum
         if (ms[u] != -INFINITY) {

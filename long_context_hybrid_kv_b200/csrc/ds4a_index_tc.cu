@@ -218,8 +218,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               float v[32];
               tmem_ld32(t_lane + ab * 256u + (uint32_t)(g * 64 + half * 32), v);
               tmem_ld_wait();
+              // the weights are the same for every thread: 16-byte broadcast
+              // reads, a quarter of the shared-memory instructions
+              const float4* w4 = reinterpret_cast<const float4*>(w_s + g * kHI + half * 32);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) sc[g] = fmaf(w_s[g * kHI + half * 32 + i], fmaxf(v[i], 0.f), sc[g]);
+              for (int i = 0; i < 32; i += 4) {
+                const float4 ww = w4[i >> 2];
+                sc[g] = fmaf(ww.x, fmaxf(v[i], 0.f), sc[g]);
+                sc[g] = fmaf(ww.y, fmaxf(v[i + 1], 0.f), sc[g]);
+                sc[g] = fmaf(ww.z, fmaxf(v[i + 2], 0.f), sc[g]);
+                sc[g] = fmaf(ww.w, fmaxf(v[i + 3], 0.f), sc[g]);
+              }
             }
           }
         }

@@ -6,6 +6,7 @@
 // where those apply.
 #include "ds4a_internal.cuh"
 
+#include <cooperative_groups.h>
 #include <float.h>
 
 namespace ds4a {
@@ -178,12 +179,184 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
   }
 }
 
+// Long entries (HCA: m' = 128 terms) when there are few of them (decode):
+// the Z blocks of a cluster split one entry's terms; each block reduces its
+// terms to one partial softmax per channel, then block r merges channels
+// [r c/Z, (r+1) c/Z) over the cluster through distributed shared memory, the
+// blocks add their RMSNorm sums of squares the same way, and each writes
+// its channels.  Same arithmetic as compress_kernel (log2-unit softmax with a
+// lazy reference), merged in a different order.
+template <int V>
+__global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(CompressArgs a, int Z) {
+  extern __shared__ float csm[];
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int c = a.c, m = a.m;
+  const int NC = c / V;
+  const int G = kCompressThreads / NC;
+  const int tid = threadIdx.x;
+  const int cc = tid % NC;
+  const int g = tid / NC;
+  const int zr = (int)cl.block_rank();
+  const int i = a.entry_begin + blockIdx.x / Z;
+  const int b = blockIdx.y;
+  const bool overlap = a.cb != nullptr;
+  const int n_terms = (overlap && i >= 1) ? 2 * m : m;
+  const int tz0 = (int)((int64_t)zr * n_terms / Z), tz1 = (int)((int64_t)(zr + 1) * n_terms / Z);
+  pdl_trigger();
+  pdl_wait();
+
+  float mx[V], l[V], acc[V];
+#pragma unroll
+  for (int u = 0; u < V; ++u) { mx[u] = -INFINITY; l[u] = 0.f; acc[u] = 0.f; }
+  if (g < G) {
+    for (int t0 = tz0 + g; t0 < tz1; t0 += 4 * G) {
+      float vals[4][V], zs[4][V], bs[4][V];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int term = t0 + u * G;
+        if (term < tz1) {
+          const bool half_a = term < m;
+          const int r = half_a ? term : term - m;
+          const int tok = half_a ? i * m + r : (i - 1) * m + r;
+          const int64_t row = (int64_t)b * a.T_tok + (tok - a.tok_begin);
+          VecLoad<V>::load((half_a ? a.ca : a.cb) + row * c + cc * V, vals[u]);
+          VecLoad<V>::load((half_a ? a.za : a.zb) + row * c + cc * V, zs[u]);
+          VecLoad<V>::load_f((half_a ? a.bias_a : a.bias_b) + (int64_t)r * c + cc * V, bs[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (t0 + u * G >= tz1) break;
+#pragma unroll
+        for (int q = 0; q < V; ++q) {
+          const float x = (zs[u][q] + bs[u][q]) * kLog2eC;
+          if (x > mx[q] + 8.f) {
+            const float sc = ex2_approx(mx[q] - x);
+            l[q] *= sc;
+            acc[q] *= sc;
+            mx[q] = x;
+          }
+          const float e = ex2_approx(x - mx[q]);
+          l[q] += e;
+          acc[q] = fmaf(e, vals[u][q], acc[q]);
+        }
+      }
+    }
+  }
+  // block partials: [G][c] each, then one (M, L, A) per channel
+  float* s_m = csm;
+  float* s_l = s_m + G * c;
+  float* s_a = s_l + G * c;
+  float* p_m = s_a + G * c;  // [c] this block's partial per channel
+  float* p_l = p_m + c;
+  float* p_a = p_l + c;
+  float* s_v = p_a + c;      // [c / Z] pooled values of this block's channels
+  __shared__ float s_red[kCompressThreads / 32];
+  __shared__ float s_tot;
+  if (g < G) {
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      s_m[g * c + cc * V + u] = mx[u];
+      s_l[g * c + cc * V + u] = l[u];
+      s_a[g * c + cc * V + u] = acc[u];
+    }
+  }
+  __syncthreads();
+  for (int ch = tid; ch < c; ch += kCompressThreads) {
+    float M = -INFINITY;
+    for (int gg = 0; gg < G; ++gg) M = fmaxf(M, s_m[gg * c + ch]);
+    float Ls = 0.f, A = 0.f;
+    if (M != -INFINITY)
+      for (int gg = 0; gg < G; ++gg) {
+        const float mm = s_m[gg * c + ch];
+        if (mm == -INFINITY) continue;
+        const float e = ex2_approx(mm - M);
+        Ls += s_l[gg * c + ch] * e;
+        A += s_a[gg * c + ch] * e;
+      }
+    p_m[ch] = M;
+    p_l[ch] = Ls;
+    p_a[ch] = A;
+  }
+  cl.sync();  // every block's partials are complete
+  const int cz = c / Z, ch0 = zr * cz;
+  float ss = 0.f;
+  for (int k = tid; k < cz; k += kCompressThreads) {
+    const int ch = ch0 + k;
+    float pm[8], M = -INFINITY;
+    for (int r = 0; r < Z; ++r) {
+      pm[r] = cl.map_shared_rank(p_m, r)[ch];
+      M = fmaxf(M, pm[r]);
+    }
+    float Ls = 0.f, A = 0.f;
+    for (int r = 0; r < Z; ++r) {
+      if (pm[r] == -INFINITY) continue;
+      const float e = ex2_approx(pm[r] - M);
+      Ls += cl.map_shared_rank(p_l, r)[ch] * e;
+      A += cl.map_shared_rank(p_a, r)[ch] * e;
+    }
+    const float v = A / Ls;
+    s_v[k] = v;
+    ss += v * v;
+  }
+  uint16_t* dst = a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c + ch0;
+  if (a.norm_g == nullptr) {
+    cl.sync();  // no block leaves while a peer may still read its partials
+    for (int k = tid; k < cz; k += kCompressThreads) dst[k] = f2bf(s_v[k]);
+    return;
+  }
+  ss = warp_sum(ss);
+  if ((tid & 31) == 0) s_red[tid >> 5] = ss;
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kCompressThreads / 32; ++w) t += s_red[w];
+    s_tot = t;
+  }
+  cl.sync();  // partials read by every peer; every block's sum is in place
+  float tot = 0.f;
+  for (int r = 0; r < Z; ++r) tot += *cl.map_shared_rank(&s_tot, r);
+  cl.sync();  // no block leaves while a peer may still read its sum
+  const float rstd = rsqrtf(tot / (float)c + a.eps);
+  const int R = a.rope_dim;
+  const int pos = i * m;
+  for (int p2 = tid; p2 < cz / 2; p2 += kCompressThreads) {
+    const int k = 2 * p2, ch = ch0 + k;
+    float x0 = s_v[k] * rstd * a.norm_g[ch];
+    float x1 = s_v[k + 1] * rstd * a.norm_g[ch + 1];
+    if (ch >= c - R) {
+      float cs, sn;
+      rope_cos_sin(pos, a.rope.t[(ch - (c - R)) >> 1], &cs, &sn);
+      const float y0 = x0 * cs - x1 * sn;
+      const float y1 = x0 * sn + x1 * cs;
+      x0 = y0;
+      x1 = y1;
+    }
+    *reinterpret_cast<unsigned int*>(dst + k) = f2_to_bf2x2(x0, x1);
+  }
+}
+
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
   const int n = a.entry_end - a.entry_begin;
   if (n <= 0 || a.B <= 0) return cudaSuccess;
   const int V = (a.c % 8 == 0) ? 8 : 2;
   const int NC = a.c / V;
   const int G = NC >= kCompressThreads ? 1 : kCompressThreads / NC;
+  const int n_terms = a.cb != nullptr ? 2 * a.m : a.m;
+  // long entries, few of them: split each entry's terms over a cluster
+  int Z = 1;
+  if (V == 8 && n_terms >= 64)
+    while (Z < 8 && (int64_t)n * a.B * Z * 2 <= 148 && n_terms / (2 * Z) >= 16 && a.c % (2 * Z * 2) == 0) Z *= 2;
+  if (Z > 1) {
+    const size_t smem = (size_t)(3 * G * a.c + 3 * a.c + a.c / Z) * sizeof(float);
+    static int cache_s[16];
+    cudaError_t e = ensure_smem(compress_split_kernel<8>, (int)smem, cache_s);
+    if (e != cudaSuccess) return e;
+    TraceScope tr("compress", s);
+    return launch_pdl_cluster(compress_split_kernel<8>, dim3(n * Z, a.B), dim3(kCompressThreads), smem, s, Z, a,
+                              Z);
+  }
   const size_t smem = (size_t)(3 * G * a.c + a.c) * sizeof(float);
   static int cache8[16], cache2[16];
   cudaError_t e = V == 8 ? ensure_smem(compress_kernel<8>, (int)smem, cache8)

@@ -213,23 +213,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 0; g < kMaxG; ++g) {
           sc[g] = 0.f;
           if (g < G) {
+            // four independent sums per query (one epilogue warp per SM
+            // sub-partition cannot hide a 64-long FMA chain)
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
+            // both 32-column halves in flight, one wait
+            float v[2][32];
+            tmem_ld32(t_lane + ab * 256u + (uint32_t)(g * 64), v[0]);
+            tmem_ld32(t_lane + ab * 256u + (uint32_t)(g * 64 + 32), v[1]);
+            tmem_ld_wait();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-              float v[32];
-              tmem_ld32(t_lane + ab * 256u + (uint32_t)(g * 64 + half * 32), v);
-              tmem_ld_wait();
               // the weights are the same for every thread: 16-byte broadcast
               // reads, a quarter of the shared-memory instructions
               const float4* w4 = reinterpret_cast<const float4*>(w_s + g * kHI + half * 32);
 #pragma unroll
               for (int i = 0; i < 32; i += 4) {
                 const float4 ww = w4[i >> 2];
-                sc[g] = fmaf(ww.x, fmaxf(v[i], 0.f), sc[g]);
-                sc[g] = fmaf(ww.y, fmaxf(v[i + 1], 0.f), sc[g]);
-                sc[g] = fmaf(ww.z, fmaxf(v[i + 2], 0.f), sc[g]);
-                sc[g] = fmaf(ww.w, fmaxf(v[i + 3], 0.f), sc[g]);
+                s4[0] = fmaf(ww.x, fmaxf(v[half][i], 0.f), s4[0]);
+                s4[1] = fmaf(ww.y, fmaxf(v[half][i + 1], 0.f), s4[1]);
+                s4[2] = fmaf(ww.z, fmaxf(v[half][i + 2], 0.f), s4[2]);
+                s4[3] = fmaf(ww.w, fmaxf(v[half][i + 3], 0.f), s4[3]);
               }
             }
+            sc[g] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
           }
         }
         tc_fence_before();

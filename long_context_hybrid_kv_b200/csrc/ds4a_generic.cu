@@ -646,12 +646,15 @@ __global__ void __launch_bounds__(kAttThreads) attend_generic_kernel(AttendArgs 
 constexpr int kCombThreads = 256;
 
 // One block per (head, query row), one thread per pair of output dims.
-// Every thread merges the splits itself, four at a time with all their
-// loads (max, sum, two accumulator values) in flight together: the split
+// Every thread merges the splits itself, K at a time with all their loads
+// (max, sum, two accumulator values) in flight together (K = 4 when that
+// covers every split, keeping registers low for many resident blocks, else
+// 8): the split
 // maxima and sums are the same addresses for the whole block (broadcast),
 // so no shared memory or block barrier is needed and a decode-sized merge
 // costs one memory round trip.  The sink enters the denominator as in the
 // split-free kernels; the rope slice is de-rotated by -pos at the end.
+template <int K>
 __global__ void __launch_bounds__(kCombThreads) attend_combine_kernel(AttendArgs a) {
   const int H = a.H, D = a.D, S = a.n_splits, R = a.R;
   const int h = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
@@ -666,11 +669,11 @@ __global__ void __launch_bounds__(kCombThreads) attend_combine_kernel(AttendArgs
   for (int d2 = threadIdx.x; d2 < D / 2; d2 += kCombThreads) {
     const int d = 2 * d2;
     float M = -INFINITY, L = 0.f, x0 = 0.f, x1 = 0.f;
-    for (int s0 = 0; s0 < S; s0 += 4) {
-      float ms[4], ls[4];
-      float2 v[4];
+    for (int s0 = 0; s0 < S; s0 += K) {
+      float ms[K], ls[K];
+      float2 v[K];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < K; ++u) {
         ms[u] = -INFINITY;
         ls[u] = 0.f;
         v[u] = make_float2(0.f, 0.f);
@@ -683,14 +686,14 @@ __global__ void __launch_bounds__(kCombThreads) attend_combine_kernel(AttendArgs
       }
       float mc = M;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) mc = fmaxf(mc, ms[u]);
+      for (int u = 0; u < K; ++u) mc = fmaxf(mc, ms[u]);
       if (mc == -INFINITY) continue;
       const float sc = __expf(M - mc);  // 0 while nothing was merged
       L *= sc;
       x0 *= sc;
       x1 *= sc;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < K; ++u) {
         // a split with no visible key has max -inf: its accumulator is
         // never read into the sum
         if (ms[u] != -INFINITY) {
@@ -770,7 +773,9 @@ cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s) {
   TraceScope tr("attend_combine", s);
-  return launch_pdl(attend_combine_kernel, dim3(a.H, a.T_q, a.B), dim3(kCombThreads), 0, s, a);
+  return a.n_splits <= 4
+             ? launch_pdl(attend_combine_kernel<4>, dim3(a.H, a.T_q, a.B), dim3(kCombThreads), 0, s, a)
+             : launch_pdl(attend_combine_kernel<8>, dim3(a.H, a.T_q, a.B), dim3(kCombThreads), 0, s, a);
 }
 
 }  // namespace ds4a

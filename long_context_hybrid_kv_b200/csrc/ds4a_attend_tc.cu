@@ -413,26 +413,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the previous tile's PV must be done before P^T and O^T change
           mbar_wait(bar(kPVDone), (gt - 1) & 1u, abort_flag, err);
           tc_fence_after();
-          if (rescale) {
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              float v[32];
-              const uint32_t addr = t_lane + 128u + 64u * c + (uint32_t)h0;
-              tmem_ld32(addr, v);
-              tmem_ld_wait();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] *= alpha_s[h0 + i];
-              tmem_st32(addr, v);
-            }
-            tmem_st_wait();
-          }
         }
         // P^T row r, heads h0 .. h0+31: 64 B = chunks 4 hf .. 4 hf + 3 of the
-        // 128-byte swizzled row
+        // 128-byte swizzled row (written before the O^T rescale, so that the
+        // packed probabilities are not live across it)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
           st_shared16(p_base + sw128(r, 4 * hf + cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
                       pk[4 * cc + 3]);
+        if (tile > 0 && rescale) {
+          const float4* al4 = reinterpret_cast<const float4*>(alpha_s + h0);
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            // 16 head columns of one 128-dim chunk at a time
+            float v[16];
+            const uint32_t addr = t_lane + 128u + 64u * (c >> 1) + (uint32_t)h0 + 16u * (c & 1);
+            tmem_ld16(addr, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+              const float4 a4 = al4[4 * (c & 1) + i4];
+              v[4 * i4] *= a4.x;
+              v[4 * i4 + 1] *= a4.y;
+              v[4 * i4 + 2] *= a4.z;
+              v[4 * i4 + 3] *= a4.w;
+            }
+            tmem_st16(addr, v);
+          }
+          tmem_st_wait();
+        }
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(bar(kPFull));

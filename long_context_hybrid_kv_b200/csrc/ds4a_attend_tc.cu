@@ -18,7 +18,7 @@
 //              (O^T is rescaled only when a head's running max grows by
 //              more than 2^8), P^T to shared memory as bf16, final
 //              normalisation with the sink, de-rotation of the rope slice
-//              by -pos, staged 16-byte stores.
+//              by -pos, stores straight from registers.
 //   warp 8     TMEM allocation; lane 0 issues every tcgen05.mma / commit.
 //   warps 9-12 producers: q^ as one 64 KB bulk copy of the image that
 //              qhat_prep_kernel wrote, then the KV rows by cp.async, one
@@ -59,7 +59,8 @@ constexpr uint32_t kOffAlpha = kOffMrun + 256;      // [64]
 constexpr uint32_t kOffInv = kOffAlpha + 256;       // [64]
 constexpr uint32_t kOffSink = kOffInv + 256;        // [64] sink * log2(e)
 constexpr uint32_t kOffNext = kOffSink + 256;       // the softmax warps' next work item
-constexpr uint32_t kSmemBytes = kOffNext + 64 + 1024;  // + alignment slack
+constexpr uint32_t kOffValid = kOffNext + 64;       // [2 tiles][128 keys] validity flags
+constexpr uint32_t kSmemBytes = kOffValid + 256 + 1024;  // + alignment slack
 
 enum Bar {
   kQFull = 0, kQEmpty, kKVFull0, kKVFull1, kKVFull2, kKVFull3, kKVEmpty0, kKVEmpty1, kKVEmpty2,
@@ -151,8 +152,6 @@ __device__ __forceinline__ const uint16_t* key_ptr(const AttendArgs& a, const It
 // runs each of them once with its code fetched cold, and the rolled loop is
 // a few cache lines instead of a few hundred instructions; a prefill block
 // runs them per tile with the code warm and keeps them unrolled.
-// omap: the output as rows of 512 bf16 ([B*T_q*64][512], box 128 dims x
-// 64 heads), written by TMA stores from the idle P^T buffer.
 // kvmap: the pool as rows of 512 bf16 (box 64 dims x 128 rows, 128-byte
 // swizzle) for the dense key ranges of HCA: a tile of 128 consecutive pool
 // entries comes in as eight TMA tile loads instead of 2048 gathered
@@ -164,8 +163,8 @@ struct DenseKV {
 
 template <bool kCompact>
 __global__ void __launch_bounds__(kThreads, 1)
-    attend_tc_kernel(const __grid_constant__ CUtensorMap omap, const __grid_constant__ CUtensorMap kvmap, DenseKV dkv, AttendArgs a, int n_items,
-                                                                const uint8_t* qimg) {
+    attend_tc_kernel(const __grid_constant__ CUtensorMap kvmap, DenseKV dkv, AttendArgs a, int n_items,
+                     const uint8_t* qimg) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -181,6 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);
   float* inv_s = reinterpret_cast<float*>(smem + kOffInv);
   float* sink_s = reinterpret_cast<float*>(smem + kOffSink);
+  // validity of each key slot of the last two tiles (written by the
+  // producers with the row pointers, read by the softmax warps once the
+  // tile's rows have landed)
+  uint8_t* vflag = smem + kOffValid;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -346,11 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) *s_next = nx;
         }
         // validity of this thread's key (an index load) before the wait
-        const int j = it.j0 + tile * kKT + r;
-        bool bad = false;
-        const bool valid = key_ptr(a, it, j, &bad) != nullptr;
         mbar_wait(bar(kSFull), gt & 1u, abort_flag, err);
+        // the last chunk's barrier (complete before S^T is) orders the
+        // producers' validity flags of this tile before the read
+        mbar_wait(bar(kKVFull0 + 3), gt & 1u, abort_flag, err);
         tc_fence_after();
+        const bool valid = vflag[(gt & 1u) * kKT + r] != 0;
         float z[32];
         tmem_ld32(t_lane + sb * 64u + (uint32_t)h0, z);
         tmem_ld_wait();
@@ -473,10 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(1, 256);
       float cs = 1.f, sn = 0.f;
       const int R = a.R;
-      // the final output goes out through the idle P^T buffer (16 KiB): per
-      // chunk [64 heads][128 dims] bf16, sent by one TMA store; split
-      // partials go straight to the workspace (coalesced 128-byte rows)
-      unsigned int* stage = reinterpret_cast<unsigned int*>(smem + kOffP);
+      // both go straight from registers to global memory: the final output
+      // as 4-byte words (two dims of one head; a warp writes two 64-byte
+      // runs per store), split partials as coalesced 128-byte rows
+      unsigned int* orow = reinterpret_cast<unsigned int*>(a.out + (int64_t)it.row * kH * kD);
       const bool odd = r & 1;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -502,16 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               x0 = y0;
               x1 = y1;
             }
-            stage[h * 64 + (r >> 1)] = f2_to_bf2x2(x0, x1);
+            orow[h * (kD / 2) + 64 * c + (r >> 1)] = f2_to_bf2x2(x0, x1);
           }
-          fence_async_smem();
-          named_bar(1, 256);
-          if (st == 0) {
-            tma_store_2d(&omap, p_base, 128 * c, it.row * kH);
-            bulk_commit();
-            bulk_wait_read();  // the buffer is free again
-          }
-          named_bar(1, 256);
         } else {
           float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
 #pragma unroll
@@ -595,6 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint16_t* p = key_ptr(a, it, it.j0 + tile * kKT + pt, &bad);
         if (bad) raise_err(err, DS4A_DEV_BAD_INDEX);
         rowptr[pt] = p;
+        vflag[(gt & 1u) * kKT + pt] = p != nullptr;
         named_bar(2, 128);
       };
       // one 128-dim chunk of the tile: 128 rows x 256 B, 16 cp.async each;
@@ -630,6 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // barrier with its bytes and starts two TMA tile loads, the
           // others arrive
           const int y = (int)(it.b * dkv.pool_rows_b + s0);
+          vflag[(gt & 1u) * kKT + pt] = 1;  // 128 entries inside the visible range
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             if (gt > 0) mbar_wait(bar(kKVEmpty0 + c), (gt - 1) & 1u, abort_flag, err);
@@ -665,7 +663,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) mbar_drain(bar(kKVFull0 + c), (gt - 1) & 1u);
   }
 
-  if (tid == 0) bulk_wait_all();  // the output stores have landed
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -787,19 +784,8 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
     e = launch_pdl(qhat_prep_kernel, dim3(rows, kH / 16), dim3(256), 0, s, a, qimg);
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap omap;
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
   if (!encode) return cudaErrorNotSupported;
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows * kH};
-    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-    const cuuint32_t box[2] = {128, (cuuint32_t)kH};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
   // HCA keys are consecutive pool entries: a row view of the pool for TMA
   // tile loads (when the sequences are a whole number of rows apart)
   CUtensorMap kvmap;
@@ -823,9 +809,9 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   {
     TraceScope tr("attend_tc", s);
     const uint8_t* qi = qimg;
-    e = compact ? launch_pdl(attend_tc_kernel<true>, dim3(grid), dim3(kThreads), kSmemBytes, s, omap, kvmap,
+    e = compact ? launch_pdl(attend_tc_kernel<true>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap,
                              dkv, a, n_items, qi)
-                : launch_pdl(attend_tc_kernel<false>, dim3(grid), dim3(kThreads), kSmemBytes, s, omap, kvmap,
+                : launch_pdl(attend_tc_kernel<false>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap,
                              dkv, a, n_items, qi);
   }
   if (e != cudaSuccess || a.n_splits == 1) return e;

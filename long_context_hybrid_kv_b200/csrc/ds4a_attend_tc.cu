@@ -358,7 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float z[32];
         tmem_ld32(t_lane + sb * 64u + (uint32_t)h0, z);
         tmem_ld_wait();
-        bool over = false;
+        // largest lead of a logit over its head's reference: fmaxf drops the
+        // NaN of (-inf) - (-inf), and a finite logit against a -inf
+        // reference leads by +inf
+        float lead = -INFINITY;
         const float4* mrun4 = reinterpret_cast<const float4*>(mrun + h0);  // broadcast, 16 B per read
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
@@ -368,10 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 4; ++u) {
             const int i = 4 * i4 + u;
             z[i] = valid ? z[i] * scale2 : -INFINITY;
-            const float mr = mr4[u];
-            over |= z[i] > mr + kRescaleLog2 || (mr == -INFINITY && z[i] != -INFINITY);
+            lead = fmaxf(lead, z[i] - mr4[u]);
           }
         }
+        const bool over = lead > kRescaleLog2;
         // the running reference moves (and O^T is rescaled) only when some
         // head's logit passes it by more than 2^8: one barrier-reduction
         // decides whether the tile maximum is needed at all
@@ -405,8 +408,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; i += 2) {
           const float2 m2 = reinterpret_cast<const float2*>(mrun + h0)[i >> 1];
           const float ma = m2.x, mb = m2.y;
-          const float pa = (z[i] == -INFINITY || ma == -INFINITY) ? 0.f : ex2_approx(z[i] - ma);
-          const float pb = (z[i + 1] == -INFINITY || mb == -INFINITY) ? 0.f : ex2_approx(z[i + 1] - mb);
+          // a -inf logit (with any reference) gives 2^-inf = 0; fmaxf turns
+          // the NaN of (-inf) - (-inf) into -inf as well
+          const float pa = ex2_approx(fmaxf(z[i] - ma, -INFINITY));
+          const float pb = ex2_approx(fmaxf(z[i + 1] - mb, -INFINITY));
           const uint32_t w2 = f2_to_bf2x2(pa, pb);
           pk[i >> 1] = w2;
           const float2 pr = bf2x2_to_f2(w2);

@@ -45,6 +45,9 @@ constexpr int kMmaWarp = 8;
 constexpr int kPG0 = 288;             // first producer thread (warps 9-12)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
+// running reference of a head that has seen no key yet: finite, so that
+// logit - reference never meets (-inf) - (-inf), and far below any logit
+constexpr float kNoRef = -1e30f;
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffKV = 0;              // 8 blocks x [128 keys][128 B]
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_async_smem();
         mbar_arrive(bar(kQFull));
       }
-      if (st < kH) mrun[st] = -INFINITY;
+      if (st < kH) mrun[st] = kNoRef;
       float lpart[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) lpart[i] = 0.f;
@@ -348,31 +351,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const Item nx = make_item(a, wn);
           if (lane == 0) *s_next = nx;
         }
-        // validity of this thread's key (an index load) before the wait
         mbar_wait(bar(kSFull), gt & 1u, abort_flag, err);
         // the last chunk's barrier (complete before S^T is) orders the
         // producers' validity flags of this tile before the read
         mbar_wait(bar(kKVFull0 + 3), gt & 1u, abort_flag, err);
         tc_fence_after();
-        const bool valid = vflag[(gt & 1u) * kKT + r] != 0;
+        // a key slot without a row (zero-filled, so its S^T row is 0) gets
+        // -inf through the bias of the scaling FMA
+        const float zbias = vflag[(gt & 1u) * kKT + r] != 0 ? 0.f : -INFINITY;
         float z[32];
         tmem_ld32(t_lane + sb * 64u + (uint32_t)h0, z);
         tmem_ld_wait();
-        // largest lead of a logit over its head's reference: fmaxf drops the
-        // NaN of (-inf) - (-inf), and a finite logit against a -inf
-        // reference leads by +inf
+        // largest lead of a logit over its head's reference (pairs of
+        // columns per instruction)
         float lead = -INFINITY;
         const float4* mrun4 = reinterpret_cast<const float4*>(mrun + h0);  // broadcast, 16 B per read
+        const float2 sc2 = make_float2(scale2, scale2), zb2 = make_float2(zbias, zbias);
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 m4 = mrun4[i4];
-          const float mr4[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int i = 4 * i4 + u;
-            z[i] = valid ? z[i] * scale2 : -INFINITY;
-            lead = fmaxf(lead, z[i] - mr4[u]);
-          }
+          const float2 za = fma_f2(make_float2(z[4 * i4], z[4 * i4 + 1]), sc2, zb2);
+          const float2 zc = fma_f2(make_float2(z[4 * i4 + 2], z[4 * i4 + 3]), sc2, zb2);
+          z[4 * i4] = za.x;
+          z[4 * i4 + 1] = za.y;
+          z[4 * i4 + 2] = zc.x;
+          z[4 * i4 + 3] = zc.y;
+          const float2 da = sub_f2(za, make_float2(m4.x, m4.y)), dc = sub_f2(zc, make_float2(m4.z, m4.w));
+          lead = fmaxf(lead, fmaxf(fmaxf(da.x, da.y), fmaxf(dc.x, dc.y)));
         }
         const bool over = lead > kRescaleLog2;
         // the running reference moves (and O^T is rescaled) only when some
@@ -386,8 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float mt = fmaxf(fmaxf(red[st], red[64 + st]), fmaxf(red[128 + st], red[192 + st]));
             const float mo = mrun[st];
             float al = 1.f;
-            if (mt > mo + kRescaleLog2 || (mo == -INFINITY && mt != -INFINITY)) {
-              al = (mo == -INFINITY) ? 0.f : exp2f(mo - mt);
+            if (mt > mo + kRescaleLog2) {  // a -inf tile maximum never moves it
+              al = exp2f(mo - mt);               // 0 from the no-key reference
               mrun[st] = mt;
             }
             alpha_s[st] = al;
@@ -397,26 +402,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i4 = 0; i4 < 8; ++i4) {
             const float4 a4 = al4[i4];
-            lpart[4 * i4] *= a4.x;
-            lpart[4 * i4 + 1] *= a4.y;
-            lpart[4 * i4 + 2] *= a4.z;
-            lpart[4 * i4 + 3] *= a4.w;
+            const float2 la = mul_f2(make_float2(lpart[4 * i4], lpart[4 * i4 + 1]), make_float2(a4.x, a4.y));
+            const float2 lc = mul_f2(make_float2(lpart[4 * i4 + 2], lpart[4 * i4 + 3]), make_float2(a4.z, a4.w));
+            lpart[4 * i4] = la.x;
+            lpart[4 * i4 + 1] = la.y;
+            lpart[4 * i4 + 2] = lc.x;
+            lpart[4 * i4 + 3] = lc.y;
           }
         }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           const float2 m2 = reinterpret_cast<const float2*>(mrun + h0)[i >> 1];
-          const float ma = m2.x, mb = m2.y;
-          // a -inf logit (with any reference) gives 2^-inf = 0; fmaxf turns
-          // the NaN of (-inf) - (-inf) into -inf as well
-          const float pa = ex2_approx(fmaxf(z[i] - ma, -INFINITY));
-          const float pb = ex2_approx(fmaxf(z[i + 1] - mb, -INFINITY));
-          const uint32_t w2 = f2_to_bf2x2(pa, pb);
+          // a -inf logit gives 2^-inf = 0 (the reference is always finite)
+          const float2 d = sub_f2(make_float2(z[i], z[i + 1]), m2);
+          const uint32_t w2 = f2_to_bf2x2(ex2_approx(d.x), ex2_approx(d.y));
           pk[i >> 1] = w2;
-          const float2 pr = bf2x2_to_f2(w2);
-          lpart[i] += pr.x;
-          lpart[i + 1] += pr.y;
+          const float2 l2 = add_f2(make_float2(lpart[i], lpart[i + 1]), bf2x2_to_f2(w2));
+          lpart[i] = l2.x;
+          lpart[i + 1] = l2.y;
         }
         if (tile > 0) {
           // the previous tile's PV must be done before P^T and O^T change
@@ -471,11 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l = red[st] + red[64 + st] + red[128 + st] + red[192 + st];
         const float m = mrun[st];
         if (final_out) {
-          const float den = (m == -INFINITY) ? 0.f : l + exp2f(sink_s[st] - m);
+          const float den = (m <= kNoRef) ? 0.f : l + exp2f(sink_s[st] - m);
           inv_s[st] = den > 0.f ? 1.f / den : 0.f;
         } else {
           float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
-          part[st] = (m == -INFINITY) ? -INFINITY : m * 0.6931471805599453f;  // natural-log units
+          part[st] = (m <= kNoRef) ? -INFINITY : m * 0.6931471805599453f;  // natural-log units
           part[kH + st] = l;
         }
       }
@@ -505,13 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float got = __shfl_xor_sync(0xffffffffu, odd ? v[i] : v[i + 1], 1);
             const int h = h0 + i + (odd ? 1 : 0);
             const float s = inv_s[h];
-            float x0 = (odd ? got : v[i]) * s, x1 = (odd ? v[i + 1] : got) * s;
-            if (rot) {
-              const float y0 = x0 * cs + x1 * sn, y1 = -x0 * sn + x1 * cs;
-              x0 = y0;
-              x1 = y1;
-            }
-            orow[h * (kD / 2) + 64 * c + (r >> 1)] = f2_to_bf2x2(x0, x1);
+            float2 x = mul_f2(make_float2(odd ? got : v[i], odd ? v[i + 1] : got), make_float2(s, s));
+            if (rot)  // (x0 cs + x1 sn, -x0 sn + x1 cs)
+              x = fma_f2(make_float2(x.x, x.x), make_float2(cs, -sn), mul_f2(make_float2(x.y, x.y), make_float2(sn, cs)));
+            orow[h * (kD / 2) + 64 * c + (r >> 1)] = f2_to_bf2x2(x.x, x.y);
           }
         } else {
           float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);

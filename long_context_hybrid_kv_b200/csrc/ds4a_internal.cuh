@@ -41,6 +41,40 @@ __device__ __forceinline__ unsigned int f2_to_bf2x2(float a, float b) {
   return u;
 }
 
+// packed fp32 pairs: one instruction works on both halves of a float2
+__device__ __forceinline__ float2 add_f2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n .reg .b64 x, y, d;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n"
+      " add.rn.f32x2 d, x, y;\n mov.b64 {%0, %1}, d;\n}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 sub_f2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n .reg .b64 x, y, d;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n"
+      " sub.rn.f32x2 d, x, y;\n mov.b64 {%0, %1}, d;\n}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 mul_f2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n .reg .b64 x, y, d;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n"
+      " mul.rn.f32x2 d, x, y;\n mov.b64 {%0, %1}, d;\n}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 fma_f2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n .reg .b64 x, y, z, d;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n"
+      " mov.b64 z, {%6, %7};\n fma.rn.f32x2 d, x, y, z;\n mov.b64 {%0, %1}, d;\n}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
 // RoPE frequencies theta_j = base^(-2j/R), j < R/2, divided by pi and
 // formed in float64 on the host once per call (float32 would lose ~0.03 rad
 // of phase at positions near 2^20).

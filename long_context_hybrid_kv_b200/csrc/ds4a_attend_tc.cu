@@ -219,7 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   unsigned int* err = a.err;
   pdl_trigger();
-  pdl_wait();
+  // the softmax warps of a decode-sized launch wait after preparing q^
+  if (!kCompact || warp >= 8) pdl_wait();
 
   if (warp < 8) {
     // =================== softmax + epilogue (8 warps) ===================
@@ -232,56 +233,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
     const float scale2 = a.scale * kLog2e;
     if (st < kH) sink_s[st] = a.sink[st] * kLog2e;  // read by the epilogues (after a named barrier)
-    // Warp 0 builds the next work item during the current item's last tile
-    // (its loads overlap the wait for S^T) and leaves it in shared memory;
-    // every softmax thread picks it up after the epilogue's last barrier.
-    Item* s_next = reinterpret_cast<Item*>(smem + kOffNext);
-    uint32_t gt = 0, active = 0;
-    Item it;
-    if (!kCompact && (int)blockIdx.x < n_items) it = make_item(a, blockIdx.x);
-    for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
-      const int wn = w + (int)gridDim.x;
-      if (kCompact) it = make_item(a, w);  // one item per block
-      else if (w != (int)blockIdx.x) it = *s_next;
-      const bool final_out = a.n_splits == 1;
-      if (it.pos < 0 && st == 0 && it.split == 0) raise_err(err, DS4A_DEV_BAD_POS);
-      if (it.n_tiles == 0) {
-        // no keys in this item: output 0, or an empty partial
-        if (final_out) {
-          if (it.pos >= 0)
-            for (int e = st; e < kH * kD / 8; e += 256)
-              reinterpret_cast<uint4*>(a.out + (int64_t)it.row * kH * kD)[e] = make_uint4(0, 0, 0, 0);
-        } else {
-          float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
-          if (st < kH) {
-            part[st] = -INFINITY;
-            part[kH + st] = 0.f;
-          }
-          for (int e = st; e < kH * kD; e += 256) part[2 * kH + e] = 0.f;
-        }
-        if (!kCompact && wn < n_items) {
-          named_bar(1, 256);  // every softmax thread has read *s_next
-          if (warp == 0) {
-            const Item nx = make_item(a, wn);
-            if (lane == 0) *s_next = nx;
-          }
-          named_bar(1, 256);
-        }
-        continue;
-      }
-      if (kCompact) {
-        // q^ = RoPE_pos(RMSNorm(q) * g) of this block's (only) query,
-        // straight into the operand layout while the K=V rows are on their
-        // way: warp w takes heads w, w + 8, ..., four heads' rows in flight
-        // per round; lane l holds dims 8l..8l+7 and 256+8l..256+8l+7
-        const uint16_t* qrow = a.q + (int64_t)it.row * kH * kD;
+    if (kCompact) {
+      // q^ = RoPE_pos(RMSNorm(q) * g) of this block's (only) query, straight
+      // into the operand layout before the wait for the preceding kernels:
+      // it reads only the query, its position and the weights, none of
+      // which a preceding kernel of the chain writes.  Warp w takes heads
+      // w, w + 8, ..., four heads' rows in flight per round; lane l holds
+      // dims 8l..8l+7 and 256+8l..256+8l+7
+      if ((int)blockIdx.x < n_items) {
+        const int row = (int)blockIdx.x / a.n_splits;
+        const int pos = a.q_pos[row];
+        const uint16_t* qrow = a.q + (int64_t)row * kH * kD;
         float rc[4], rs[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           rc[u] = 1.f;
           rs[u] = 0.f;
           const int d = 256 + 8 * lane + 2 * u;
-          if (d >= kD - a.R) rope_cos_sin(it.pos, a.rope.t[(d - (kD - a.R)) >> 1], &rc[u], &rs[u]);
+          if (d >= kD - a.R) rope_cos_sin(pos, a.rope.t[(d - (kD - a.R)) >> 1], &rc[u], &rs[u]);
         }
         const float4 g0 = *reinterpret_cast<const float4*>(a.q_norm_g + 8 * lane);
         const float4 g1 = *reinterpret_cast<const float4*>(a.q_norm_g + 8 * lane + 4);
@@ -339,6 +308,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_async_smem();
         mbar_arrive(bar(kQFull));
+      }
+      pdl_wait();
+    }
+    // Warp 0 builds the next work item during the current item's last tile
+    // (its loads overlap the wait for S^T) and leaves it in shared memory;
+    // every softmax thread picks it up after the epilogue's last barrier.
+    Item* s_next = reinterpret_cast<Item*>(smem + kOffNext);
+    uint32_t gt = 0, active = 0;
+    Item it;
+    if (!kCompact && (int)blockIdx.x < n_items) it = make_item(a, blockIdx.x);
+    for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+      const int wn = w + (int)gridDim.x;
+      if (kCompact) it = make_item(a, w);  // one item per block
+      else if (w != (int)blockIdx.x) it = *s_next;
+      const bool final_out = a.n_splits == 1;
+      if (it.pos < 0 && st == 0 && it.split == 0) raise_err(err, DS4A_DEV_BAD_POS);
+      if (it.n_tiles == 0) {
+        // no keys in this item: output 0, or an empty partial
+        if (final_out) {
+          if (it.pos >= 0)
+            for (int e = st; e < kH * kD / 8; e += 256)
+              reinterpret_cast<uint4*>(a.out + (int64_t)it.row * kH * kD)[e] = make_uint4(0, 0, 0, 0);
+        } else {
+          float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
+          if (st < kH) {
+            part[st] = -INFINITY;
+            part[kH + st] = 0.f;
+          }
+          for (int e = st; e < kH * kD; e += 256) part[2 * kH + e] = 0.f;
+        }
+        if (!kCompact && wn < n_items) {
+          named_bar(1, 256);  // every softmax thread has read *s_next
+          if (warp == 0) {
+            const Item nx = make_item(a, wn);
+            if (lane == 0) *s_next = nx;
+          }
+          named_bar(1, 256);
+        }
+        continue;
       }
       if (st < kH) mrun[st] = kNoRef;
       float lpart[32];

@@ -19,6 +19,16 @@
  * - Execution: every call is asynchronous on the given CUDA stream (NULL =
  *   the legacy default stream).  Pointers named "device" must be device (or
  *   managed) memory of the current device; "host" pointers are host memory.
+ * - Overlap: the library's kernels are launched with programmatic dependent
+ *   launch, so a kernel may start while the library kernel before it on the
+ *   stream is still running.  It waits for that kernel before it reads what
+ *   a library call writes (pool, scores, indices, workspace) and before it
+ *   writes anything, but it may read its pure inputs (queries, raw C/Z
+ *   rows, weights, positions, window rows) earlier.  Those inputs must
+ *   therefore not be written by a still-running library kernel: produce
+ *   them with ordinary stream work (any kernel or copy that is not part of
+ *   this library orders fully), never by feeding one call's output buffer
+ *   to the next call as an input.
  * - Storage types: ds4a_bf16 is a bfloat16 bit pattern.  Arithmetic is
  *   float32 (bf16 x bf16 products accumulated in float32 on tensor cores).
  * - Layouts: contiguous row-major, dimensions listed outermost first; batch

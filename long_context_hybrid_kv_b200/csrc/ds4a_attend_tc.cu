@@ -692,9 +692,11 @@ __global__ void __launch_bounds__(256) qhat_prep_kernel(AttendArgs a, uint8_t* q
   const int row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
-  pdl_wait();
   // every load goes out before any of them is used: the two heads' rows
-  // (heads 16 y + w and 16 y + 8 + w), this lane's gains, the position
+  // (heads 16 y + w and 16 y + 8 + w), this lane's gains, the position --
+  // all inputs that no kernel of the chain writes, so they go out before
+  // the wait for the preceding kernels, which only the image writes need
+  // (the previous attention may still be reading the image)
   const uint16_t* qrow = a.q + (int64_t)row * kH * kD;
   uint4 v[2][2];
 #pragma unroll
@@ -721,6 +723,7 @@ __global__ void __launch_bounds__(256) qhat_prep_kernel(AttendArgs a, uint8_t* q
     rt[j] = make_float2(cs, sn);
   }
   __syncthreads();
+  pdl_wait();
   uint8_t* img = qimg + (size_t)row * 65536u;
 #pragma unroll
   for (int u = 0; u < 2; ++u) {

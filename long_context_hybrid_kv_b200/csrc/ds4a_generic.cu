@@ -73,7 +73,10 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
   const bool overlap = a.cb != nullptr;
   const int n_terms = (overlap && i >= 1) ? 2 * m : m;
   pdl_trigger();
-  pdl_wait();
+  // The C/Z rows, gate biases and norm weights are inputs that no kernel of
+  // the chain writes: the pooling runs while the preceding kernel finishes,
+  // and only the pool write waits for it (a preceding kernel may still read
+  // the entry this one overwrites).
 
   float mx[V], l[V], acc[V];
 #pragma unroll
@@ -148,6 +151,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
     s_v[ch] = v;
     ss += v * v;
   }
+  pdl_wait();
   uint16_t* dst = a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c;
   if (a.norm_g == nullptr) {
     __syncthreads();
@@ -204,7 +208,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
   const int n_terms = (overlap && i >= 1) ? 2 * m : m;
   const int tz0 = (int)((int64_t)zr * n_terms / Z), tz1 = (int)((int64_t)(zr + 1) * n_terms / Z);
   pdl_trigger();
-  pdl_wait();
+  // as in compress_kernel, only the pool write waits for the preceding kernel
 
   float mx[V], l[V], acc[V];
 #pragma unroll
@@ -300,6 +304,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
     s_v[k] = v;
     ss += v * v;
   }
+  pdl_wait();
   uint16_t* dst = a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c + ch0;
   if (a.norm_g == nullptr) {
     cl.sync();  // no block leaves while a peer may still read its partials
@@ -660,9 +665,9 @@ __global__ void __launch_bounds__(kCombThreads) attend_combine_kernel(AttendArgs
   const int h = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
   const int row = b * a.T_q + t;
   pdl_trigger();
-  pdl_wait();
-  const int pos = a.q_pos[row];
+  const int pos = a.q_pos[row];  // inputs: read before the wait
   const float sink = a.sink[h];
+  pdl_wait();
   const int64_t stride = 2 * H + (int64_t)H * D;
   const float* base = a.ws + (int64_t)row * S * stride;
   uint16_t* orow = a.out + ((int64_t)row * H + h) * D;

@@ -125,20 +125,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();
-  pdl_wait();
+  // Each role waits for the preceding kernels only before its first read of
+  // their output (the keys) or its first write: the queries, weights and
+  // positions are inputs that no kernel of the chain writes, so the first
+  // pair's queries and weights come in while the preceding kernel finishes.
 
   if (warp == 0) {
     // =================== TMA producer ===================
     if (lane == 0) {
       uint32_t kt = 0, active = 0;
-      for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
-        const Pair q = make_pair(p, w);
-        if (q.tile1 <= q.tile0) continue;
-        if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
+      auto load_q = [&](const Pair& q) {
         mbar_expect_tx(bar(kQFull), q_bytes);
         const int qrow = (q.b * a.T_q + q.t0) * kHI;
         tma_load_2d(q_base, &qmap, 0, qrow, bar(kQFull));
         tma_load_2d(q_base + q_blk, &qmap, 64, qrow, bar(kQFull));
+      };
+      int w_first = -1;
+      for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
+        const Pair q = make_pair(p, w);
+        if (q.tile1 <= q.tile0) continue;
+        load_q(q);
+        w_first = w;
+        break;
+      }
+      pdl_wait();
+      for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
+        const Pair q = make_pair(p, w);
+        if (q.tile1 <= q.tile0) continue;
+        if (w != w_first) {
+          if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
+          load_q(q);
+        }
         for (int tile = q.tile0; tile < q.tile1; ++tile, ++kt) {
           const uint32_t s = kt % kStages;
           if (kt >= (uint32_t)kStages)
@@ -151,9 +168,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++active;
       }
     }
+    if (lane != 0) pdl_wait();
     __syncwarp();
   } else if (warp == 1) {
     // =================== MMA issuer ===================
+    pdl_wait();
     if (lane == 0) {
       uint32_t kt = 0, at = 0, active = 0;
       const uint32_t idesc = idesc_bf16(128, 64 * G, 0, 0);
@@ -195,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;       // key row within the tile
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
     uint32_t at = 0;
+    bool first = true;
     for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
       const Pair q = make_pair(p, w);
       if (q.tile1 <= q.tile0) continue;
@@ -203,6 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int g = e / kHI;
         w_s[e] = g < q.nrows ? bf2f(a.w[((int64_t)q.b * a.T_q + q.t0 + g) * kHI + (e % kHI)]) : 0.f;
       }
+      if (first) pdl_wait();  // before the first score is written
+      first = false;
       named_bar(1, 128);
       for (int tile = q.tile0; tile < q.tile1; ++tile, ++at) {
         const uint32_t ab = at & 1u;

@@ -26,7 +26,9 @@
 //              PV products that read it.
 // qhat_prep_kernel computes q^ = RoPE_pos(RMSNorm(q) * g) for every query
 // (one warp per head, coalesced) straight into that shared-memory image
-// (K-major, 128-byte swizzle, 64 KB per query) in the workspace.
+// (K-major, 128-byte swizzle, 64 KB per query) in the workspace.  Decode-
+// sized launches (kCompact) skip it: their softmax warps compute q^ into
+// shared memory themselves, before waiting for the preceding kernels.
 // Work items are (query, key split) pairs taken round-robin by the blocks;
 // with one split the block writes the final bf16 output, otherwise the
 // float partials (max, sum, accumulator) the combine kernel merges.

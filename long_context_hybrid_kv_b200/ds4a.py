@@ -85,19 +85,21 @@ def lib():
     return _lib
 
 
+# plain ints (or None) for pointer arguments: ctypes converts them through
+# the c_void_p argtypes without a wrapper object per argument
 def _ptr(t):
     if t is None:
         return None
-    return _P(t.data_ptr())
+    return t.data_ptr()
 
 
 def _stream(stream):
     if stream is None:
         import torch
-        return _P(torch.cuda.current_stream().cuda_stream)
+        return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, int):
-        return _P(stream)
-    return _P(stream.cuda_stream)
+        return stream
+    return stream.cuda_stream
 
 
 def _ok(rc: int, where: str):

@@ -98,13 +98,6 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-// order-preserving map float -> uint32 (larger float -> larger key)
 // 2^x with the hardware approximation (about 2 ulp)
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -112,13 +105,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// order-preserving map float -> uint32 (larger float -> larger key)
 __device__ __forceinline__ unsigned int f2key(float f) {
   unsigned int b = __float_as_uint(f);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float key2f(unsigned int k) {
-  unsigned int b = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
-  return __uint_as_float(b);
 }
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current

@@ -172,25 +172,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
-      "%29, %30, %31, %32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -246,11 +227,6 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-// arrive on the mbarrier once every cp.async this thread issued so far has
-// landed (the barrier's expected count already includes this arrival)
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
 __device__ __forceinline__ void st_shared_zero16(uint32_t dst) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
 }
@@ -303,61 +279,6 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
 // 128-byte swizzle inside a 1024-byte atom: 16-byte chunk c of row r
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
   return row * 128u + (((chunk ^ row) & 7u) << 4);
-}
-
-// Reduce 64 values per lane over the 32 lanes of a warp; afterwards lane l
-// holds the results of entries 2l and 2l+1 (a transposing butterfly: 62
-// shuffles instead of 320).
-template <bool kMax>
-__device__ __forceinline__ void warp_reduce64(const float (&v)[64], float& r0, float& r1) {
-  const int lane = threadIdx.x & 31;
-  float a[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const bool up = lane & 16;
-    const float send = up ? v[i] : v[i + 32];
-    const float keep = up ? v[i + 32] : v[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 16);
-    a[i] = kMax ? fmaxf(keep, got) : keep + got;
-  }
-  float b[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const bool up = lane & 8;
-    const float send = up ? a[i] : a[i + 16];
-    const float keep = up ? a[i + 16] : a[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 8);
-    b[i] = kMax ? fmaxf(keep, got) : keep + got;
-  }
-  float c[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const bool up = lane & 4;
-    const float send = up ? b[i] : b[i + 8];
-    const float keep = up ? b[i + 8] : b[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 4);
-    c[i] = kMax ? fmaxf(keep, got) : keep + got;
-  }
-  float d[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const bool up = lane & 2;
-    const float send = up ? c[i] : c[i + 4];
-    const float keep = up ? c[i + 4] : c[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 2);
-    d[i] = kMax ? fmaxf(keep, got) : keep + got;
-  }
-  float e[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const bool up = lane & 1;
-    const float send = up ? d[i] : d[i + 2];
-    const float keep = up ? d[i + 2] : d[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 1);
-    e[i] = kMax ? fmaxf(keep, got) : keep + got;
-  }
-  r0 = e[0];
-  r1 = e[1];
 }
 
 // Reduce 32 values per lane over the 32 lanes of a warp; afterwards lane l

@@ -7,13 +7,17 @@
 // lands in tensor memory; the epilogue thread that owns a key row applies
 // the ReLU and the head weights in registers and writes the G scores.
 //
-// Thread block (192 threads, one per SM):
+// Thread block (320 threads, one per SM):
 //   warp 0     lane 0 streams K tiles with TMA (3-D map [B][N_c][128],
 //              128-byte swizzle, two 64-dim boxes per tile) into 4 stages,
 //              and the group's queries (2-D map over [B*T_q*64][128]);
 //   warp 1     TMEM allocation; lane 0 issues the MMAs (8 x K=16 per tile)
 //              into two accumulator buffers;
-//   warps 2-5  epilogue (they cover the four TMEM lane quarters).
+//   warps 2-9  epilogue: two warps per TMEM lane quarter, each with every
+//              other query of the group (with G = 1 the second warp of a
+//              quarter idles).  The epilogue bounds the prefill indexer (it
+//              took ~40 % of its time with one warp per quarter), so two
+//              warps per SM sub-partition hide each other's latencies.
 // Work: (query group, chunk of key tiles) pairs, taken round-robin by the
 // blocks; pairs past a group's visible entries are skipped.
 #include <cuda.h>
@@ -30,7 +34,11 @@ constexpr int kHI = 64;
 constexpr int kDI = 128;
 constexpr int kKT = 128;      // keys per tile
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 256;
+// registers are granted for whole groups of four warps: cap the kernel's
+// registers as for 384 threads so that its 10 warps fit in one SM's file
+constexpr int kRegBoundThreads = 384;
 constexpr int kMaxG = 4;
 
 constexpr uint32_t kOffK = 0;                       // kStages x 2 blocks x 16 KB
@@ -81,7 +89,7 @@ __device__ __forceinline__ Pair make_pair(const TcIndexParams& p, int w) {
   return q;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kRegBoundThreads, 1)
     index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                     const TcIndexParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -111,8 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(kQEmpty), 1);
     mbar_init(bar(kAccFull0), 1);
     mbar_init(bar(kAccFull1), 1);
-    mbar_init(bar(kAccEmpty0), 128);
-    mbar_init(bar(kAccEmpty1), 128);
+    mbar_init(bar(kAccEmpty0), kEpiThreads);
+    mbar_init(bar(kAccEmpty1), kEpiThreads);
     mbar_init(bar(kDrain), 1);
     fence_barrier_init();
   }
@@ -209,34 +217,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // =================== epilogue ===================
-    const int et = tid - 64;                 // 0..127
+    const int et = tid - 64;                 // 0..255
     const int quarter = warp & 3;            // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;       // key row within the tile
+    const int gpar = (warp - 2) >> 2;        // this warp's queries: g = gpar, gpar + 2
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
     uint32_t at = 0;
     bool first = true;
     for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
       const Pair q = make_pair(p, w);
       if (q.tile1 <= q.tile0) continue;
-      named_bar(1, 128);  // everyone is done with the previous pair's weights
-      for (int e = et; e < G * kHI; e += 128) {
+      named_bar(1, kEpiThreads);  // everyone is done with the previous pair's weights
+      for (int e = et; e < G * kHI; e += kEpiThreads) {
         const int g = e / kHI;
         w_s[e] = g < q.nrows ? bf2f(a.w[((int64_t)q.b * a.T_q + q.t0 + g) * kHI + (e % kHI)]) : 0.f;
       }
       if (first) pdl_wait();  // before the first score is written
       first = false;
-      named_bar(1, 128);
+      named_bar(1, kEpiThreads);
       for (int tile = q.tile0; tile < q.tile1; ++tile, ++at) {
         const uint32_t ab = at & 1u;
         mbar_wait(bar(kAccFull0 + ab), (at >> 1) & 1u, abort_flag, err);
         tc_fence_after();
-        float sc[kMaxG];
+        float sc[kMaxG / 2];
 #pragma unroll
-        for (int g = 0; g < kMaxG; ++g) {
-          sc[g] = 0.f;
+        for (int gi = 0; gi < kMaxG / 2; ++gi) {
+          const int g = gpar + 2 * gi;
+          sc[gi] = 0.f;
           if (g < G) {
-            // four independent sums per query (one epilogue warp per SM
-            // sub-partition cannot hide a 64-long FMA chain)
+            // four independent sums per query (a 64-long FMA chain would
+            // stall the warp)
             float s4[4] = {0.f, 0.f, 0.f, 0.f};
             // both 32-column halves in flight, one wait
             float v[2][32];
@@ -257,16 +267,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s4[3] = fmaf(ww.w, fmaxf(v[half][i + 3], 0.f), s4[3]);
               }
             }
-            sc[g] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            sc[gi] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
           }
         }
         tc_fence_before();
         mbar_arrive(bar(kAccEmpty0 + ab));
         const int s = tile * kKT + r;
 #pragma unroll
-        for (int g = 0; g < kMaxG; ++g)
-          if (g < q.nrows && s < q.n_vis[g])
-            a.scores[((int64_t)q.b * a.T_q + q.t0 + g) * a.N_c + s] = sc[g];
+        for (int gi = 0; gi < kMaxG / 2; ++gi) {
+          const int g = gpar + 2 * gi;
+          const int nv = gpar ? q.n_vis[2 * gi + 1] : q.n_vis[2 * gi];  // constant indices
+          if (g < q.nrows && s < nv)
+            a.scores[((int64_t)q.b * a.T_q + q.t0 + g) * a.N_c + s] = sc[gi];
+        }
       }
     }
   }

@@ -287,10 +287,10 @@ def test_attend_many_splits_and_empty_splits():
 
 def test_attend_prefill_sized_launches():
     # more than 148 queries: the prefill form of the kernel (work items
-    # round-robin over the blocks, selected rows gathered by TMA gather4 in
-    # groups of four slots, padding slots masked); positions cover empty,
-    # partial and full windows and selected counts that are not multiples
-    # of four
+    # round-robin over the blocks, q-hat prepared by its own kernel, the
+    # next item built during the last tile); positions cover empty, partial
+    # and full windows, selected counts that are not multiples of four and
+    # ragged last tiles
     pos = sorted(set([0, 1, 2, 3, 5, 6, 7, 126, 127, 128, 129, 130, 131] + list(range(200, 3999, 23))))
     assert len(pos) > 148
     _attend_case("pf", FLASH, 1, pos, 1000, True, 4096)

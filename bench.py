@@ -117,33 +117,36 @@ def _csa_prefill_layer(w, dev, T, toy=None):
     return ly
 
 
-def _run_layer(ly):
+def _run_layer(ly, stream=None):
+    """One layer's calls on `stream` (a CUDA stream handle; None = the
+    current stream, looked up by each call)."""
     import long_context_hybrid_kv_b200 as L
 
     t = ly.t
+    S = stream
     if ly.kind == "csa":
         L.ds4a_compress(ly.cfg, t["kv_ca"], t["kv_za"], t["kv_ba"], t["pool"], cb=t["kv_cb"], zb=t["kv_zb"],
                         bias_b=t["kv_bb"], norm_g=t["kv_g"], tok_begin=ly.tok_begin,
-                        entry_begin=ly.entry, entry_end=ly.entry + 1)
+                        entry_begin=ly.entry, entry_end=ly.entry + 1, stream=S)
         L.ds4a_compress(ly.cfg, t["ix_ca"], t["ix_za"], t["ix_ba"], t["ki"], cb=t["ix_cb"], zb=t["ix_zb"],
                         bias_b=t["ix_bb"], tok_begin=ly.tok_begin, entry_begin=ly.entry,
-                        entry_end=ly.entry + 1)
-        L.ds4a_index_topk(ly.cfg, ly.q_pos, t["qi"], t["wi"], t["ki"], ly.n_c, ly.idx, ly.ws_index)
+                        entry_end=ly.entry + 1, stream=S)
+        L.ds4a_index_topk(ly.cfg, ly.q_pos, t["qi"], t["wi"], t["ki"], ly.n_c, ly.idx, ly.ws_index, stream=S)
         L.ds4a_sparse_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], t["pool"], ly.n_c, ly.idx, t["win"],
-                             t["win"].shape[1], t["sink"], ly.out, ly.ws_att)
+                             t["win"].shape[1], t["sink"], ly.out, ly.ws_att, stream=S)
     elif ly.kind == "hca":
         L.ds4a_compress(ly.cfg, t["kv_c"], t["kv_z"], t["kv_b"], t["pool"], norm_g=t["kv_g"],
-                        tok_begin=ly.tok_begin, entry_begin=ly.entry, entry_end=ly.entry + 1)
+                        tok_begin=ly.tok_begin, entry_begin=ly.entry, entry_end=ly.entry + 1, stream=S)
         L.ds4a_hca_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], t["pool"], ly.n_c, t["win"],
-                          t["win"].shape[1], t["sink"], ly.out, ly.ws_att)
+                          t["win"].shape[1], t["sink"], ly.out, ly.ws_att, stream=S)
     else:  # prefill
         L.ds4a_compress(ly.cfg, t["kv_ca"], t["kv_za"], t["kv_ba"], ly.pool, cb=t["kv_cb"], zb=t["kv_zb"],
-                        bias_b=t["kv_bb"], norm_g=t["kv_g"], entry_begin=0, entry_end=ly.n_c)
+                        bias_b=t["kv_bb"], norm_g=t["kv_g"], entry_begin=0, entry_end=ly.n_c, stream=S)
         L.ds4a_compress(ly.cfg, t["ix_ca"], t["ix_za"], t["ix_ba"], ly.ki, cb=t["ix_cb"], zb=t["ix_zb"],
-                        bias_b=t["ix_bb"], entry_begin=0, entry_end=ly.n_c)
-        L.ds4a_index_topk(ly.cfg, ly.q_pos, t["qi"], t["wi"], ly.ki, ly.n_c, ly.idx, ly.ws_index)
+                        bias_b=t["ix_bb"], entry_begin=0, entry_end=ly.n_c, stream=S)
+        L.ds4a_index_topk(ly.cfg, ly.q_pos, t["qi"], t["wi"], ly.ki, ly.n_c, ly.idx, ly.ws_index, stream=S)
         L.ds4a_sparse_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], ly.pool, ly.n_c, ly.idx, t["win"],
-                             ly.T, t["sink"], ly.out, ly.ws_att)
+                             ly.T, t["sink"], ly.out, ly.ws_att, stream=S)
 
 
 class State:
@@ -180,8 +183,11 @@ class State:
         self.tensors = T
 
     def step(self):
+        import torch
+
+        s = torch.cuda.current_stream().cuda_stream  # once per step
         for ly in self.layers:
-            _run_layer(ly)
+            _run_layer(ly, s)
 
     # per-step input / output tensors for the end-to-end measurement
     def step_io(self):

@@ -16,15 +16,18 @@ void fill_rope_theta(RopeTheta* r, int rope_dim, float base) {
 }
 
 unsigned int* err_word() {
-  static unsigned int* addr[64] = {nullptr};
+  // filled once per device; concurrent first calls store the same address
+  static std::atomic<unsigned int*> addr[kMaxDevices];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  unsigned int* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<unsigned int*>(p);
+    a = static_cast<unsigned int*>(p);
+    addr[dev].store(a, std::memory_order_release);
   }
-  return addr[dev];
+  return a;
 }
 
 // ---------------------------------------------------------------------------

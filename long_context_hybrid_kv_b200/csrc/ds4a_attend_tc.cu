@@ -793,7 +793,7 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   a.ws = reinterpret_cast<float*>(qimg + (size_t)rows * 65536u);
   const int n_items = rows * a.n_splits;
   const bool compact = n_items <= 148;  // every block takes at most one item
-  static int cache[16], cache_c[16];
+  static std::atomic<int> cache[kMaxDevices], cache_c[kMaxDevices];
   cudaError_t e = compact ? ensure_smem(attend_tc_kernel<true>, (int)kSmemBytes, cache_c)
                           : ensure_smem(attend_tc_kernel<false>, (int)kSmemBytes, cache);
   if (e != cudaSuccess) return e;

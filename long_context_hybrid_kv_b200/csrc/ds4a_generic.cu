@@ -355,7 +355,7 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
     while (Z < 8 && (int64_t)n * a.B * Z * 2 <= 148 && n_terms / (2 * Z) >= 16 && a.c % (2 * Z * 2) == 0) Z *= 2;
   if (Z > 1) {
     const size_t smem = (size_t)(3 * G * a.c + 3 * a.c + a.c / Z) * sizeof(float);
-    static int cache_s[16];
+    static std::atomic<int> cache_s[kMaxDevices];
     cudaError_t e = ensure_smem(compress_split_kernel<8>, (int)smem, cache_s);
     if (e != cudaSuccess) return e;
     TraceScope tr("compress", s);
@@ -363,7 +363,7 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
                               Z);
   }
   const size_t smem = (size_t)(3 * G * a.c + a.c) * sizeof(float);
-  static int cache8[16], cache2[16];
+  static std::atomic<int> cache8[kMaxDevices], cache2[kMaxDevices];
   cudaError_t e = V == 8 ? ensure_smem(compress_kernel<8>, (int)smem, cache8)
                          : ensure_smem(compress_kernel<2>, (int)smem, cache2);
   if (e != cudaSuccess) return e;
@@ -422,7 +422,7 @@ cudaError_t launch_index_scores_generic(const IndexArgs& a, cudaStream_t s) {
   const int rows = a.B * a.T_q;
   if (rows <= 0 || a.N_c <= 0) return cudaSuccess;
   const size_t smem = (size_t)(a.H * a.D + a.H + kIdxKeys * (a.D + 1)) * sizeof(float);
-  static int cache[16];
+  static std::atomic<int> cache[kMaxDevices];
   cudaError_t e = ensure_smem(index_score_generic_kernel, (int)smem, cache);
   if (e != cudaSuccess) return e;
   TraceScope tr("index_score_generic", s);
@@ -763,7 +763,7 @@ cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   const size_t smem = (size_t)(a.H * a.D + kAttKT * a.D + a.H * kAttKT + ((3 * a.H + 1) & ~1)) * sizeof(float) +
                       (size_t)(a.R / 2 + 1) * sizeof(float2) + (size_t)a.H * a.D * sizeof(uint16_t);
-  static int cache[16];
+  static std::atomic<int> cache[kMaxDevices];
   cudaError_t e0 = ensure_smem(attend_generic_kernel, (int)smem, cache);
   if (e0 != cudaSuccess) return e0;
   {

@@ -295,17 +295,21 @@ __global__ void __launch_bounds__(kRegBoundThreads, 1)
 // The driver's tensor-map encoder, looked up once through the runtime (no
 // link against the driver library); null when the driver has none.
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // concurrent first calls store the same pointer
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 f = fn.load(std::memory_order_acquire);
+  if (!f) {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    else
+        q == cudaDriverEntryPointSuccess) {
+      f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+      fn.store(f, std::memory_order_release);
+    } else {
       (void)cudaGetLastError();
+    }
   }
-  return fn;
+  return f;
 }
 
 
@@ -355,7 +359,7 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  static int cache[16];
+  static std::atomic<int> cache[kMaxDevices];
   cudaError_t e = ensure_smem(index_tc_kernel, (int)kSmemBytes, cache);
   if (e != cudaSuccess) return e;
   const int grid = min(p.n_pairs, 148);

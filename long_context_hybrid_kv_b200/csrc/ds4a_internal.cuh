@@ -5,6 +5,9 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "ds4a.h"
 
 namespace ds4a {
@@ -111,22 +114,40 @@ __device__ __forceinline__ unsigned int f2key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// Per-device caches of the host side hold up to this many devices (a call
+// on a device beyond it fails with cudaErrorInvalidDevice).
+constexpr int kMaxDevices = 64;
+
+// Serialises the slow path of ensure_smem across host threads.
+inline std::mutex& smem_attr_mutex() {
+  static std::mutex m;
+  return m;
+}
+
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current
-// device when it is below that (cache[dev] holds the value set so far; up to
-// 16 devices).  Returns the error of cudaFuncSetAttribute, if any.
+// device when it is below that (cache[dev] holds the limit set so far).  The
+// limit only grows, under a lock, so a launch that another host thread
+// prepared for a smaller size stays valid.  Returns the error of
+// cudaFuncSetAttribute, if any.
 template <typename F>
-inline cudaError_t ensure_smem(F* f, int bytes, int* cache) {
+inline cudaError_t ensure_smem(F* f, int bytes, std::atomic<int>* cache) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) dev = 0;
-  if (cache[dev] >= bytes) return cudaSuccess;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return cudaErrorInvalidDevice;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (cache[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(smem_attr_mutex());
+  if (cache[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(f),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();  // do not leave it for a later launch check
     return e;
   }
-  cache[dev] = bytes;
+  cache[dev].store(bytes, std::memory_order_release);
   return cudaSuccess;
 }
 

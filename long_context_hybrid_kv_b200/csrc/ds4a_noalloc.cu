@@ -23,13 +23,15 @@ static __device__ __align__(256) float g_topk_scratch[kNoAllocScores];
 // memory: the kernels get the device address looked up here, once per
 // device, with that device current.
 float* scratch_for_current_device(int* rc) {
-  static float* addr[64] = {nullptr};
+  // filled once per device; concurrent first calls store the same address
+  static std::atomic<float*> addr[kMaxDevices];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     *rc = DS4A_ECUDA;
     return nullptr;
   }
-  if (!addr[dev]) {
+  float* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_topk_scratch);
     if (e != cudaSuccess || p == nullptr) {
@@ -37,10 +39,11 @@ float* scratch_for_current_device(int* rc) {
       *rc = DS4A_ECUDA;
       return nullptr;
     }
-    addr[dev] = static_cast<float*>(p);
+    a = static_cast<float*>(p);
+    addr[dev].store(a, std::memory_order_release);
   }
   *rc = DS4A_OK;
-  return addr[dev];
+  return a;
 }
 
 }  // namespace

@@ -364,7 +364,7 @@ cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   if (a.N_c <= kSmemRowMax) {
     const size_t smem = (size_t)((max(1, a.N_c) + 31) & ~31) * sizeof(unsigned int);
-    static int cache[16];
+    static std::atomic<int> cache[kMaxDevices];
     cudaError_t e = ensure_smem(topk_smem_kernel, (int)smem, cache);
     if (e != cudaSuccess) return e;
     TraceScope tr("topk_smem", s);
@@ -372,7 +372,7 @@ cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
   }
   if (a.N_c <= kCluster * kClusterSlice) {
     const size_t smem = (size_t)kClusterSlice * sizeof(unsigned int);
-    static int cache[16];
+    static std::atomic<int> cache[kMaxDevices];
     cudaError_t e = ensure_smem(topk_cluster_kernel, (int)smem, cache);
     if (e != cudaSuccess) return e;
     TraceScope tr("topk_cluster", s);

@@ -19,6 +19,10 @@
  * - Execution: every call is asynchronous on the given CUDA stream (NULL =
  *   the legacy default stream).  Pointers named "device" must be device (or
  *   managed) memory of the current device; "host" pointers are host memory.
+ * - Host threads: the compute calls may be made from several host threads
+ *   at once (the library's host state is a few per-device caches, filled
+ *   once under atomics or a lock); the launch trace is not thread safe, and
+ *   ds4a_check reads and clears the one error word of the current device.
  * - Overlap: the library's kernels are launched with programmatic dependent
  *   launch, so a kernel may start while the library kernel before it on the
  *   stream is still running.  It waits for that kernel before it reads what

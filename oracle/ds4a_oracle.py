@@ -30,7 +30,9 @@ listed with its reason in the design notes):
  R4  the index score has no scale, norm or RoPE: sum_h w_h ReLU(q_h . k).
  R5  softmax scale 1 / sqrt(head_dim).
  R6  RoPE on interleaved pairs (2j, 2j+1) of the last R dims, angle
-     pos * base^(-2j/R), base 10000, no YaRN.        -- base parity unpinned
+     pos * base^(-2j/R), base 10000, no YaRN (the pages print only one pair
+     at theta_0 = 1; the R = 64 ladder is pinned against an installed
+     library's interleaved RoPE).
  R7  compressed entry i carries position i * m.      -- parity unpinned
  R8  RMSNorm eps 1e-6 with a learned gain after normalising; window K=V
      rows arrive in final form.

@@ -145,6 +145,61 @@ def pin_rope_pairs_interleaved(O):
     _close(O.rope(x, 0, R, 10000.0), x, 0.0, "RoPE at 0")
 
 
+_LIB_ROPE: dict = {}
+
+
+def _library_rope(x, positions, base):
+    """Interleaved-pair RoPE as the installed transformers library computes
+    it for DeepSeek-V2 (its rotary embedding's default frequencies and its
+    complex-pair rotation), in float32: x [n, d] at positions [n]."""
+    key = (x.tobytes(), positions.tobytes(), base)
+    if key not in _LIB_ROPE:
+        from transformers import DeepseekV2Config
+        from transformers.models.deepseek_v2 import modeling_deepseek_v2 as M
+
+        d = x.shape[-1]
+        cfg = DeepseekV2Config(qk_rope_head_dim=d, rope_theta=base)
+        rot = M.DeepseekV2RotaryEmbedding(cfg)
+        xt = torch.from_numpy(x.astype(np.float32))[None, None]  # [1, 1, n, d]
+        fc = rot(xt, torch.from_numpy(positions.astype(np.int64))[None])
+        y, _ = M.apply_rotary_emb(xt, xt, fc)
+        _LIB_ROPE[key] = y[0, 0].double().numpy()
+    return _LIB_ROPE[key]
+
+
+def pin_rope_ladder_library(O):
+    """At the Flash rope width (R = 64, base 10000) the oracle's rotation of
+    the last R dims matches an installed library's interleaved-pair RoPE
+    (transformers, DeepSeek-V2), which fixes every pair's frequency
+    (RoFormer, Su et al. 2021, eq. 15: theta_j = base^(-2j/d)); the leading
+    D - R dims stay untouched."""
+    R, D = 64, 80
+    rng = np.random.default_rng(15)
+    positions = np.array([0, 1, 3, 17, 100, 1000, 4097])
+    x = rng.standard_normal((positions.size, D))
+    got = O.rope(x, positions, R, 10000.0)
+    _close(got[:, : D - R], x[:, : D - R], 0.0, "RoPE leaves the leading dims")
+    _close(got[:, D - R:], _library_rope(x[:, D - R:], positions, 10000.0), 2e-3, "RoPE vs library, R=64")
+
+
+def pin_store_bf16_library(O):
+    """The oracle's bfloat16 storage rounding equals torch's float32 ->
+    bfloat16 conversion (round to nearest, ties to even), including exact
+    halfway cases and values next to them."""
+    rng = np.random.default_rng(16)
+    x = (rng.standard_normal(4096) * np.exp2(rng.integers(-20, 20, 4096))).astype(np.float32)
+    hi = rng.integers(0, 1 << 15, 512, dtype=np.uint32) << np.uint32(16)
+    edge = np.concatenate([hi | np.uint32(0x8000), hi | np.uint32(0x10000 | 0x8000), hi | np.uint32(0x7FFF),
+                           hi | np.uint32(0x8001), hi | np.uint32(0x80000000 | 0x8000)]).view(np.float32)
+    x = np.concatenate([x, edge, np.float32([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38])])
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = O.store_bf16(x)
+    bad = np.flatnonzero(got != ref)
+    assert bad.size == 0, f"store_bf16 differs from torch at {bad.size} values, e.g. {x[bad[:3]]}"
+    _close(O.widen(got), torch.from_numpy(ref.view(np.int16)).view(torch.bfloat16).double().numpy(), 0.0,
+           "widen of bf16 bits")
+
+
 def pin_rms_norm_library(O):
     rng = np.random.default_rng(2)
     x = rng.standard_normal((5, 16)) * 3.0

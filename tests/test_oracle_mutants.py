@@ -43,6 +43,11 @@ MUTANTS = {
                                 '"""HCA: keys = every visible pool entry followed by the window."""\n    n_vis = n_c')],
     "window ring slot": [("return widen(win)[window_positions(pos, window) % win_cap]",
                           "return widen(win)[window_positions(pos, window) % win.shape[0] if False else window_positions(pos, window) - window_positions(pos, window)[0]]")],
+    "rope exponent -j/R": [("return base ** (-2.0 * j / rope_dim)", "return base ** (-1.0 * j / rope_dim)")],
+    "store_bf16 truncates": [("return ((b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)",
+                              "return (b >> np.uint32(16)).astype(np.uint16)")],
+    "store_bf16 ties away from zero": [("return ((b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)",
+                                        "return ((b + np.uint32(0x8000)) >> np.uint32(16)).astype(np.uint16)")],
     "pool row ignores idx": [("rows = np.concatenate([widen(pool)[sel], window_rows",
                               "rows = np.concatenate([widen(pool)[: sel.size], window_rows")],
 }

@@ -35,9 +35,22 @@ def lib():
         _lib = ctypes.CDLL(SO)
         _lib.ds4gen_fill.restype = ctypes.c_int
         _lib.ds4gen_fill.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64,
-                                     ctypes.c_uint64, ctypes.c_float, ctypes.c_int, ctypes.c_float,
+                                     ctypes.c_uint64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
                                      ctypes.c_int, ctypes.c_float, ctypes.c_void_p]
     return _lib
+
+
+_tables: dict = {}
+
+
+def _table(device):
+    """The host's normal table, uploaded once per device."""
+    import torch
+
+    key = str(device)
+    if key not in _tables:
+        _tables[key] = torch.from_numpy(host.normal_table().reshape(-1).copy()).to(device)
+    return _tables[key]
 
 
 def fill(t, seed: int, name: str, scale=None, offset=None, start: int = 0, stream=None):
@@ -49,7 +62,7 @@ def fill(t, seed: int, name: str, scale=None, offset=None, start: int = 0, strea
     s = torch.cuda.current_stream().cuda_stream if stream is None else stream
     rc = lib().ds4gen_fill(
         ctypes.c_void_p(t.data_ptr()), is_bf16, t.numel(), host.stream_key(seed, name), start,
-        float(host.NORMAL_SCALE), scale is not None, 0.0 if scale is None else float(np.float32(scale)),
+        ctypes.c_void_p(_table(t.device).data_ptr()), scale is not None, 0.0 if scale is None else float(np.float32(scale)),
         offset is not None, 0.0 if offset is None else float(np.float32(offset)), ctypes.c_void_p(s))
     if rc != 0:
         raise RuntimeError(f"ds4gen_fill failed ({rc})")

@@ -1,6 +1,7 @@
 """The seeded generator: its definition (SplitMix64 counter form, FNV-1a keys,
-Irwin-Hall normal approximation, RNE bfloat16) checked against plain
-Python-integer restatements and torch's own float32 -> bfloat16 rounding."""
+table inverse of the normal CDF, RNE bfloat16) checked against plain
+Python-integer restatements, scipy's normal distribution and torch's own
+float32 -> bfloat16 rounding."""
 import math
 
 import numpy as np
@@ -38,14 +39,63 @@ def test_fnv1a_known_values():
     assert host.fnv1a64("a") == 0xAF63DC4C8601EC8C
 
 
-def test_normal_moments_and_range():
-    x = host.normal_f32(1, "moments", (1 << 20,)).astype(np.float64)
-    assert abs(x.mean()) < 0.005
-    assert abs(x.var() - 1.0) < 0.01
-    assert np.abs(x).max() <= 2 * math.sqrt(3) + 1e-6
-    # Irwin-Hall(4) kurtosis is 3 - 1.2/4 = 2.7
+def test_normal_is_standard_normal():
+    from scipy import stats
+
+    x = host.normal_f32(1, "moments", (1 << 21,)).astype(np.float64)
+    assert abs(x.mean()) < 0.003
+    assert abs(x.var() - 1.0) < 0.004
     kurt = np.mean(x ** 4) / np.mean(x ** 2) ** 2
-    assert abs(kurt - 2.7) < 0.03
+    assert abs(kurt - 3.0) < 0.03, kurt
+    # Kolmogorov-Smirnov against N(0, 1): at 2^21 samples the 1% critical
+    # value is 1.63 / sqrt(n) = 0.0011
+    assert stats.kstest(x, "norm").statistic < 0.0011
+    # the tails are there (Irwin-Hall-type sums stop near 3.5)
+    for t in (3.0, 4.0):
+        want = 2 * stats.norm.sf(t) * x.size
+        got = np.count_nonzero(np.abs(x) > t)
+        assert abs(got - want) < 5 * math.sqrt(want) + 1, (t, got, want)
+    assert np.abs(x).max() > 4.5
+
+
+def test_normal_table_accuracy():
+    """The piecewise-linear inverse CDF stays within 1e-6 (+ float32
+    rounding) of the exact quantile at the middle of every segment."""
+    from scipy.special import ndtri
+
+    tab = host.normal_table().astype(np.float64)
+    e = np.arange(63, dtype=np.float64)[:, None]
+    s = np.arange(256, dtype=np.float64)[None, :]
+    p_mid = (1.0 + (s + 0.5) / 256) * np.exp2(-(e + 2.0))
+    exact = -ndtri(p_mid)
+    interp = tab[:, :, 0] + 0.5 * tab[:, :, 1]
+    assert np.max(np.abs(interp - exact) / (1.0 + exact)) < 1.5e-6
+    assert np.all(tab[:, :, 1] < 0) and np.all(tab[:, :, 0] > 0)
+
+
+def _normal_by_integers(u: int) -> float:
+    """One output of the normal definition, restated with Python integers
+    and float32 scalars."""
+    tab = host.normal_table()
+    v = max(u & ((1 << 63) - 1), 1)
+    e = 62 - (v.bit_length() - 1)
+    w = v << e
+    seg = (w >> 54) & 0xFF
+    f = np.float32((w >> 31) & 0x7FFFFF) * np.float32(2.0 ** -23)
+    x = np.float32(tab[e, seg, 0] + np.float32(f * tab[e, seg, 1]))
+    return float(-x if u >> 63 else x)
+
+
+def test_normal_definition_bit_by_bit():
+    key = host.stream_key(7, "def")
+    us = [int(v) for v in host.u64(key, 0, 64)]
+    us += [0, 1, (1 << 63) - 1, 1 << 63, (1 << 63) + 1, (1 << 64) - 1, 1 << 40, (1 << 62) + (1 << 61)]
+    got = host._normal_from_u64(np.array(us, dtype=np.uint64))
+    want = np.array([_normal_by_integers(u) for u in us], dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    # the deepest octave reaches p = 2^-64 and the shallowest starts at 0
+    assert 9.0 < float(got[us.index(1)]) < 9.2 and -9.2 < float(got[us.index(1 << 63)]) < -9.0
+    assert 0.0 < float(got[us.index((1 << 63) - 1)]) < 1e-3
 
 
 def test_bf16_rounding_matches_torch():

@@ -57,6 +57,11 @@ extern "C" int ds4a_index_topk_noalloc(const ds4a_layer_cfg* cfg, int B, int T_q
   if (B < 0 || T_q < 0 || N_c < 0) return DS4A_EINVAL;
   const size_t n_scores = (size_t)B * (size_t)T_q * (size_t)N_c;
   if (n_scores > ds4a::kNoAllocScores) return DS4A_ENOSPACE;
+  // no scores to write: the scratch is not needed, so its address is not
+  // looked up (such a call may come first and inside a stream capture)
+  if (n_scores == 0)
+    return ds4a_index_topk(cfg, B, T_q, q_pos, q_idx, w_idx, k_idx, k_bstride, N_c, idx_out, score_out,
+                           nullptr, 0, stream);
   int rc = DS4A_OK;
   float* scratch = ds4a::scratch_for_current_device(&rc);
   if (rc != DS4A_OK) return rc;

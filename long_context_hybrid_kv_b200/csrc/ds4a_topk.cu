@@ -1,6 +1,6 @@
 // Top-k selector of the Lightning indexer ("DeepSeek-v4 Beyond Basics"
-// 3.2.2 eq. 17; "Phase 1 Module 1" "Top-k selects", "only kicks in once
-// there are more than 512 rows"): keep the k highest of a row's n_vis
+// 3.2.2 eq. 17; "Phase 1 Module 1", section on the indexer: the selection
+// prunes only when more entries are visible than k): keep the k highest of a row's n_vis
 // visible scores, ties to the lower index; write the kept indices
 // ascending, padded with -1 when n_vis <= k.
 //

@@ -160,8 +160,9 @@ def compress(m: int, entry_begin: int, entry_end: int, tok_begin: int,
 
 # --------------------------------------------------------------------------
 # (2) Lightning indexer and top-k selector
-# [beyond] 3.2.2, eqs. 13-17; [module1] "It scores every compressed row",
-# "Top-k selects", "only kicks in once there are more than 512 rows";
+# [beyond] 3.2.2, eqs. 13-17; [module1] section on the indexer (every
+# compressed row is scored; the selection prunes only when more than k
+# entries are visible);
 # [hf-doc] attention-mask layout: -1 sentinels, visibility w < (t+1)//m.
 # --------------------------------------------------------------------------
 def visible_entries(pos: int, m: int) -> int:

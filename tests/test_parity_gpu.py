@@ -399,21 +399,48 @@ def _decode_csa_ref(w, ly, bsel):
     return res
 
 
+def _reattend_with(ly, pool, n_c, win, win_cap, oracle_idx: dict):
+    """The layer's attention rerun on the GPU, in the same launch
+    configuration, with the oracle's index set substituted for the rows in
+    ``oracle_idx`` ((b, t) -> int indices).  Rows whose GPU set differs from
+    the oracle's only inside the tie zone are checked this way: the input
+    flows from the oracle to the GPU, never back."""
+    idx2 = ly.idx.clone()
+    for (b, t), ix in oracle_idx.items():
+        idx2[b, t] = torch.from_numpy(np.asarray(ix, np.int32)).to(idx2.device)
+    out2 = torch.empty_like(ly.out)
+    t_ = ly.t
+    L.ds4a_sparse_attend(ly.cfg, ly.q_pos, t_["q"], t_["q_norm_g"], pool, n_c, idx2, win, win_cap,
+                         t_["sink"], out2, ly.ws_att)
+    check_ok()
+    return f64(out2)
+
+
 def _check_csa_decode(st, ly, w, bsel):
+    """Every sampled sequence: compressed entries, the top-k set (tie rule)
+    and the attention output, each against the oracle's own chain."""
     ref = _decode_csa_ref(w, ly, bsel)
     gpool = ly.t["pool"]
     gki = ly.t["ki"]
     gidx = ly.idx.cpu().numpy()
     gout = f64(ly.out)
     e = w.n_csa - 1
+    redo = {}
     for b, (ent, kent, idx, scores, out) in ref.items():
         assert C.max_abs_rel(f64(gpool[b, e]), ent) < C.OUT_TOL
         assert C.max_abs_rel(f64(gki[b, e]), kent) < C.OUT_TOL
         msg = C.check_topk_row(gidx[b, 0], scores, w.csa.topk)
         assert msg is None, f"seq {b}: {msg}"
-        if np.array_equal(gidx[b, 0], idx):
-            err = C.max_abs_rel(gout[b, 0], out)
-            assert err < C.OUT_TOL, f"seq {b}: attend err {err}"
+        if not np.array_equal(gidx[b, 0], idx):
+            redo[(b, 0)] = idx
+    gout2 = _reattend_with(ly, gpool, ly.n_c, ly.t["win"], ly.t["win"].shape[1], redo) if redo else None
+    compared = 0
+    for b, (ent, kent, idx, scores, out) in ref.items():
+        got = gout2[b, 0] if (b, 0) in redo else gout[b, 0]
+        err = C.max_abs_rel(got, out)
+        assert err < C.OUT_TOL, f"seq {b}: attend err {err} (oracle index set: {(b, 0) in redo})"
+        compared += 1
+    assert compared == len(bsel)
 
 
 def _check_hca_decode(st, ly, w, bsel):
@@ -454,9 +481,14 @@ def test_workload_toy_csa_prefill():
         assert C.check_topk_row(gidx[0, t], scores[(0, t)], c.topk) is None
     out = O.csa_attend_batch(x["csa.q"], x["csa.q_norm_g"], O.store_bf16(pool), idx, x["csa.win"], 64,
                              x["csa.sink"], qp, c)
-    rows = [t for t in range(64) if np.array_equal(gidx[0, t], idx[0, t])]
-    assert len(rows) >= 62
-    assert C.max_abs_rel(f64(ly.out)[0, rows], out[0, rows]) < C.OUT_TOL
+    redo = {(0, t): idx[0, t] for t in range(64) if not np.array_equal(gidx[0, t], idx[0, t])}
+    got = f64(ly.out)
+    if redo:
+        got2 = _reattend_with(ly, ly.pool, n, ly.t["win"], ly.T, redo)
+        for (_, t) in redo:
+            got[0, t] = got2[0, t]
+    # every one of the 64 rows is compared
+    assert C.max_abs_rel(got[0], out[0]) < C.OUT_TOL
 
 
 def test_workload_csa_decode_b1_8k():
@@ -510,6 +542,7 @@ def test_workload_csa_prefill_16k_sampled():
     gidx = ly.idx.cpu().numpy()
     gout = ly.out
     pb, kb = O.store_bf16(pool), O.store_bf16(ki)
+    refs, redo = {}, {}
     for t in rows:
         qi = W.host_rows(w, "csa.qi", t * c.idx_heads + np.arange(c.idx_heads))
         wi = W.host_rows(w, "csa.wi", np.array([t]))[0]
@@ -517,7 +550,14 @@ def test_workload_csa_prefill_16k_sampled():
         idx, scores = O.index_topk(qi, wi, kb, t, c.ratio, c.topk, n)
         msg = C.check_topk_row(gidx[0, t], scores, c.topk)
         assert msg is None, f"row {t}: {msg}"
-        if np.array_equal(gidx[0, t], idx):
-            out = O.csa_attend(q, Hs["q_norm_g"], pb, idx, Hs["win"][0], 16384, Hs["sink"], t, c)
-            err = C.max_abs_rel(f64(gout[0, t]), out)
-            assert err < C.OUT_TOL, f"row {t}: err {err}"
+        refs[t] = O.csa_attend(q, Hs["q_norm_g"], pb, idx, Hs["win"][0], 16384, Hs["sink"], t, c)
+        if not np.array_equal(gidx[0, t], idx):
+            redo[(0, t)] = idx
+    got2 = _reattend_with(ly, ly.pool, n, ly.t["win"], ly.T, redo) if redo else None
+    compared = 0
+    for t in rows:
+        got = got2[0, t] if (0, t) in redo else f64(gout[0, t])
+        err = C.max_abs_rel(got, refs[t])
+        assert err < C.OUT_TOL, f"row {t}: err {err} (oracle index set: {(0, t) in redo})"
+        compared += 1
+    assert compared == len(rows)

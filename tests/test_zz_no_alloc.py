@@ -53,6 +53,31 @@ def test_noalloc_matches_workspace_call(shape):
         assert np.max(np.abs(a[fin] - b[fin]) / (np.abs(b[fin]) + 1e-6)) <= 1e-6, f"call {call}: scores differ"
 
 
+def test_noalloc_fills_the_whole_scratch():
+    # exactly 2^21 scores (B * T_q * N_c = 1 * 16 * 131072) on the
+    # tensor-core scorer: accepted, and equal to the workspace call; one
+    # more entry is rejected
+    torch.cuda.set_device(0)
+    B, Tq, n_c = 1, 16, 131072
+    positions = [4 * n_c - 1 - 37 * i for i in range(Tq)]
+    cfg = L.layer_cfg(W.FLASH_CSA)
+    k = W.FLASH_CSA.topk
+    for call, seed in enumerate((21, 22)):
+        pos, qi, wi, ki = _inputs(seed, B, Tq, n_c, positions)
+        idx_ref = torch.empty((B, Tq, k), dtype=torch.int32, device="cuda")
+        ws = torch.empty(L.ds4a_index_topk_workspace(cfg, B, Tq, n_c) // 4, dtype=torch.float32, device="cuda")
+        L.ds4a_index_topk(cfg, pos, qi, wi, ki, n_c, idx_ref, ws)
+        idx = torch.full((B, Tq, k), -7, dtype=torch.int32, device="cuda")
+        L.ds4a_index_topk_noalloc(cfg, pos, qi, wi, ki, n_c, idx)
+        rc, bits = L.ds4a_check()
+        assert rc == 0, (rc, bits)
+        assert torch.equal(idx, idx_ref), f"call {call}: indices differ"
+    kbig = torch.empty((B, n_c + 1, W.FLASH_CSA.idx_dim), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(L.Ds4aError) as ex:
+        L.ds4a_index_topk_noalloc(cfg, pos, qi, wi, kbig, n_c + 1, idx)
+    assert ex.value.code == L.DS4A_ENOSPACE
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     cfg = L.layer_cfg(W.FLASH_CSA)
     A = ctypes.c_void_p(1 << 20)

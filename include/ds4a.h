@@ -182,11 +182,13 @@ int ds4a_index_topk_noalloc(const ds4a_layer_cfg* cfg, int B, int T_q, const int
                             const ds4a_bf16* k_idx, int64_t k_bstride, int N_c,
                             int32_t* idx_out, float* score_out, ds4a_stream stream);
 
-/* Bytes of workspace the attend calls can use for these sizes.  On the
- * tensor-core path (64 heads x 512) it holds one prepared query (64 KiB)
- * per query plus the partial results of key splits (used when few queries
- * are given).  Passing less is allowed: the work is then split less, and
- * below B * T_q * 64 KiB the CUDA-core path runs instead. */
+/* Bytes of workspace the attend calls can use for these sizes.  For the
+ * Flash head shape (64 heads x 512, tensor cores) it holds one prepared
+ * query (64 KiB) per query plus the partial results of key splits (used
+ * when few queries are given).  Passing less is allowed down to
+ * B * T_q * 64 KiB (the work is then split less); below that the call
+ * returns DS4A_ENOSPACE.  Other head shapes run on CUDA cores and use the
+ * workspace only for key splits (any size, NULL included, is accepted). */
 size_t ds4a_attend_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c, int sparse);
 
 /*
@@ -227,6 +229,16 @@ int ds4a_hca_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_
                     int64_t pool_bstride, int N_c, const ds4a_bf16* win, int win_cap,
                     int64_t win_bstride, const float* sink, ds4a_bf16* out, void* ws,
                     size_t ws_bytes, ds4a_stream stream);
+
+/* Failure-detection self test (no counterpart on the pages): launches one
+ * block that waits, through the same bounded mbarrier wait the tensor-core
+ * kernels use, on a barrier no thread ever arrives at, with a limit of
+ * limit_cycles SM cycles (1 .. 2^32) instead of the kernels' ~2 s.  The
+ * wait runs out, the block records DS4A_DEV_TIMEOUT in the error word,
+ * writes 2 to *status_out (device int32; 1 would mean the barrier
+ * completed) and exits, so ds4a_check then returns DS4A_ETIMEOUT and the
+ * context stays usable.  No GPU fault is involved. */
+int ds4a_selftest_wait_timeout(int64_t limit_cycles, int32_t* status_out, ds4a_stream stream);
 
 /* Synchronise the stream, then read and clear the current device's error
  * word.  Returns DS4A_OK, DS4A_EDEVICE (bad index / position),

@@ -233,6 +233,7 @@ static int attend_common(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_
     return DS4A_EINVAL;
   if (ws_bytes > 0 && !ws) return DS4A_EINVAL;
 
+  const size_t have = ws ? ws_bytes : 0;
   AttendArgs a;
   a.B = B; a.T_q = T_q; a.H = cfg->n_heads; a.D = D; a.R = cfg->rope_dim; a.W = cfg->window;
   a.m = cfg->ratio; a.k = cfg->topk; a.N_c = N_c; a.win_cap = win_cap; a.sparse = sparse;
@@ -241,17 +242,17 @@ static int attend_common(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_
   a.idx = idx; a.win = win; a.win_bstride = win_bstride; a.sink = sink; a.out = out;
   a.ws = reinterpret_cast<float*>(ws);
   a.keys_max = (sparse ? cfg->topk : N_c) + cfg->window;
+  // the shape decides the kernel: 64 heads x 512 run on the tensor cores and
+  // need the prepared-query workspace (no silent second path); other shapes
+  // run the CUDA-core kernel
+  const bool tc = attend_tc_supported(a);
+  a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, tc, have, nullptr);
+  if (tc && a.n_splits == 0) return DS4A_ENOSPACE;
   fill_rope_theta(&a.rope, a.R, cfg->rope_base);
   a.err = err_word();
   if (!a.err) return DS4A_ECUDA;
-  const size_t have = ws ? ws_bytes : 0;
   cudaStream_t s = (cudaStream_t)stream;
-  if (attend_tc_supported(a)) {
-    a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, true, have, nullptr);
-    if (a.n_splits > 0) return cuda_rc(launch_attend_tc(a, s));
-  }
-  a.n_splits = attend_splits(B, T_q, a.keys_max, a.H, a.D, false, have, nullptr);
-  return cuda_rc(launch_attend_generic(a, s));
+  return cuda_rc(tc ? launch_attend_tc(a, s) : launch_attend_generic(a, s));
 }
 
 int ds4a_sparse_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,

@@ -53,14 +53,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase of the given parity to complete.  False on timeout or
 // when another thread of the block has aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* err) {
+                                          unsigned int* err, long long limit = kWaitCycles) {
   if (*abort_flag) return false;
   const long long t0 = clock64();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 63u) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         atomicOr(err, (unsigned int)DS4A_DEV_TIMEOUT);
         return false;

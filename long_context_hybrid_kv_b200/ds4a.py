@@ -16,7 +16,7 @@ __all__ = [
     "DS4A_ENOSPACE", "Ds4aError", "LayerCfg", "layer_cfg", "lib", "LIB_PATH", "ds4a_compress",
     "ds4a_index_topk_workspace", "ds4a_index_topk", "ds4a_index_topk_noalloc", "ds4a_attend_workspace", "ds4a_sparse_attend",
     "ds4a_hca_attend", "ds4a_check", "ds4a_strerror", "ds4a_trace_enable", "ds4a_trace_read",
-    "ds4a_version",
+    "ds4a_version", "ds4a_selftest_wait_timeout",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libds4a.so")
@@ -63,6 +63,7 @@ _SIGS = {
     "ds4a_sparse_attend": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _I, _I64, _P, _P, _P, _SZ, _P]),
     "ds4a_hca_attend": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _I, _I64, _P, _P, _P, _SZ, _P]),
     "ds4a_check": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "ds4a_selftest_wait_timeout": (_I, [_I64, _P, _P]),
     "ds4a_strerror": (ctypes.c_char_p, [_I]),
     "ds4a_trace_enable": (_I, [_I]),
     "ds4a_trace_read": (_I, [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float), _I]),
@@ -201,6 +202,14 @@ def ds4a_check(stream=None) -> tuple[int, int]:
     bits = ctypes.c_uint32(0)
     rc = lib().ds4a_check(_stream(stream), ctypes.byref(bits))
     return rc, bits.value
+
+
+def ds4a_selftest_wait_timeout(limit_cycles: int, status_out, *, stream=None):
+    """One block waits on a barrier nothing arrives at, with a bound of
+    limit_cycles SM cycles; status_out (int32 device tensor) gets 2 when the
+    bound ran out.  ds4a_check then reports DS4A_ETIMEOUT."""
+    rc = lib().ds4a_selftest_wait_timeout(int(limit_cycles), _ptr(status_out), _stream(stream))
+    _ok(rc, "ds4a_selftest_wait_timeout")
 
 
 def ds4a_trace_enable(on: bool = True):

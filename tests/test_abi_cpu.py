@@ -80,6 +80,21 @@ def test_attend_rejects_bad_args(bad):
     assert attend(flash_cfg(), **bad) == L.DS4A_EINVAL
 
 
+def test_flash_shape_needs_the_prepared_query_workspace():
+    # the tensor-core path has no silent CUDA-core fallback: too little
+    # workspace is an error, reported before any launch
+    assert attend(flash_cfg()) == L.DS4A_ENOSPACE
+    assert attend(flash_cfg(), ws=A, wsb=65536 - 16) == L.DS4A_ENOSPACE
+    assert attend(flash_cfg(), B=2, ws=A, wsb=65536) == L.DS4A_ENOSPACE
+
+
+def test_selftest_rejects_bad_limits():
+    lib = L.lib()
+    assert lib.ds4a_selftest_wait_timeout(0, A, None) == L.DS4A_EINVAL
+    assert lib.ds4a_selftest_wait_timeout((1 << 32) + 1, A, None) == L.DS4A_EINVAL
+    assert lib.ds4a_selftest_wait_timeout(1000, None, None) == L.DS4A_EINVAL
+
+
 def test_empty_batches_are_noops():
     assert attend(flash_cfg(), B=0) == L.DS4A_OK
     assert attend(flash_cfg(), T_q=0) == L.DS4A_OK

@@ -244,15 +244,17 @@ def _attend_case(name, cfg_py, B, positions, n_c, sparse, win_cap, use_ws=True, 
     return got, ref
 
 
-@pytest.mark.parametrize("use_ws", [True, False], ids=["split", "nosplit"])
-def test_sparse_attend_flash(use_ws):
+@pytest.mark.parametrize("split", [True, False], ids=["split", "nosplit"])
+def test_sparse_attend_flash(split):
     # positions: inside the first window, exactly W, few entries, many entries
-    _attend_case("sp", FLASH, 2, [0, 5, 127, 300, 3999], 1000, True, 128, use_ws)
+    _attend_case("sp", FLASH, 2, [0, 5, 127, 300, 3999], 1000, True, 128,
+                 ws_bytes=None if split else 2 * 5 * 65536)
 
 
-@pytest.mark.parametrize("use_ws", [True, False], ids=["split", "nosplit"])
-def test_hca_attend_flash(use_ws):
-    _attend_case("hc", HCA, 2, [126, 127, 5119, 6000], 40, False, 128, use_ws)
+@pytest.mark.parametrize("split", [True, False], ids=["split", "nosplit"])
+def test_hca_attend_flash(split):
+    _attend_case("hc", HCA, 2, [126, 127, 5119, 6000], 40, False, 128,
+                 ws_bytes=None if split else 2 * 4 * 65536)
 
 
 def test_attend_tensor_core_without_splits():
@@ -267,10 +269,14 @@ def test_attend_tensor_core_without_splits():
 
 def test_attend_paths_used():
     # Flash shapes with the recommended workspace take the tensor-core
-    # kernels; without a workspace the CUDA-core kernel runs
+    # kernels; without the prepared-query workspace the call is refused
+    # (no silent CUDA-core fallback); other head shapes run on CUDA cores
     names = kernels_used(lambda: _attend_case("path", FLASH, 1, [3999], 1000, True, 128))
     assert names == ["attend_tc", "attend_combine"], names  # decode-sized: q^ inside the kernel
-    names = kernels_used(lambda: _attend_case("path0", FLASH, 1, [3999], 1000, True, 128, use_ws=False))
+    with pytest.raises(L.Ds4aError) as ex:
+        _attend_case("path0", FLASH, 1, [3999], 1000, True, 128, use_ws=False)
+    assert ex.value.code == L.DS4A_ENOSPACE
+    names = kernels_used(lambda: _attend_case("pathtoy", W.TOY_CSA, 1, [63], 32, True, 4, use_ws=False))
     assert names == ["attend_generic"], names
 
 
@@ -280,9 +286,10 @@ def test_attend_many_splits_and_empty_splits():
     names = kernels_used(lambda: _attend_case("many", HCA, 1, [140000], 1100, False, 128))
     assert names == ["attend_tc", "attend_combine"], names
     _attend_case("two", HCA, 1, [130, 140000], 1100, False, 128)
-    # the CUDA-core path with a pool whose sequences are not a whole number
-    # of rows apart
-    _attend_case("gen", FLASH, 2, [0, 5, 127, 300, 3999], 1000, True, 128, use_ws=False, pool_pad=8)
+    # a pool whose sequences are not a whole number of rows apart (gathered
+    # rows; the dense HCA tile loads need whole rows)
+    _attend_case("pad", FLASH, 2, [0, 5, 127, 300, 3999], 1000, True, 128, pool_pad=8)
+    _attend_case("padh", HCA, 2, [5119, 6000], 40, False, 128, pool_pad=8)
 
 
 def test_attend_prefill_sized_launches():
@@ -315,7 +322,8 @@ def test_no_window():
     out = torch.full((1, 1, 64, 512), 7.0, dtype=torch.bfloat16, device="cuda")
     z = torch.zeros(512, dtype=torch.float32, device="cuda")
     idx = torch.full((1, 1, 512), -1, dtype=torch.int32, device="cuda")
-    L.ds4a_sparse_attend(L.layer_cfg(cfg0), i32([[2]]), q, z + 1, None, 0, idx, None, 0, z[:64], out)
+    ws = ws_f32(L.ds4a_attend_workspace(L.layer_cfg(cfg0), 1, 1, 0, True))
+    L.ds4a_sparse_attend(L.layer_cfg(cfg0), i32([[2]]), q, z + 1, None, 0, idx, None, 0, z[:64], out, ws)
     check_ok()
     assert float(out.float().abs().max()) == 0.0
 
@@ -351,14 +359,29 @@ def test_bad_index_sets_error_word():
     idx = torch.arange(512, dtype=torch.int32, device="cuda").reshape(1, 1, 512)
     idx[0, 0, 100] = 5000  # beyond N_c = 2048
     out = torch.empty((1, 1, 64, 512), dtype=torch.bfloat16, device="cuda")
-    L.ds4a_sparse_attend(cfg, i32([[8191]]), q, g, pool, 2048, idx, win, 128, sink, out)
+    ws = ws_f32(L.ds4a_attend_workspace(cfg, 1, 1, 2048, True))
+    L.ds4a_sparse_attend(cfg, i32([[8191]]), q, g, pool, 2048, idx, win, 128, sink, out, ws)
     rc, b = L.ds4a_check()
     assert rc == L.DS4A_EDEVICE and (b & 1)
     assert torch.isfinite(out.float()).all()
     assert L.ds4a_check() == (0, 0)  # cleared
-    L.ds4a_sparse_attend(cfg, i32([[-4]]), q, g, pool, 2048, idx, win, 128, sink, out)
+    L.ds4a_sparse_attend(cfg, i32([[-4]]), q, g, pool, 2048, idx, win, 128, sink, out, ws)
     rc, b = L.ds4a_check()
     assert rc == L.DS4A_EDEVICE and (b & 2)
+
+
+def test_bounded_wait_runs_out_and_reports():
+    # a kernel waits on an mbarrier nothing arrives at, with a ~1 ms bound:
+    # it records the timeout, exits, and the host reads DS4A_ETIMEOUT; the
+    # context stays usable for the next call
+    assert L.ds4a_check() == (0, 0)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.ds4a_selftest_wait_timeout(2_000_000, status)
+    rc, b = L.ds4a_check()
+    assert rc == L.DS4A_ETIMEOUT and (b & 4), (rc, b)
+    assert int(status.item()) == 2
+    assert L.ds4a_check() == (0, 0)  # cleared
+    _attend_case("after_timeout", FLASH, 1, [3999], 1000, True, 128)
 
 
 # ---------------------------------------------------------------------------

@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the ds4a hot path (DeepSeek-V4 hybrid CSA/HCA attention).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workloads 2,3,4,5]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workloads 5,2,3,4]
                     [--impl ours|reference]
 
 One "step" is one pass of the whole path over one batch of the workload:
@@ -39,6 +39,9 @@ if ROOT not in sys.path:
 METRIC = "CSA/HCA attention tokens/s (decode & prefill) at 1 B200; % of HBM/TC roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA datasheet figures for one B200 (dense bf16), reported beside the
+# measured peaks
+DATASHEET_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -502,27 +505,41 @@ def oracle_step_fn(wid: int):
     return fn, len(rows), f"compressor over all 16384 tokens + {len(rows)} of 16384 query rows"
 
 
-def oracle_threads() -> int:
+def host_cores() -> int:
+    """Cores of this host that the process may run on."""
     try:
-        from threadpoolctl import threadpool_info
-        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
-        return int(max(n)) if n else 1
+        return len(os.sched_getaffinity(0))
     except Exception:
-        return 1
+        return os.cpu_count() or 1
 
 
-def time_oracle(wid: int, budget_s: float = 12.0, min_reps: int = 1):
+def time_oracle(wid: int, budget_s: float = 12.0, min_reps: int = 1, threads: int | None = None):
+    """Oracle throughput on the host with its BLAS limited to `threads`
+    (every host core by default); returns (tokens/s, s per pass, sample,
+    threads used)."""
+    from threadpoolctl import threadpool_limits
+
+    n = threads or host_cores()
     fn, tokens, sample = oracle_step_fn(wid)
-    fn()  # warm-up
-    t0 = time.perf_counter()
-    reps = 0
-    while reps < min_reps or time.perf_counter() - t0 < budget_s:
-        fn()
-        reps += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = (time.perf_counter() - t0) / reps
-    return tokens / dt, dt, sample
+    with threadpool_limits(limits=n, user_api="blas"):
+        fn()  # warm-up
+        t0 = time.perf_counter()
+        reps = 0
+        while reps < min_reps or time.perf_counter() - t0 < budget_s:
+            fn()
+            reps += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = (time.perf_counter() - t0) / reps
+    return tokens / dt, dt, sample, n
+
+
+def cpu_baseline_line(wid: int) -> dict:
+    """The oracle on every host core, and on one core, over a bounded sample."""
+    v, dt, sample, n = time_oracle(wid)
+    v1, dt1, _, _ = time_oracle(wid, budget_s=8.0, threads=1)
+    return {"value": v, "unit": UNIT, "cores": n, "kind": "oracle", "sample": sample,
+            "single_core": {"value": v1, "unit": UNIT, "cores": 1}}
 
 
 # ---------------------------------------------------------------------------
@@ -584,8 +601,45 @@ def measure_workload(wid, args, stream, flush, barrier, world, dev, primary):
     return res
 
 
+def step_roofline(res, peaks, peak_src, workload):
+    """The whole step against the roofline: decode moves its algorithmic
+    bytes in one step time (HBM bound); prefill runs its indexer and
+    attention flops, over the step and over those kernels' own time."""
+    work = res["work"]
+    ms = res["ms_per_step"]
+    if "prefill" in workload:
+        flops = work.get("index_score", (0, 0, 0))[1] + work.get("attend", (0, 0, 0))[1]
+        fam_ms = {}
+        for name, k in res["kernels"].items():
+            f = kernel_family(name)
+            fam_ms[f] = fam_ms.get(f, 0.0) + k["avg_ms"] * k["launches_per_step"]
+        # the indexer's top-k and the prepared-query kernel belong to the
+        # indexer + attention work
+        ia_ms = sum(v for f, v in fam_ms.items() if f in ("index_score", "topk", "attend", "qhat_prep",
+                                                          "attend_combine"))
+        ach = flops / (ms / 1e3) / 1e12
+        ach_ia = flops / (ia_ms / 1e3) / 1e12 if ia_ms > 0 else None
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        return {"bound": "tensor", "unit": "TFLOP/s", "what": "indexer + attention flops per step",
+                "algorithmic": flops, "achieved": ach, "frac": ach / peak,
+                "frac_datasheet": ach / DATASHEET_PEAKS["bf16_tflops"],
+                "indexer_attention_kernels": {"ms": ia_ms, "achieved": ach_ia,
+                                              "frac": None if ach_ia is None else ach_ia / peak,
+                                              "frac_datasheet": None if ach_ia is None else
+                                              ach_ia / DATASHEET_PEAKS["bf16_tflops"]},
+                "peak": peak, "peak_source": peak_src, "peak_datasheet": DATASHEET_PEAKS["bf16_tflops"]}
+    nbytes = sum(v[0] for v in work.values())
+    ach = nbytes / (ms / 1e3) / 1e9
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    return {"bound": "hbm", "unit": "GB/s", "what": "algorithmic bytes of the whole step / step time",
+            "algorithmic": nbytes, "achieved": ach, "frac": ach / peak,
+            "frac_datasheet": ach / DATASHEET_PEAKS["hbm_gbs"], "peak": peak, "peak_source": peak_src,
+            "peak_datasheet": DATASHEET_PEAKS["hbm_gbs"]}
+
+
 def roofline_for(res, peaks, peak_src, workload):
-    """Roofline of the kernel with the largest share of the step."""
+    """Roofline of the kernel with the largest share of the step (and the
+    whole step's, under "step")."""
     kinfo = res["kernels"]
     if not kinfo:
         return None
@@ -608,8 +662,10 @@ def roofline_for(res, peaks, peak_src, workload):
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
     r.update({"kernel": top, "traffic": ncu_traffic(top, workload), "peak_source": peak_src,
+              "frac_datasheet": achieved / DATASHEET_PEAKS["bf16_tflops" if r["bound"] == "tensor" else "hbm_gbs"],
               "algorithmic_bytes_per_launch": b_launch, "algorithmic_flops_per_launch": f_launch,
-              "avg_launch_ms": per_launch_ms, "share_of_step": share[top] / max(1e-12, sum(share.values()))})
+              "avg_launch_ms": per_launch_ms, "share_of_step": share[top] / max(1e-12, sum(share.values())),
+              "step": step_roofline(res, peaks, peak_src, workload)})
     return r
 
 
@@ -675,18 +731,21 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
+    from threadpoolctl import threadpool_limits
+
     wid = args.workload_ids[0]
     steps = []
     fn, tokens, sample = oracle_step_fn(wid)
-    for _ in range(args.warmup):
-        fn()
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        fn()
-        steps.append(time.perf_counter() - t0)
+    cores = host_cores()
+    with threadpool_limits(limits=cores, user_api="blas"):
+        for _ in range(args.warmup):
+            fn()
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            fn()
+            steps.append(time.perf_counter() - t0)
     dt = statistics.mean(steps)
     value = tokens / dt
-    cores = oracle_threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -702,7 +761,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workloads", default="2,3,4,5")
+    ap.add_argument("--workloads", default="5,2,3,4")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -754,9 +813,7 @@ def main(argv=None):
     if not args.no_e2e:
         line["e2e"] = measure_e2e(r["state"], args, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, dt, sample = time_oracle(prim)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                                "sample": sample}
+        line["cpu_baseline"] = cpu_baseline_line(prim)
     others = {}
     for wid in wids[1:]:
         rr = results[wid]

@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the ds4a hot path (DeepSeek-V4 hybrid CSA/HCA attention).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workloads 5,2,3,4]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workloads 5,2,3,4,7]
                     [--impl ours|reference]
 
 One "step" is one pass of the whole path over one batch of the workload:
@@ -12,7 +12,12 @@ One "step" is one pass of the whole path over one batch of the workload:
               the window;
   csa_prefill compress every entry (KV and indexer keys), index top-k for all
               16384 queries, sparse attention for all of them;
-  mix_decode  one CSA decode layer and one HCA decode layer.
+  mix_decode  one CSA decode layer and one HCA decode layer;
+  schedule_decode  one decode step through the 43 attention layers of the
+              Flash schedule (two window-only layers, then CSA and HCA
+              alternating).
+Decode layers keep the compressor's cache (ds4a_compress_append): a step
+appends the query token's C/Z rows and compresses the entry it closes.
 The first workload listed is the headline line; the others are reported in
 ``workloads``.  Inputs are seeded synthetic tensors (gen/), resident in HBM.
 Timing: W warm-up steps, then K steps, each bracketed by CUDA events on the
@@ -52,16 +57,33 @@ class Layer:
     """Device tensors and outputs of one attention layer of a workload."""
 
 
-def _csa_decode_layer(w, B, pos, n_c, dev, T):
+def _ring_state(ly, names, cap, dev):
+    """The compressor cache of a decode layer: the streams' rows of the tokens
+    before the query's (positions pos - len + 1 .. pos - 1) in their ring
+    slots (position mod cap), and the query token's own rows as the step's
+    new input ("<name>_new", [B, c])."""
+    import torch
+
+    first = ly.t[names[0]]
+    B, n_rows, c = first.shape
+    state = torch.zeros((B, len(names), cap, c), dtype=torch.bfloat16, device=dev)
+    tb = ly.pos - n_rows + 1
+    for si, nm in enumerate(names):
+        for j in range(n_rows - 1):
+            state[:, si, (tb + j) % cap] = ly.t[nm][:, j]
+        ly.t[nm + "_new"] = ly.t[nm][:, n_rows - 1].contiguous()
+    return state
+
+
+def _csa_decode_layer(w, B, pos, n_c, dev, T, pre=""):
     import torch
     import long_context_hybrid_kv_b200 as L
-    from gen import device as gd
 
     c = w.csa
-    names = [n for n in T if n.startswith("csa.")]
+    key = pre + "csa."
     ly = Layer()
-    ly.kind, ly.cfg_py, ly.cfg = "csa", c, L.layer_cfg(c)
-    ly.t = {n[4:]: T[n] for n in names}
+    ly.kind, ly.cfg_py, ly.cfg, ly.prefix = "csa", c, L.layer_cfg(c), pre
+    ly.t = {n[len(key):]: T[n] for n in T if n.startswith(key)}
     ly.B, ly.pos, ly.n_c, ly.m = B, pos, n_c, c.ratio
     ly.q_pos = torch.full((B, 1), pos, dtype=torch.int32, device=dev)
     ly.idx = torch.empty((B, 1, c.topk), dtype=torch.int32, device=dev)
@@ -71,27 +93,50 @@ def _csa_decode_layer(w, B, pos, n_c, dev, T):
     ly.ws_att = torch.empty(max(1, L.ds4a_attend_workspace(ly.cfg, B, 1, n_c, True) // 4),
                             dtype=torch.float32, device=dev)
     ly.entry = (pos + 1) // c.ratio - 1  # the entry that closes at this token
-    ly.tok_begin = pos - 2 * c.ratio + 1
-    ly.step_inputs = ["q", "qi", "wi", "kv_ca", "kv_cb", "kv_za", "kv_zb", "ix_ca", "ix_cb", "ix_za", "ix_zb"]
+    ly.state_kv = _ring_state(ly, ["kv_ca", "kv_cb", "kv_za", "kv_zb"], 2 * c.ratio, dev)
+    ly.state_ix = _ring_state(ly, ["ix_ca", "ix_cb", "ix_za", "ix_zb"], 2 * c.ratio, dev)
+    ly.step_inputs = ["q", "qi", "wi", "kv_ca_new", "kv_cb_new", "kv_za_new", "kv_zb_new", "ix_ca_new",
+                      "ix_cb_new", "ix_za_new", "ix_zb_new"]
     return ly
 
 
-def _hca_decode_layer(w, B, pos, n_c, dev, T):
+def _hca_decode_layer(w, B, pos, n_c, dev, T, pre=""):
     import torch
     import long_context_hybrid_kv_b200 as L
 
     h = w.hca
+    key = pre + "hca."
     ly = Layer()
-    ly.kind, ly.cfg_py, ly.cfg = "hca", h, L.layer_cfg(h)
-    ly.t = {n[4:]: T[n] for n in T if n.startswith("hca.")}
+    ly.kind, ly.cfg_py, ly.cfg, ly.prefix = "hca", h, L.layer_cfg(h), pre
+    ly.t = {n[len(key):]: T[n] for n in T if n.startswith(key)}
     ly.B, ly.pos, ly.n_c, ly.m = B, pos, n_c, h.ratio
     ly.q_pos = torch.full((B, 1), pos, dtype=torch.int32, device=dev)
     ly.out = torch.empty((B, 1, h.n_heads, h.head_dim), dtype=torch.bfloat16, device=dev)
     ly.ws_att = torch.empty(max(1, L.ds4a_attend_workspace(ly.cfg, B, 1, n_c, False) // 4),
                             dtype=torch.float32, device=dev)
     ly.entry = (pos + 1) // h.ratio - 1
-    ly.tok_begin = pos - h.ratio + 1
-    ly.step_inputs = ["q", "kv_c", "kv_z"]
+    ly.state_kv = _ring_state(ly, ["kv_c", "kv_z"], h.ratio, dev)
+    ly.step_inputs = ["q", "kv_c_new", "kv_z_new"]
+    return ly
+
+
+def _swa_decode_layer(w, B, pos, dev, T, pre):
+    """A sliding-window-only layer: attention over the window alone (the HCA
+    call with no pool entries)."""
+    import torch
+    import long_context_hybrid_kv_b200 as L
+
+    h = w.hca
+    key = pre + "swa."
+    ly = Layer()
+    ly.kind, ly.cfg_py, ly.cfg, ly.prefix = "swa", h, L.layer_cfg(h), pre
+    ly.t = {n[len(key):]: T[n] for n in T if n.startswith(key)}
+    ly.B, ly.pos, ly.n_c, ly.m = B, pos, 0, h.ratio
+    ly.q_pos = torch.full((B, 1), pos, dtype=torch.int32, device=dev)
+    ly.out = torch.empty((B, 1, h.n_heads, h.head_dim), dtype=torch.bfloat16, device=dev)
+    ly.ws_att = torch.empty(max(1, L.ds4a_attend_workspace(ly.cfg, B, 1, 0, False) // 4),
+                            dtype=torch.float32, device=dev)
+    ly.step_inputs = ["q"]
     return ly
 
 
@@ -128,20 +173,22 @@ def _run_layer(ly, stream=None):
     t = ly.t
     S = stream
     if ly.kind == "csa":
-        L.ds4a_compress(ly.cfg, t["kv_ca"], t["kv_za"], t["kv_ba"], t["pool"], cb=t["kv_cb"], zb=t["kv_zb"],
-                        bias_b=t["kv_bb"], norm_g=t["kv_g"], tok_begin=ly.tok_begin,
-                        entry_begin=ly.entry, entry_end=ly.entry + 1, stream=S)
-        L.ds4a_compress(ly.cfg, t["ix_ca"], t["ix_za"], t["ix_ba"], t["ki"], cb=t["ix_cb"], zb=t["ix_zb"],
-                        bias_b=t["ix_bb"], tok_begin=ly.tok_begin, entry_begin=ly.entry,
-                        entry_end=ly.entry + 1, stream=S)
+        pos = ly.q_pos.view(-1)
+        L.ds4a_compress_append(ly.cfg, pos, t["kv_ca_new"], t["kv_za_new"], t["kv_ba"], ly.state_kv, t["pool"],
+                               cb=t["kv_cb_new"], zb=t["kv_zb_new"], bias_b=t["kv_bb"], norm_g=t["kv_g"], stream=S)
+        L.ds4a_compress_append(ly.cfg, pos, t["ix_ca_new"], t["ix_za_new"], t["ix_ba"], ly.state_ix, t["ki"],
+                               cb=t["ix_cb_new"], zb=t["ix_zb_new"], bias_b=t["ix_bb"], stream=S)
         L.ds4a_index_topk(ly.cfg, ly.q_pos, t["qi"], t["wi"], t["ki"], ly.n_c, ly.idx, ly.ws_index, stream=S)
         L.ds4a_sparse_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], t["pool"], ly.n_c, ly.idx, t["win"],
                              t["win"].shape[1], t["sink"], ly.out, ly.ws_att, stream=S)
     elif ly.kind == "hca":
-        L.ds4a_compress(ly.cfg, t["kv_c"], t["kv_z"], t["kv_b"], t["pool"], norm_g=t["kv_g"],
-                        tok_begin=ly.tok_begin, entry_begin=ly.entry, entry_end=ly.entry + 1, stream=S)
+        L.ds4a_compress_append(ly.cfg, ly.q_pos.view(-1), t["kv_c_new"], t["kv_z_new"], t["kv_b"], ly.state_kv,
+                               t["pool"], norm_g=t["kv_g"], stream=S)
         L.ds4a_hca_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], t["pool"], ly.n_c, t["win"],
                           t["win"].shape[1], t["sink"], ly.out, ly.ws_att, stream=S)
+    elif ly.kind == "swa":
+        L.ds4a_hca_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], None, 0, t["win"], t["win"].shape[1],
+                          t["sink"], ly.out, ly.ws_att, stream=S)
     else:  # prefill
         L.ds4a_compress(ly.cfg, t["kv_ca"], t["kv_za"], t["kv_ba"], ly.pool, cb=t["kv_cb"], zb=t["kv_zb"],
                         bias_b=t["kv_bb"], norm_g=t["kv_g"], entry_begin=0, entry_end=ly.n_c, stream=S)
@@ -182,6 +229,14 @@ class State:
                 self.layers.append(_hca_decode_layer(w, w.B, w.pos, w.n_hca, dev, T))
             if w.kind == "csa_prefill":
                 self.layers.append(_csa_prefill_layer(w, dev, T))
+            if w.kind == "schedule_decode":
+                for pre, kind in W.schedule_layers(w):
+                    if kind == "csa":
+                        self.layers.append(_csa_decode_layer(w, w.B, w.pos, w.n_csa, dev, T, pre))
+                    elif kind == "hca":
+                        self.layers.append(_hca_decode_layer(w, w.B, w.pos, w.n_hca, dev, T, pre))
+                    else:
+                        self.layers.append(_swa_decode_layer(w, w.B, w.pos, dev, T, pre))
             self.tokens = w.B if w.kind != "csa_prefill" else w.pos + 1
         self.tensors = T
 
@@ -217,6 +272,11 @@ def kernel_work(state) -> dict:
 
     for ly in state.layers:
         c = ly.cfg_py
+        if ly.kind == "swa":
+            B, pos, D, H = ly.B, ly.pos, c.head_dim, c.n_heads
+            n_win = pos - max(0, pos - c.window + 1) + 1
+            add("attend", B * (n_win * D * 2 + 2 * H * D * 2 + H * 4 + D * 4), 4.0 * B * n_win * H * D)
+            continue
         if ly.kind in ("csa", "hca"):
             B, pos, n_c, m = ly.B, ly.pos, ly.n_c, ly.m
             n_vis = min((pos + 1) // m, n_c)
@@ -761,7 +821,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workloads", default="5,2,3,4")
+    ap.add_argument("--workloads", default="5,2,3,4,7")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -53,17 +53,35 @@ class Spec:
 class Workload:
     wid: int
     name: str
-    kind: str  # "toy" | "csa_decode" | "hca_decode" | "csa_prefill" | "mix_decode"
+    kind: str  # "toy" | "csa_decode" | "hca_decode" | "csa_prefill" | "mix_decode" | "schedule_decode"
     B: int
     pos: int  # decode: position of the query token; prefill: T - 1
     csa: LayerCfg | None
     hca: LayerCfg | None
     n_csa: int  # compressed entries in the CSA pool
     n_hca: int
+    n_layers: int = 0  # schedule_decode: layers of the Flash schedule
 
     @property
     def seed(self) -> int:
         return 20260000 + self.wid
+
+
+def layer_ratio(layer: int) -> int:
+    """Compression ratio of a Flash layer ("Phase 1 Module 1", section on the
+    per-layer pattern; "DeepSeek V4 Inside", compress_ratios of the config):
+    layers 0 and 1 keep only the sliding window (0), then even layers are
+    CSA (4) and odd layers HCA (128)."""
+    if layer < 2:
+        return 0
+    return 4 if layer % 2 == 0 else 128
+
+
+def schedule_layers(w: Workload) -> list[tuple[str, str]]:
+    """(tensor-name prefix, kind) of every layer of a schedule workload, kind
+    in "swa" | "csa" | "hca"."""
+    kinds = {0: "swa", 4: "csa", 128: "hca"}
+    return [(f"L{l:02d}.", kinds[layer_ratio(l)]) for l in range(w.n_layers)]
 
 
 FLASH_CSA = LayerCfg(n_heads=64, head_dim=512, rope_dim=64, window=128,
@@ -82,11 +100,58 @@ WORKLOADS = {
     5: Workload(5, "mix_decode_b8_ctx1m", "mix_decode", 8, 1048575, FLASH_CSA, FLASH_HCA, 262144, 8192),
     # a 4096-token prefill, small enough for multi-pass profiler captures
     6: Workload(6, "csa_prefill_b1_t4k", "csa_prefill", 1, 4095, FLASH_CSA, None, 1024, 0),
+    # one decode step through the 43 attention layers of the Flash schedule
+    7: Workload(7, "schedule43_decode_b8_ctx128k", "schedule_decode", 8, 131071, FLASH_CSA, FLASH_HCA,
+                32768, 1024, n_layers=43),
+    # the same schedule at a size the oracle checks layer by layer quickly
+    8: Workload(8, "schedule43_decode_b2_ctx16k", "schedule_decode", 2, 16383, FLASH_CSA, FLASH_HCA,
+                4096, 128, n_layers=43),
 }
 
 
 def _gain(shape):
     return Spec(shape, "f32", 0.1, 1.0)
+
+
+def _csa_decode_specs(s: dict, pre: str, B: int, c: LayerCfg, n_csa: int):
+    m = c.ratio
+    s[pre + "csa.q"] = Spec((B, 1, c.n_heads, c.head_dim), "bf16")
+    s[pre + "csa.q_norm_g"] = _gain((c.head_dim,))
+    s[pre + "csa.sink"] = Spec((c.n_heads,), "f32")
+    s[pre + "csa.qi"] = Spec((B, 1, c.idx_heads, c.idx_dim), "bf16")
+    s[pre + "csa.wi"] = Spec((B, 1, c.idx_heads), "bf16")
+    s[pre + "csa.ki"] = Spec((B, n_csa, c.idx_dim), "bf16")
+    s[pre + "csa.pool"] = Spec((B, n_csa, c.head_dim), "bf16")
+    s[pre + "csa.win"] = Spec((B, c.window, c.head_dim), "bf16")
+    # compressor streams of the 2m newest tokens (the entry that closes now)
+    for st in ("ca", "cb", "za", "zb"):
+        s[pre + f"csa.kv_{st}"] = Spec((B, 2 * m, c.head_dim), "bf16")
+        s[pre + f"csa.ix_{st}"] = Spec((B, 2 * m, c.idx_dim), "bf16")
+    s[pre + "csa.kv_ba"] = Spec((m, c.head_dim), "f32", 1.0 / math.sqrt(m))
+    s[pre + "csa.kv_bb"] = Spec((m, c.head_dim), "f32", 1.0 / math.sqrt(m))
+    s[pre + "csa.ix_ba"] = Spec((m, c.idx_dim), "f32", 1.0 / math.sqrt(m))
+    s[pre + "csa.ix_bb"] = Spec((m, c.idx_dim), "f32", 1.0 / math.sqrt(m))
+    s[pre + "csa.kv_g"] = _gain((c.head_dim,))
+
+
+def _hca_decode_specs(s: dict, pre: str, B: int, h: LayerCfg, n_hca: int):
+    m = h.ratio
+    s[pre + "hca.q"] = Spec((B, 1, h.n_heads, h.head_dim), "bf16")
+    s[pre + "hca.q_norm_g"] = _gain((h.head_dim,))
+    s[pre + "hca.sink"] = Spec((h.n_heads,), "f32")
+    s[pre + "hca.pool"] = Spec((B, n_hca, h.head_dim), "bf16")
+    s[pre + "hca.win"] = Spec((B, h.window, h.head_dim), "bf16")
+    s[pre + "hca.kv_c"] = Spec((B, m, h.head_dim), "bf16")
+    s[pre + "hca.kv_z"] = Spec((B, m, h.head_dim), "bf16")
+    s[pre + "hca.kv_b"] = Spec((m, h.head_dim), "f32", 1.0 / math.sqrt(m))
+    s[pre + "hca.kv_g"] = _gain((h.head_dim,))
+
+
+def _swa_decode_specs(s: dict, pre: str, B: int, h: LayerCfg):
+    s[pre + "swa.q"] = Spec((B, 1, h.n_heads, h.head_dim), "bf16")
+    s[pre + "swa.q_norm_g"] = _gain((h.head_dim,))
+    s[pre + "swa.sink"] = Spec((h.n_heads,), "f32")
+    s[pre + "swa.win"] = Spec((B, h.window, h.head_dim), "bf16")
 
 
 def specs(w: Workload) -> dict[str, Spec]:
@@ -95,37 +160,17 @@ def specs(w: Workload) -> dict[str, Spec]:
     s: dict[str, Spec] = {}
     B = w.B
     if w.kind in ("csa_decode", "mix_decode"):
-        c = w.csa
-        m = c.ratio
-        s["csa.q"] = Spec((B, 1, c.n_heads, c.head_dim), "bf16")
-        s["csa.q_norm_g"] = _gain((c.head_dim,))
-        s["csa.sink"] = Spec((c.n_heads,), "f32")
-        s["csa.qi"] = Spec((B, 1, c.idx_heads, c.idx_dim), "bf16")
-        s["csa.wi"] = Spec((B, 1, c.idx_heads), "bf16")
-        s["csa.ki"] = Spec((B, w.n_csa, c.idx_dim), "bf16")
-        s["csa.pool"] = Spec((B, w.n_csa, c.head_dim), "bf16")
-        s["csa.win"] = Spec((B, c.window, c.head_dim), "bf16")
-        # compressor streams of the 2m newest tokens (the entry that closes now)
-        for st in ("ca", "cb", "za", "zb"):
-            s[f"csa.kv_{st}"] = Spec((B, 2 * m, c.head_dim), "bf16")
-            s[f"csa.ix_{st}"] = Spec((B, 2 * m, c.idx_dim), "bf16")
-        s["csa.kv_ba"] = Spec((m, c.head_dim), "f32", 1.0 / math.sqrt(m))
-        s["csa.kv_bb"] = Spec((m, c.head_dim), "f32", 1.0 / math.sqrt(m))
-        s["csa.ix_ba"] = Spec((m, c.idx_dim), "f32", 1.0 / math.sqrt(m))
-        s["csa.ix_bb"] = Spec((m, c.idx_dim), "f32", 1.0 / math.sqrt(m))
-        s["csa.kv_g"] = _gain((c.head_dim,))
+        _csa_decode_specs(s, "", B, w.csa, w.n_csa)
     if w.kind in ("hca_decode", "mix_decode"):
-        h = w.hca
-        m = h.ratio
-        s["hca.q"] = Spec((B, 1, h.n_heads, h.head_dim), "bf16")
-        s["hca.q_norm_g"] = _gain((h.head_dim,))
-        s["hca.sink"] = Spec((h.n_heads,), "f32")
-        s["hca.pool"] = Spec((B, w.n_hca, h.head_dim), "bf16")
-        s["hca.win"] = Spec((B, h.window, h.head_dim), "bf16")
-        s["hca.kv_c"] = Spec((B, m, h.head_dim), "bf16")
-        s["hca.kv_z"] = Spec((B, m, h.head_dim), "bf16")
-        s["hca.kv_b"] = Spec((m, h.head_dim), "f32", 1.0 / math.sqrt(m))
-        s["hca.kv_g"] = _gain((h.head_dim,))
+        _hca_decode_specs(s, "", B, w.hca, w.n_hca)
+    if w.kind == "schedule_decode":
+        for pre, kind in schedule_layers(w):
+            if kind == "csa":
+                _csa_decode_specs(s, pre, B, w.csa, w.n_csa)
+            elif kind == "hca":
+                _hca_decode_specs(s, pre, B, w.hca, w.n_hca)
+            else:
+                _swa_decode_specs(s, pre, B, w.hca)
     if w.kind == "csa_prefill":
         c = w.csa
         m = c.ratio

@@ -130,6 +130,48 @@ int ds4a_compress(const ds4a_layer_cfg* cfg, int B, int T_tok, int tok_begin, in
                   const float* norm_g, int entry_begin, int entry_end, ds4a_bf16* pool,
                   int64_t pool_bstride, ds4a_stream stream);
 
+/* Bytes of the per-layer compressor state ds4a_compress_append keeps for B
+ * sequences of width c: overlap != 0 (CSA, two streams) holds 4 streams
+ * (C^a, C^b, Z^a, Z^b) x 2m token rows; overlap == 0 (HCA) 2 streams (C, Z)
+ * x m rows; bf16 each. */
+size_t ds4a_compress_state_bytes(const ds4a_layer_cfg* cfg, int B, int c, int overlap);
+
+/*
+ * ds4a_compress_append -- the compressor's decode-time cache ([hf-doc] cache
+ * layers: the CSA / HCA compressors keep a buffer of raw rows, a count and,
+ * for CSA, the overlap state between calls; the entries are those of
+ * ds4a_compress, [beyond] 3.2.2 eqs. 9-12 and 3.3 eqs. 20-23).
+ *
+ * One call per decoded token.  Sequence b's new token at position pos[b]
+ * brings its rows ca[b], za[b] (and cb[b], zb[b] for CSA); they are stored in
+ * the sequence's state at slot pos[b] mod 2m (CSA) or mod m (HCA).  When the
+ * token closes entry i = (pos[b] + 1) / m - 1 (that is, (pos[b] + 1) mod m
+ * == 0), the entry is compressed from the state exactly as ds4a_compress
+ * computes it from the full streams and written to pool[b][i]; otherwise
+ * nothing else happens.  Sequences may sit at different positions.
+ *
+ *   pos       device int32 [B]; every sequence must append its tokens in
+ *             order, one per call (the state holds only the last 2m or m
+ *             tokens; rows of tokens never appended read as whatever the
+ *             state held -- zero it to start a sequence at position 0)
+ *   ca .. zb  device bf16 [B, c]: the new token's rows (cb == NULL: HCA)
+ *   bias_a/b, norm_g   as ds4a_compress
+ *   state     device bf16, ds4a_compress_state_bytes(cfg, B, c, cb != NULL)
+ *             bytes, caller-owned, layout [B][stream][slot][c]
+ *   N_cap     pool capacity in entries; an entry index >= N_cap is skipped
+ *             and recorded as DS4A_DEV_BAD_INDEX, a negative position as
+ *             DS4A_DEV_BAD_POS
+ *   pool      device bf16, entry i of sequence b at pool + b * pool_bstride
+ *             + i * c
+ * The state is read after the preceding library kernels finish (it is a
+ * library output), so calls chain on one stream without host syncs.
+ */
+int ds4a_compress_append(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
+                         const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                         const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                         const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
+                         int64_t pool_bstride, ds4a_stream stream);
+
 /* Bytes of workspace ds4a_index_topk needs for these sizes. */
 size_t ds4a_index_topk_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c);
 

@@ -153,6 +153,53 @@ int ds4a_compress(const ds4a_layer_cfg* cfg, int B, int T_tok, int tok_begin, in
   a.bias_a = bias_a; a.bias_b = bias_b; a.norm_g = norm_g;
   a.entry_begin = entry_begin; a.entry_end = entry_end;
   a.pool = pool; a.pool_bstride = pool_bstride;
+  a.app_pos = nullptr; a.ring = nullptr; a.ring_cap = 0; a.n_cap = 0;
+  fill_rope_theta(&a.rope, a.rope_dim, cfg->rope_base);
+  a.err = err_word();
+  if (!a.err) return DS4A_ECUDA;
+  return cuda_rc(launch_compress(a, (cudaStream_t)stream));
+}
+
+size_t ds4a_compress_state_bytes(const ds4a_layer_cfg* cfg, int B, int c, int overlap) {
+  if (!cfg || cfg->ratio < 1 || B <= 0 || c <= 0) return 0;
+  const size_t S = overlap ? 4 : 2, cap = overlap ? 2 * (size_t)cfg->ratio : (size_t)cfg->ratio;
+  return (size_t)B * S * cap * (size_t)c * sizeof(uint16_t);
+}
+
+int ds4a_compress_append(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
+                         const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                         const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                         const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
+                         int64_t pool_bstride, ds4a_stream stream) {
+  if (!cfg || cfg->ratio < 1) return DS4A_EINVAL;
+  if (B < 0 || N_cap < 0 || c < 2 || c > 1024 || (c % 2) != 0) return DS4A_EINVAL;
+  if ((c % 8) != 0 && c > 512) return DS4A_EINVAL;
+  if (B == 0) return DS4A_OK;
+  if (!pos || !ca || !za || !bias_a || !state || !pool) return DS4A_EINVAL;
+  const bool overlap = cb != nullptr;
+  if (overlap && (!zb || !bias_b)) return DS4A_EINVAL;
+  if (!overlap && (zb || bias_b)) return DS4A_EINVAL;
+  if (!aligned16(pos) || !aligned16(ca) || !aligned16(za) || !aligned16(bias_a) || !aligned16(state) ||
+      !aligned16(pool))
+    return DS4A_EINVAL;
+  if (overlap && (!aligned16(cb) || !aligned16(zb) || !aligned16(bias_b))) return DS4A_EINVAL;
+  if (norm_g) {
+    if (check_cfg(cfg) != DS4A_OK) return DS4A_EINVAL;
+    if (cfg->rope_dim > c) return DS4A_EINVAL;
+  }
+  if (pool_bstride < (int64_t)N_cap * c || (pool_bstride % 2) != 0) return DS4A_EINVAL;
+  const int m = cfg->ratio;
+  if ((int64_t)(overlap ? 2 * m : m) * c > (int64_t)1 << 24) return DS4A_EINVAL;
+
+  CompressArgs a;
+  a.B = B; a.T_tok = 1; a.tok_begin = 0; a.c = c; a.m = m;
+  a.rope_dim = norm_g ? cfg->rope_dim : 0;
+  a.rope_base = cfg->rope_base; a.eps = cfg->rms_eps;
+  a.ca = ca; a.cb = cb; a.za = za; a.zb = zb;
+  a.bias_a = bias_a; a.bias_b = bias_b; a.norm_g = norm_g;
+  a.entry_begin = 0; a.entry_end = 1;
+  a.pool = pool; a.pool_bstride = pool_bstride;
+  a.app_pos = pos; a.ring = state; a.ring_cap = overlap ? 2 * m : m; a.n_cap = N_cap;
   fill_rope_theta(&a.rope, a.rope_dim, cfg->rope_base);
   a.err = err_word();
   if (!a.err) return DS4A_ECUDA;

@@ -59,6 +59,56 @@ struct VecLoad<2> {  // 2 bf16 = 4 bytes
   }
 };
 
+// Row of one stream (C or Z of half a or b) for token tok of sequence b:
+// the caller's streams in range mode; in append mode the new token's input
+// row or the ring slot of an earlier token.
+__device__ __forceinline__ const uint16_t* term_row(const CompressArgs& a, bool half_a, bool is_z, int b,
+                                                    int tok, int newtok) {
+  const uint16_t* src = half_a ? (is_z ? a.za : a.ca) : (is_z ? a.zb : a.cb);
+  if (a.app_pos == nullptr) return src + ((int64_t)b * a.T_tok + (tok - a.tok_begin)) * a.c;
+  if (tok == newtok) return src + (int64_t)b * a.c;
+  const bool overlap = a.cb != nullptr;
+  const int S = overlap ? 4 : 2;
+  const int st = overlap ? (is_z ? 2 : 0) + (half_a ? 0 : 1) : (is_z ? 1 : 0);
+  return a.ring + (((int64_t)b * S + st) * a.ring_cap + (tok % a.ring_cap)) * a.c;
+}
+
+// Append mode: store the new token's rows of every stream in its ring slot
+// (threads tid0, tid0 + nthr, ... of the block; 16-byte pieces when c is a
+// multiple of 8).  Returns the entry the token closes, or -1.
+__device__ __forceinline__ int append_token(const CompressArgs& a, int b, int tid0, int nthr, int* newtok) {
+  const int p = a.app_pos[b];
+  *newtok = p;
+  if (p < 0) {
+    if (tid0 == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
+    return -1;
+  }
+  const bool overlap = a.cb != nullptr;
+  const int S = overlap ? 4 : 2;
+  const uint16_t* srcs[4] = {a.ca, overlap ? a.cb : a.za, a.za, a.zb};
+  const int slot = p % a.ring_cap;
+  if (a.c % 8 == 0) {
+    const int pieces = a.c / 8;
+    for (int k = tid0; k < S * pieces; k += nthr) {
+      const int st = k / pieces, q = k % pieces;
+      const uint4 v = reinterpret_cast<const uint4*>(srcs[st] + (int64_t)b * a.c)[q];
+      reinterpret_cast<uint4*>(a.ring + (((int64_t)b * S + st) * a.ring_cap + slot) * a.c)[q] = v;
+    }
+  } else {
+    for (int k = tid0; k < S * a.c; k += nthr) {
+      const int st = k / a.c, q = k % a.c;
+      a.ring[(((int64_t)b * S + st) * a.ring_cap + slot) * a.c + q] = srcs[st][(int64_t)b * a.c + q];
+    }
+  }
+  if ((p + 1) % a.m != 0) return -1;
+  const int i = (p + 1) / a.m - 1;
+  if (i >= a.n_cap) {
+    if (tid0 == 0) raise_err(a.err, DS4A_DEV_BAD_INDEX);
+    return -1;
+  }
+  return i;
+}
+
 template <int V>
 __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs a) {
   extern __shared__ float csm[];
@@ -68,15 +118,21 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
   const int tid = threadIdx.x;
   const int cc = tid % NC;
   const int g = tid / NC;
-  const int i = a.entry_begin + blockIdx.x;
   const int b = blockIdx.y;
   const bool overlap = a.cb != nullptr;
-  const int n_terms = (overlap && i >= 1) ? 2 * m : m;
   pdl_trigger();
   // The C/Z rows, gate biases and norm weights are inputs that no kernel of
   // the chain writes: the pooling runs while the preceding kernel finishes,
   // and only the pool write waits for it (a preceding kernel may still read
-  // the entry this one overwrites).
+  // the entry this one overwrites).  In append mode the ring was written by
+  // an earlier call, so everything waits.
+  int i = a.entry_begin + blockIdx.x, newtok = -1;
+  if (a.app_pos != nullptr) {
+    pdl_wait();
+    i = append_token(a, b, tid, kCompressThreads, &newtok);
+    if (i < 0) return;
+  }
+  const int n_terms = (overlap && i >= 1) ? 2 * m : m;
 
   float mx[V], l[V], acc[V];
 #pragma unroll
@@ -92,9 +148,8 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
           const bool half_a = term < m;
           const int r = half_a ? term : term - m;
           const int tok = half_a ? i * m + r : (i - 1) * m + r;
-          const int64_t row = (int64_t)b * a.T_tok + (tok - a.tok_begin);
-          VecLoad<V>::load((half_a ? a.ca : a.cb) + row * c + cc * V, vals[u]);
-          VecLoad<V>::load((half_a ? a.za : a.zb) + row * c + cc * V, zs[u]);
+          VecLoad<V>::load(term_row(a, half_a, false, b, tok, newtok) + cc * V, vals[u]);
+          VecLoad<V>::load(term_row(a, half_a, true, b, tok, newtok) + cc * V, zs[u]);
           VecLoad<V>::load_f((half_a ? a.bias_a : a.bias_b) + (int64_t)r * c + cc * V, bs[u]);
         }
       }
@@ -202,13 +257,26 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
   const int cc = tid % NC;
   const int g = tid / NC;
   const int zr = (int)cl.block_rank();
-  const int i = a.entry_begin + blockIdx.x / Z;
   const int b = blockIdx.y;
   const bool overlap = a.cb != nullptr;
+  pdl_trigger();
+  // as in compress_kernel, only the pool write waits for the preceding
+  // kernel, except in append mode (the ring comes from an earlier call).
+  // Every block of a cluster serves the same sequence, so all of them take
+  // the same early exit.
+  int i = a.entry_begin + blockIdx.x / Z, newtok = -1;
+  if (a.app_pos != nullptr) {
+    pdl_wait();
+    i = zr == 0 ? append_token(a, b, tid, kCompressThreads, &newtok) : -2;
+    if (zr != 0) {
+      const int p = a.app_pos[b];
+      newtok = p;
+      i = (p >= 0 && (p + 1) % m == 0 && (p + 1) / m - 1 < a.n_cap) ? (p + 1) / m - 1 : -1;
+    }
+    if (i < 0) return;
+  }
   const int n_terms = (overlap && i >= 1) ? 2 * m : m;
   const int tz0 = (int)((int64_t)zr * n_terms / Z), tz1 = (int)((int64_t)(zr + 1) * n_terms / Z);
-  pdl_trigger();
-  // as in compress_kernel, only the pool write waits for the preceding kernel
 
   float mx[V], l[V], acc[V];
 #pragma unroll
@@ -223,9 +291,8 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
           const bool half_a = term < m;
           const int r = half_a ? term : term - m;
           const int tok = half_a ? i * m + r : (i - 1) * m + r;
-          const int64_t row = (int64_t)b * a.T_tok + (tok - a.tok_begin);
-          VecLoad<V>::load((half_a ? a.ca : a.cb) + row * c + cc * V, vals[u]);
-          VecLoad<V>::load((half_a ? a.za : a.zb) + row * c + cc * V, zs[u]);
+          VecLoad<V>::load(term_row(a, half_a, false, b, tok, newtok) + cc * V, vals[u]);
+          VecLoad<V>::load(term_row(a, half_a, true, b, tok, newtok) + cc * V, zs[u]);
           VecLoad<V>::load_f((half_a ? a.bias_a : a.bias_b) + (int64_t)r * c + cc * V, bs[u]);
         }
       }
@@ -343,7 +410,8 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
 }
 
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
-  const int n = a.entry_end - a.entry_begin;
+  // append mode: one (possible) entry per sequence
+  const int n = a.app_pos != nullptr ? 1 : a.entry_end - a.entry_begin;
   if (n <= 0 || a.B <= 0) return cudaSuccess;
   const int V = (a.c % 8 == 0) ? 8 : 2;
   const int NC = a.c / V;

@@ -221,6 +221,14 @@ struct CompressArgs {
   uint16_t* pool;
   int64_t pool_bstride;
   unsigned int* err;
+  // append mode (app_pos != nullptr): ca..zb are the new token's rows
+  // [B, c]; the earlier tokens come from the ring state [B][S][ring_cap][c]
+  // (S = 4 streams ca, cb, za, zb for CSA, 2 streams ca, za for HCA; slot =
+  // position mod ring_cap); each sequence's entry is the one its token
+  // closes, if any, and must be below n_cap
+  const int32_t* app_pos;
+  uint16_t* ring;
+  int ring_cap, n_cap;
   RopeTheta rope;
 };
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);

@@ -14,7 +14,7 @@ import os
 __all__ = [
     "DS4A_OK", "DS4A_EINVAL", "DS4A_EUNSUPPORTED", "DS4A_ECUDA", "DS4A_EDEVICE", "DS4A_ETIMEOUT",
     "DS4A_ENOSPACE", "Ds4aError", "LayerCfg", "layer_cfg", "lib", "LIB_PATH", "ds4a_compress",
-    "ds4a_index_topk_workspace", "ds4a_index_topk", "ds4a_index_topk_noalloc", "ds4a_attend_workspace", "ds4a_sparse_attend",
+    "ds4a_compress_state_bytes", "ds4a_compress_append", "ds4a_index_topk_workspace", "ds4a_index_topk", "ds4a_index_topk_noalloc", "ds4a_attend_workspace", "ds4a_sparse_attend",
     "ds4a_hca_attend", "ds4a_check", "ds4a_strerror", "ds4a_trace_enable", "ds4a_trace_read",
     "ds4a_version", "ds4a_selftest_wait_timeout",
 ]
@@ -56,6 +56,8 @@ _CFG = ctypes.POINTER(LayerCfg)
 
 _SIGS = {
     "ds4a_compress": (_I, [_CFG, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I64, _P]),
+    "ds4a_compress_state_bytes": (_SZ, [_CFG, _I, _I, _I]),
+    "ds4a_compress_append": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _I64, _P]),
     "ds4a_index_topk_workspace": (_SZ, [_CFG, _I, _I, _I]),
     "ds4a_index_topk": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
     "ds4a_index_topk_noalloc": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _P]),
@@ -137,6 +139,22 @@ def ds4a_compress(cfg: LayerCfg, ca, za, bias_a, pool, *, entry_begin: int, entr
                              _ptr(zb), _ptr(bias_a), _ptr(bias_b), _ptr(norm_g), entry_begin,
                              entry_end, _ptr(pool), pool.stride(0), _stream(stream))
     _ok(rc, "ds4a_compress")
+
+
+def ds4a_compress_state_bytes(cfg: LayerCfg, B: int, c: int, overlap: bool) -> int:
+    return lib().ds4a_compress_state_bytes(ctypes.byref(cfg), B, c, int(bool(overlap)))
+
+
+def ds4a_compress_append(cfg: LayerCfg, pos, ca, za, bias_a, state, pool, *, cb=None, zb=None, bias_b=None,
+                         norm_g=None, stream=None):
+    """New token rows ca/za (cb/zb) [B, c] at positions pos [B] into the
+    ring state; entries that close go to pool [B, N_cap, c]."""
+    _bf16(ca, "ca"), _bf16(za, "za"), _bf16(cb, "cb"), _bf16(zb, "zb")
+    B, c = ca.shape
+    rc = lib().ds4a_compress_append(ctypes.byref(cfg), B, c, _ptr(pos), _ptr(ca), _ptr(cb), _ptr(za), _ptr(zb),
+                                    _ptr(bias_a), _ptr(bias_b), _ptr(norm_g), _ptr(state), pool.shape[1],
+                                    _ptr(pool), pool.stride(0), _stream(stream))
+    _ok(rc, "ds4a_compress_append")
 
 
 def ds4a_index_topk_workspace(cfg: LayerCfg, B: int, T_q: int, N_c: int) -> int:

@@ -143,6 +143,31 @@ def test_compress_rejects_bad_args():
     assert call(e0=4, e1=4) == L.DS4A_OK        # nothing to do
 
 
+def test_compress_append_rejects_bad_args():
+    lib = L.lib()
+    cfg = flash_cfg()
+
+    def call(**kw):
+        a = dict(B=2, c=512, pos=A, ca=A, cb=A, za=A, zb=A, ba=A, bb=A, g=A, st=A, cap=2048, pool=A,
+                 pbs=2048 * 512)
+        a.update(kw)
+        return lib.ds4a_compress_append(ctypes.byref(cfg), a["B"], a["c"], a["pos"], a["ca"], a["cb"], a["za"],
+                                        a["zb"], a["ba"], a["bb"], a["g"], a["st"], a["cap"], a["pool"], a["pbs"],
+                                        None)
+
+    assert call(B=0) == L.DS4A_OK
+    assert call(c=13) == L.DS4A_EINVAL
+    assert call(pos=None) == L.DS4A_EINVAL
+    assert call(st=None) == L.DS4A_EINVAL
+    assert call(st=MIS) == L.DS4A_EINVAL
+    assert call(cb=None) == L.DS4A_EINVAL      # zb / bias_b without cb
+    assert call(pbs=100) == L.DS4A_EINVAL
+    assert call(cap=-1) == L.DS4A_EINVAL
+    assert L.ds4a_compress_state_bytes(cfg, 8, 512, True) == 8 * 4 * 8 * 512 * 2
+    hca = flash_cfg(ratio=128)
+    assert L.ds4a_compress_state_bytes(hca, 8, 512, False) == 8 * 2 * 128 * 512 * 2
+
+
 def test_workspace_queries():
     cfg = flash_cfg()
     assert L.ds4a_index_topk_workspace(cfg, 8, 1, 262144) == 8 * 262144 * 4

@@ -401,21 +401,22 @@ def _decode_csa_ref(w, ly, bsel):
     n_c, pos, m = w.n_csa, w.pos, c.ratio
     e = n_c - 1
     tb = pos - 2 * m + 1
-    H = {n: W.host_tensor(w, f"csa.{n}") for n in ("kv_ca", "kv_cb", "kv_za", "kv_zb", "ix_ca", "ix_cb",
-                                                  "ix_za", "ix_zb", "kv_ba", "kv_bb", "ix_ba", "ix_bb",
-                                                  "kv_g", "q", "qi", "wi", "q_norm_g", "sink", "win")}
+    pre = ly.prefix + "csa."
+    H = {n: W.host_tensor(w, pre + n) for n in ("kv_ca", "kv_cb", "kv_za", "kv_zb", "ix_ca", "ix_cb",
+                                               "ix_za", "ix_zb", "kv_ba", "kv_bb", "ix_ba", "ix_bb",
+                                               "kv_g", "q", "qi", "wi", "q_norm_g", "sink", "win")}
     res = {}
     for b in bsel:
         ent = O.compress(m, e, e + 1, tb, H["kv_ca"][b], H["kv_za"][b], H["kv_ba"], H["kv_cb"][b],
                          H["kv_zb"][b], H["kv_bb"], H["kv_g"], c.rope_dim)[0]
         kent = O.compress(m, e, e + 1, tb, H["ix_ca"][b], H["ix_za"][b], H["ix_ba"], H["ix_cb"][b],
                           H["ix_zb"][b], H["ix_bb"])[0]
-        ki = W.host_rows(w, "csa.ki", b * n_c + np.arange(n_c))
+        ki = W.host_rows(w, pre + "ki", b * n_c + np.arange(n_c))
         ki[e] = O.store_bf16(kent)
         idx, scores = O.index_topk(H["qi"][b, 0], H["wi"][b, 0], ki, pos, m, c.topk, n_c)
         sel = idx[idx >= 0]
         pool = np.zeros((n_c, c.head_dim), np.uint16)
-        pool[sel] = W.host_rows(w, "csa.pool", b * n_c + sel)
+        pool[sel] = W.host_rows(w, pre + "pool", b * n_c + sel)
         pool[e] = O.store_bf16(ent)
         out = O.csa_attend(H["q"][b, 0], H["q_norm_g"], pool, idx, H["win"][b], c.window, H["sink"], pos, c)
         res[b] = (ent, kent, idx, scores, out)
@@ -471,17 +472,48 @@ def _check_hca_decode(st, ly, w, bsel):
     n_c, pos, m = w.n_hca, w.pos, h.ratio
     e = n_c - 1
     tb = pos - m + 1
-    Hh = {n: W.host_tensor(w, f"hca.{n}") for n in ("kv_c", "kv_z", "kv_b", "kv_g", "q", "q_norm_g", "sink", "win")}
+    pre = ly.prefix + "hca."
+    Hh = {n: W.host_tensor(w, pre + n) for n in ("kv_c", "kv_z", "kv_b", "kv_g", "q", "q_norm_g", "sink", "win")}
     gout = f64(ly.out)
     for b in bsel:
         ent = O.compress(m, e, e + 1, tb, Hh["kv_c"][b], Hh["kv_z"][b], Hh["kv_b"], norm_g=Hh["kv_g"],
                          rope_dim=h.rope_dim)[0]
         assert C.max_abs_rel(f64(ly.t["pool"][b, e]), ent) < C.OUT_TOL
-        pool = W.host_rows(w, "hca.pool", b * n_c + np.arange(n_c))
+        pool = W.host_rows(w, pre + "pool", b * n_c + np.arange(n_c))
         pool[e] = O.store_bf16(ent)
         out = O.hca_attend(Hh["q"][b, 0], Hh["q_norm_g"], pool, n_c, Hh["win"][b], h.window, Hh["sink"], pos, h)
         err = C.max_abs_rel(gout[b, 0], out)
         assert err < C.OUT_TOL, f"seq {b}: err {err}"
+
+
+def _check_swa_decode(st, ly, w, bsel):
+    h = w.hca
+    pre = ly.prefix + "swa."
+    Hs = {n: W.host_tensor(w, pre + n) for n in ("q", "q_norm_g", "sink", "win")}
+    gout = f64(ly.out)
+    for b in bsel:
+        out = O.hca_attend(Hs["q"][b, 0], Hs["q_norm_g"], np.zeros((0, h.head_dim)), 0, Hs["win"][b], h.window,
+                           Hs["sink"], w.pos, h)
+        err = C.max_abs_rel(gout[b, 0], out)
+        assert err < C.OUT_TOL, f"{ly.prefix} seq {b}: err {err}"
+
+
+def test_workload_schedule43_decode():
+    # one decode step through the 43 layers of the Flash schedule (two
+    # window-only layers, then CSA and HCA alternating): every layer's output
+    # against the oracle, both sequences
+    st = _state(8)
+    w = st.w
+    kinds = [ly.kind for ly in st.layers]
+    assert kinds[:4] == ["swa", "swa", "csa", "hca"] and len(kinds) == 43
+    assert kinds.count("csa") == 21 and kinds.count("hca") == 20
+    for ly in st.layers:
+        if ly.kind == "csa":
+            _check_csa_decode(st, ly, w, [0, 1])
+        elif ly.kind == "hca":
+            _check_hca_decode(st, ly, w, [0, 1])
+        else:
+            _check_swa_decode(st, ly, w, [0, 1])
 
 
 def test_workload_toy_csa_prefill():

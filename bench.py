@@ -165,6 +165,25 @@ def _csa_prefill_layer(w, dev, T, toy=None):
     return ly
 
 
+def _out_proj_layer(w, dev, T):
+    """The grouped output projection of one Flash layer for w.B tokens."""
+    import torch
+    import long_context_hybrid_kv_b200 as L
+    from gen import workloads as W
+
+    c = w.csa
+    ly = Layer()
+    ly.kind, ly.cfg_py = "out_proj", c
+    ly.cfg = L.OprojCfg(c.n_heads, c.head_dim, W.OPROJ_GROUPS, W.OPROJ_RANK, W.OPROJ_HIDDEN)
+    ly.t = {n[3:]: T[n] for n in T if n.startswith("op.")}
+    ly.B = w.B
+    ly.mid = torch.empty((w.B, W.OPROJ_GROUPS * W.OPROJ_RANK), dtype=torch.bfloat16, device=dev)
+    ly.out = torch.empty((w.B, W.OPROJ_HIDDEN), dtype=torch.bfloat16, device=dev)
+    ly.ws = torch.empty(max(1, L.ds4a_out_proj_workspace(ly.cfg, w.B) // 4), dtype=torch.float32, device=dev)
+    ly.step_inputs = ["o"]
+    return ly
+
+
 def _run_layer(ly, stream=None):
     """One layer's calls on `stream` (a CUDA stream handle; None = the
     current stream, looked up by each call)."""
@@ -186,6 +205,8 @@ def _run_layer(ly, stream=None):
                                t["pool"], norm_g=t["kv_g"], stream=S)
         L.ds4a_hca_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], t["pool"], ly.n_c, t["win"],
                           t["win"].shape[1], t["sink"], ly.out, ly.ws_att, stream=S)
+    elif ly.kind == "out_proj":
+        L.ds4a_out_proj(ly.cfg, t["o"], t["w_a"], t["w_b"], ly.mid, ly.out, ly.ws, stream=S)
     elif ly.kind == "swa":
         L.ds4a_hca_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], None, 0, t["win"], t["win"].shape[1],
                           t["sink"], ly.out, ly.ws_att, stream=S)
@@ -229,6 +250,8 @@ class State:
                 self.layers.append(_hca_decode_layer(w, w.B, w.pos, w.n_hca, dev, T))
             if w.kind == "csa_prefill":
                 self.layers.append(_csa_prefill_layer(w, dev, T))
+            if w.kind == "out_proj":
+                self.layers.append(_out_proj_layer(w, dev, T))
             if w.kind == "schedule_decode":
                 for pre, kind in W.schedule_layers(w):
                     if kind == "csa":
@@ -272,6 +295,14 @@ def kernel_work(state) -> dict:
 
     for ly in state.layers:
         c = ly.cfg_py
+        if ly.kind == "out_proj":
+            cf = ly.cfg
+            M = ly.B
+            k1 = (cf.n_heads // cf.n_groups) * cf.head_dim
+            n1 = cf.n_groups * cf.group_rank
+            nbytes = 2 * (M * cf.n_heads * cf.head_dim + n1 * k1 + cf.hidden * n1 + 2 * M * n1 + M * cf.hidden)
+            add("out_proj_gemm", nbytes, 2.0 * M * (n1 * k1 + cf.hidden * n1), launches=2)
+            continue
         if ly.kind == "swa":
             B, pos, D, H = ly.B, ly.pos, c.head_dim, c.n_heads
             n_win = pos - max(0, pos - c.window + 1) + 1
@@ -311,7 +342,7 @@ def kernel_work(state) -> dict:
 
 
 def kernel_family(name: str) -> str:
-    for fam in ("compress", "index_score", "topk", "attend_combine", "attend"):
+    for fam in ("compress", "index_score", "topk", "attend_combine", "attend", "out_proj_gemm"):
         if name.startswith(fam):
             return fam
     return name
@@ -658,6 +689,9 @@ def measure_workload(wid, args, stream, flush, barrier, world, dev, primary):
         "state": st,
         "work": work,
     }
+    lib_ref = library_gemm_ms(st)
+    if lib_ref is not None:
+        res["library_reference"] = lib_ref
     return res
 
 
@@ -667,6 +701,13 @@ def step_roofline(res, peaks, peak_src, workload):
     attention flops, over the step and over those kernels' own time."""
     work = res["work"]
     ms = res["ms_per_step"]
+    if "outproj_prefill" in workload:
+        flops = work.get("out_proj_gemm", (0, 0, 0))[1]
+        ach = flops / (ms / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        return {"bound": "tensor", "unit": "TFLOP/s", "what": "projection flops per step", "algorithmic": flops,
+                "achieved": ach, "frac": ach / peak, "frac_datasheet": ach / DATASHEET_PEAKS["bf16_tflops"],
+                "peak": peak, "peak_source": peak_src, "peak_datasheet": DATASHEET_PEAKS["bf16_tflops"]}
     if "prefill" in workload:
         flops = work.get("index_score", (0, 0, 0))[1] + work.get("attend", (0, 0, 0))[1]
         fam_ms = {}
@@ -695,6 +736,42 @@ def step_roofline(res, peaks, peak_src, workload):
             "algorithmic": nbytes, "achieved": ach, "frac": ach / peak,
             "frac_datasheet": ach / DATASHEET_PEAKS["hbm_gbs"], "peak": peak, "peak_source": peak_src,
             "peak_datasheet": DATASHEET_PEAKS["hbm_gbs"]}
+
+
+def library_gemm_ms(st, K: int = 10) -> dict | None:
+    """For the output-projection workloads: the same two products through
+    torch (cuBLAS), timed with CUDA events as a reference point (not part of
+    this library's path)."""
+    import torch
+
+    ly = st.layers[0]
+    if ly.kind != "out_proj":
+        return None
+    cf = ly.cfg
+    M = ly.B
+    o = ly.t["o"].view(M, cf.n_groups, -1).transpose(0, 1)         # [g, M, K1]
+    wa = ly.t["w_a"].transpose(1, 2)                                 # [g, K1, r]
+    wb = ly.t["w_b"]
+
+    def run():
+        mid = torch.bmm(o, wa).transpose(0, 1).reshape(M, -1)
+        return mid @ wb.t()
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = statistics.mean(ts)
+    flops = st_flops = 2.0 * M * 2 * (cf.n_groups * cf.group_rank) * ((cf.n_heads // cf.n_groups) * cf.head_dim)
+    return {"what": "torch bmm + matmul (cuBLAS), same products, context only", "ms": ms,
+            "tflops": st_flops / (ms / 1e3) / 1e12}
 
 
 def roofline_for(res, peaks, peak_src, workload):
@@ -882,6 +959,8 @@ def main(argv=None):
                        "tokens_per_step": rr["tokens_per_step"],
                        "roofline": roofline_for(rr, peaks, peak_src, lab),
                        "kernels": rr["kernels"]}
+        if "library_reference" in rr:
+            others[lab]["library_reference"] = rr["library_reference"]
     line["kernels"] = r["kernels"]
     if others:
         line["workloads"] = others

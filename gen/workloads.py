@@ -106,7 +106,14 @@ WORKLOADS = {
     # the same schedule at a size the oracle checks layer by layer quickly
     8: Workload(8, "schedule43_decode_b2_ctx16k", "schedule_decode", 2, 16383, FLASH_CSA, FLASH_HCA,
                 4096, 128, n_layers=43),
+    # grouped output projection of a Flash layer (64 heads x 512 in 8 groups,
+    # rank 1024, hidden 4096) for a decode batch and for a prefill
+    9: Workload(9, "outproj_decode_b8", "out_proj", 8, 0, FLASH_CSA, None, 0, 0),
+    10: Workload(10, "outproj_prefill_t16k", "out_proj", 16384, 0, FLASH_CSA, None, 0, 0),
 }
+
+# Flash grouped output projection: groups of heads, rank per group, hidden
+OPROJ_GROUPS, OPROJ_RANK, OPROJ_HIDDEN = 8, 1024, 4096
 
 
 def _gain(shape):
@@ -163,6 +170,13 @@ def specs(w: Workload) -> dict[str, Spec]:
         _csa_decode_specs(s, "", B, w.csa, w.n_csa)
     if w.kind in ("hca_decode", "mix_decode"):
         _hca_decode_specs(s, "", B, w.hca, w.n_hca)
+    if w.kind == "out_proj":
+        c = w.csa
+        k1 = (c.n_heads // OPROJ_GROUPS) * c.head_dim
+        s["op.o"] = Spec((B, c.n_heads, c.head_dim), "bf16")
+        s["op.w_a"] = Spec((OPROJ_GROUPS, OPROJ_RANK, k1), "bf16", 1.0 / math.sqrt(k1))
+        s["op.w_b"] = Spec((OPROJ_HIDDEN, OPROJ_GROUPS * OPROJ_RANK), "bf16",
+                           1.0 / math.sqrt(OPROJ_GROUPS * OPROJ_RANK))
     if w.kind == "schedule_decode":
         for pre, kind in schedule_layers(w):
             if kind == "csa":

@@ -272,6 +272,43 @@ int ds4a_hca_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_
                     int64_t win_bstride, const float* sink, ds4a_bf16* out, void* ws,
                     size_t ws_bytes, ds4a_stream stream);
 
+/* Grouped low-rank output projection of one layer ([beyond] 3.3 after eq.
+ * 26; [V4-inside] layer-0 section, grouped W_O with the 64 Flash heads in
+ * o_groups = 8; [hf-doc] grouped o_a projection followed by o_b).  Flash:
+ * {64, 512, 8, 1024, 4096}.
+ *   n_heads, head_dim  H, D of the attention output
+ *   n_groups           g: consecutive heads H/g form a group
+ *   group_rank         r: width of a group's intermediate projection
+ *   hidden             width of the layer's output */
+typedef struct ds4a_oproj_cfg {
+  int32_t n_heads, head_dim, n_groups, group_rank, hidden;
+} ds4a_oproj_cfg;
+
+/* Bytes of workspace ds4a_out_proj needs for M tokens (float partial sums
+ * when M is too small for the row and output tiles to fill the SMs, else
+ * 0). */
+size_t ds4a_out_proj_workspace(const ds4a_oproj_cfg* cfg, int M);
+
+/*
+ * ds4a_out_proj -- for each token t:
+ *   mid[t][j*r + i] = sum_c W_a[j][i][c] * o[t][j*(H/g)*D + c]   (group j)
+ *   y[t][n]         = sum_c W_b[n][c] * mid[t][c]                (c < g*r)
+ * with bf16 storage and float32 accumulation on the tensor cores (mid is
+ * stored as bf16 and read back by the second product).
+ *
+ *   o     device bf16 [M, H, D] (the attention output, heads in order)
+ *   w_a   device bf16 [g][r][(H/g)*D]  (each group's weight, rows = outputs)
+ *   w_b   device bf16 [hidden][g*r]
+ *   mid   device bf16 [M, g*r]  (output)
+ *   y     device bf16 [M, hidden] (output)
+ *   ws    device workspace of ds4a_out_proj_workspace(cfg, M) bytes
+ * (H/g)*D must be a multiple of 64, r and hidden multiples of 256
+ * (DS4A_EUNSUPPORTED otherwise).
+ */
+int ds4a_out_proj(const ds4a_oproj_cfg* cfg, int M, const ds4a_bf16* o, const ds4a_bf16* w_a,
+                  const ds4a_bf16* w_b, ds4a_bf16* mid, ds4a_bf16* y, void* ws, size_t ws_bytes,
+                  ds4a_stream stream);
+
 /* Failure-detection self test (no counterpart on the pages): launches one
  * block that waits, through the same bounded mbarrier wait the tensor-core
  * kernels use, on a barrier no thread ever arrives at, with a limit of

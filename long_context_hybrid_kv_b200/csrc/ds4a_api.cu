@@ -320,6 +320,53 @@ int ds4a_hca_attend(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_
                        win_cap, win_bstride, sink, out, ws, ws_bytes, stream, 0);
 }
 
+static int check_oproj(const ds4a_oproj_cfg* c) {
+  if (!c) return DS4A_EINVAL;
+  if (c->n_heads < 1 || c->head_dim < 1 || c->n_groups < 1 || c->group_rank < 1 || c->hidden < 1)
+    return DS4A_EINVAL;
+  if (c->n_heads % c->n_groups != 0) return DS4A_EINVAL;
+  const int64_t k1 = (int64_t)(c->n_heads / c->n_groups) * c->head_dim;
+  if (k1 % 64 != 0 || c->group_rank % 256 != 0 || c->hidden % 256 != 0) return DS4A_EUNSUPPORTED;
+  if (k1 > (1 << 20) || (int64_t)c->n_groups * c->group_rank > (1 << 20) || c->hidden > (1 << 20))
+    return DS4A_EUNSUPPORTED;
+  return DS4A_OK;
+}
+
+size_t ds4a_out_proj_workspace(const ds4a_oproj_cfg* cfg, int M) {
+  if (check_oproj(cfg) != DS4A_OK || M <= 0) return 0;
+  const int k1 = (cfg->n_heads / cfg->n_groups) * cfg->head_dim;
+  const int n1 = cfg->n_groups * cfg->group_rank;
+  const size_t a = gemm_acc_bytes(M, n1, k1), b = gemm_acc_bytes(M, cfg->hidden, n1);
+  return a > b ? a : b;
+}
+
+int ds4a_out_proj(const ds4a_oproj_cfg* cfg, int M, const ds4a_bf16* o, const ds4a_bf16* w_a,
+                  const ds4a_bf16* w_b, ds4a_bf16* mid, ds4a_bf16* y, void* ws, size_t ws_bytes,
+                  ds4a_stream stream) {
+  const int rc = check_oproj(cfg);
+  if (rc != DS4A_OK) return rc;
+  if (M < 0) return DS4A_EINVAL;
+  if (M == 0) return DS4A_OK;
+  if (!o || !w_a || !w_b || !mid || !y) return DS4A_EINVAL;
+  if (!aligned16(o) || !aligned16(w_a) || !aligned16(w_b) || !aligned16(mid) || !aligned16(y) ||
+      (ws && !aligned16(ws)))
+    return DS4A_EINVAL;
+  if (ws_bytes > 0 && !ws) return DS4A_EINVAL;
+  if ((ws ? ws_bytes : 0) < ds4a_out_proj_workspace(cfg, M)) return DS4A_ENOSPACE;
+  unsigned int* err = err_word();
+  if (!err) return DS4A_ECUDA;
+  const int H = cfg->n_heads, D = cfg->head_dim, g = cfg->n_groups, r = cfg->group_rank;
+  const int k1 = (H / g) * D, n1 = g * r;
+  cudaStream_t s = (cudaStream_t)stream;
+  float* acc = reinterpret_cast<float*>(ws);
+  // mid[t][j r + i] = W_a[j][i] . o[t][j K1 .. (j+1) K1)
+  cudaError_t e = launch_gemm(o, (int64_t)H * D, (int64_t)H * D, w_a, M, n1, k1, r, k1, mid, n1, acc, err, s);
+  if (e != cudaSuccess) return DS4A_ECUDA;
+  // y[t][n] = W_b[n] . mid[t]
+  e = launch_gemm(mid, n1, n1, w_b, M, cfg->hidden, n1, cfg->hidden, 0, y, cfg->hidden, acc, err, s);
+  return cuda_rc(e);
+}
+
 int ds4a_check(ds4a_stream stream, uint32_t* bits_out) {
   if (bits_out) *bits_out = 0;
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

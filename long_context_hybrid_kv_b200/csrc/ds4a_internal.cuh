@@ -276,4 +276,14 @@ bool attend_tc_supported(const AttendArgs& a);
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s);
 
+// Tensor-core GEMM of the grouped output projection (ds4a_outproj.cu):
+// out[M][N] (row stride ldo) = A x B^T with B = bf16 [N][K]; output tile
+// columns n read A's columns from (n / n_per_group) * a_group_k on.  acc: a
+// float [M][N] workspace when gemm_ksplit(M, N, K) > 1.
+int gemm_ksplit(int M, int N, int K);
+size_t gemm_acc_bytes(int M, int N, int K);
+cudaError_t launch_gemm(const uint16_t* a, int64_t a_cols, int64_t a_ld, const uint16_t* b, int M, int N, int K,
+                        int n_per_group, int a_group_k, uint16_t* out, int64_t ldo, float* acc,
+                        unsigned int* err, cudaStream_t s);
+
 }  // namespace ds4a

@@ -102,6 +102,33 @@ __device__ __forceinline__ void find_digit(const unsigned int* hist, int remaini
 // array is sized to whole groups of 32.
 __device__ __forceinline__ int kpos(int i) { return i ^ ((i >> 5) & 31); }
 
+// Stage scores [0, n) of `src` as keys in shared memory (slot kpos(i)),
+// every thread's loads in flight together (coalesced, kBatch per thread per
+// round), and return the largest key this thread staged.
+template <int kBatch>
+__device__ __forceinline__ unsigned int stage_keys(const float* __restrict__ src, int n, unsigned int* keys) {
+  unsigned int tmax = 0u;
+  const int nt = blockDim.x, tid = threadIdx.x;
+  for (int base = 0; base < n; base += kBatch * nt) {
+    float v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * nt + tid;
+      v[u] = i < n ? src[i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * nt + tid;
+      if (i < n) {
+        const unsigned int key = f2key(v[u]);
+        keys[kpos(i)] = key;
+        tmax = max(tmax, key);
+      }
+    }
+  }
+  return tmax;
+}
+
 __device__ __forceinline__ void write_identity(const IndexArgs& a, int n_vis, const float* sc, int32_t* out,
                                                float* so) {
   for (int i = threadIdx.x; i < a.k; i += blockDim.x) {
@@ -130,7 +157,7 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
     write_identity(a, n_vis, sc, out, so);
     return;
   }
-  for (int i = tid; i < n_vis; i += blockDim.x) keys[kpos(i)] = f2key(sc[i]);
+  stage_keys<8>(sc, n_vis, keys);
   unsigned int prefix = 0, mask = 0;
   int remaining = a.k;
   for (int pass = 0; pass < 4; ++pass) {
@@ -208,13 +235,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   const int lo = min(n_vis, rank * slice), hi = min(n_vis, lo + slice);
   const int n = hi - lo;
   // stage the slice; thread t's keys are t, t + 1024, ...: keep their max
-  unsigned int tmax = 0u;
-  for (int i = tid; i < n; i += blockDim.x) {
-    const unsigned int u = f2key(sc[lo + i]);
-    keys[kpos(i)] = u;
-    tmax = max(tmax, u);
-  }
-  tmaxs[tid] = tmax;
+  tmaxs[tid] = stage_keys<8>(sc + lo, n, keys);
   // Radix select over the cluster (k-th largest of vals[0..nv) in every
   // block, counting only values >= floor): the key T and how many of the
   // values equal to T are needed.

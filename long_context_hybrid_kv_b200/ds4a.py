@@ -16,7 +16,7 @@ __all__ = [
     "DS4A_ENOSPACE", "Ds4aError", "LayerCfg", "layer_cfg", "lib", "LIB_PATH", "ds4a_compress",
     "ds4a_compress_state_bytes", "ds4a_compress_append", "ds4a_index_topk_workspace", "ds4a_index_topk", "ds4a_index_topk_noalloc", "ds4a_attend_workspace", "ds4a_sparse_attend",
     "ds4a_hca_attend", "ds4a_check", "ds4a_strerror", "ds4a_trace_enable", "ds4a_trace_read",
-    "ds4a_version", "ds4a_selftest_wait_timeout",
+    "ds4a_version", "ds4a_selftest_wait_timeout", "OprojCfg", "ds4a_out_proj_workspace", "ds4a_out_proj",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libds4a.so")
@@ -37,6 +37,11 @@ class LayerCfg(ctypes.Structure):
                 ("topk", ctypes.c_int32), ("ratio", ctypes.c_int32),
                 ("sm_scale", ctypes.c_float), ("rope_base", ctypes.c_float),
                 ("rms_eps", ctypes.c_float)]
+
+
+class OprojCfg(ctypes.Structure):
+    _fields_ = [("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("n_groups", ctypes.c_int32),
+                ("group_rank", ctypes.c_int32), ("hidden", ctypes.c_int32)]
 
 
 def layer_cfg(c) -> LayerCfg:
@@ -65,6 +70,8 @@ _SIGS = {
     "ds4a_sparse_attend": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _I, _I64, _P, _P, _P, _SZ, _P]),
     "ds4a_hca_attend": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _I, _I64, _P, _P, _P, _SZ, _P]),
     "ds4a_check": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "ds4a_out_proj_workspace": (_SZ, [ctypes.POINTER(OprojCfg), _I]),
+    "ds4a_out_proj": (_I, [ctypes.POINTER(OprojCfg), _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "ds4a_selftest_wait_timeout": (_I, [_I64, _P, _P]),
     "ds4a_strerror": (ctypes.c_char_p, [_I]),
     "ds4a_trace_enable": (_I, [_I]),
@@ -213,6 +220,20 @@ def ds4a_hca_attend(cfg: LayerCfg, q_pos, q, q_norm_g, pool, N_c: int, win, win_
                                win_cap, 0 if win is None else win.stride(0), _ptr(sink), _ptr(out),
                                _ptr(ws), ws_bytes, _stream(stream))
     _ok(rc, "ds4a_hca_attend")
+
+
+def ds4a_out_proj_workspace(cfg: OprojCfg, M: int) -> int:
+    return lib().ds4a_out_proj_workspace(ctypes.byref(cfg), M)
+
+
+def ds4a_out_proj(cfg: OprojCfg, o, w_a, w_b, mid, y, ws=None, *, stream=None):
+    """o [M, H, D] -> mid [M, g*r] and y [M, hidden] (grouped projection)."""
+    _bf16(o, "o"), _bf16(w_a, "w_a"), _bf16(w_b, "w_b")
+    M = o.shape[0]
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = lib().ds4a_out_proj(ctypes.byref(cfg), M, _ptr(o), _ptr(w_a), _ptr(w_b), _ptr(mid), _ptr(y), _ptr(ws),
+                             ws_bytes, _stream(stream))
+    _ok(rc, "ds4a_out_proj")
 
 
 def ds4a_check(stream=None) -> tuple[int, int]:

@@ -266,6 +266,33 @@ def attended_key_count(pos: int, cfg, n_c: int, sparse: bool) -> int:
 
 
 # --------------------------------------------------------------------------
+# (5) grouped low-rank output projection
+# [beyond] 3.3 after eq. 26: the head outputs of a token, concatenated, are
+# split into g groups of consecutive heads; each group is projected to an
+# intermediate of rank r, and the g intermediates side by side are projected
+# to the layer's output.  [V4-inside] layer-0 section: grouped W_O (Flash:
+# 64 heads in 8 groups); [hf-doc]: grouped o_a projection, then o_b.
+# --------------------------------------------------------------------------
+def out_proj_mid(o, w_a, n_groups: int) -> np.ndarray:
+    """o [M, H, D], w_a [g][r][(H/g) D] -> float64 [M, g r]: group j's
+    intermediate is W_a[j] applied to the concatenation of its heads."""
+    o = widen(o)
+    M = o.shape[0]
+    x = o.reshape(M, n_groups, -1)  # [M, g, (H/g) D], heads in order
+    wa = widen(w_a)
+    return np.concatenate([x[:, j] @ wa[j].T for j in range(n_groups)], axis=1)
+
+
+def out_proj(o, w_a, w_b, n_groups: int):
+    """(intermediate float64 [M, g r], output float64 [M, hidden]).  The
+    intermediate goes through the ABI's bf16 storage before the second
+    product (reading R12)."""
+    mid = out_proj_mid(o, w_a, n_groups)
+    y = widen(store_bf16(mid)) @ widen(w_b).T
+    return mid, y
+
+
+# --------------------------------------------------------------------------
 # batch drivers (loops over sequences and queries)
 # --------------------------------------------------------------------------
 def index_topk_batch(qi, wi, ki, q_pos, m: int, k: int, n_c: int, rows=None):

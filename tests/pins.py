@@ -531,4 +531,40 @@ def pin_compress_norm_and_rope(O):
     _close(unrot, raw / np.sqrt(ms + 1e-6)[:, None], 1e-12, "norm then RoPE at i*m")
 
 
+# --------------------------------------------------------------------------
+# grouped output projection
+# --------------------------------------------------------------------------
+def pin_out_proj_block_diagonal(O):
+    """The grouped projection equals one dense product with the block-diagonal
+    matrix of the group weights (torch.block_diag), applied to the heads in
+    order."""
+    rng = np.random.default_rng(17)
+    M, H, D, g, r = 5, 6, 4, 3, 5
+    o = rng.standard_normal((M, H, D))
+    wa = rng.standard_normal((g, r, (H // g) * D))
+    big = torch.block_diag(*[torch.from_numpy(wa[j]) for j in range(g)]).numpy()  # [g r, H D]
+    _close(O.out_proj_mid(o, wa, g), o.reshape(M, -1) @ big.T, 1e-12, "grouped == block-diagonal")
+
+
+def pin_out_proj_groups_are_separate(O):
+    """A token whose only non-zero value sits in head h feeds only the
+    intermediate of h's group; with W_b the identity the output is that
+    intermediate as stored (bf16)."""
+    rng = np.random.default_rng(18)
+    M, H, D, g, r = 1, 8, 2, 4, 3
+    wa = rng.standard_normal((g, r, (H // g) * D))
+    for h in range(H):
+        o = np.zeros((M, H, D))
+        o[0, h, 1] = 1.0
+        mid = O.out_proj_mid(o, wa, g)
+        j = h // (H // g)
+        mask = np.zeros(g * r, bool)
+        mask[j * r:(j + 1) * r] = True
+        assert np.all(mid[0, ~mask] == 0.0), f"head {h} leaks outside group {j}"
+        _close(mid[0, mask], wa[j][:, (h % (H // g)) * D + 1], 0.0, f"head {h} column")
+    o = rng.standard_normal((M, H, D))
+    mid, y = O.out_proj(o, wa, np.eye(g * r), g)
+    _close(y, O.widen(O.store_bf16(mid)), 0.0, "identity W_b")
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

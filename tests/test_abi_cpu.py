@@ -168,6 +168,29 @@ def test_compress_append_rejects_bad_args():
     assert L.ds4a_compress_state_bytes(hca, 8, 512, False) == 8 * 2 * 128 * 512 * 2
 
 
+def test_out_proj_rejects_bad_args():
+    lib = L.lib()
+
+    def call(cfg=(64, 512, 8, 1024, 4096), M=8, **kw):
+        a = dict(o=A, wa=A, wb=A, mid=A, y=A, ws=A, wsb=8 << 20)
+        a.update(kw)
+        c = L.OprojCfg(*cfg)
+        return lib.ds4a_out_proj(ctypes.byref(c), M, a["o"], a["wa"], a["wb"], a["mid"], a["y"], a["ws"],
+                                 a["wsb"], None)
+
+    assert call(M=0) == L.DS4A_OK
+    assert call(M=-1) == L.DS4A_EINVAL
+    assert call(cfg=(64, 512, 7, 1024, 4096)) == L.DS4A_EINVAL      # heads not divisible
+    assert call(cfg=(64, 512, 8, 1000, 4096)) == L.DS4A_EUNSUPPORTED  # rank not a multiple of 256
+    assert call(cfg=(64, 512, 8, 1024, 4000)) == L.DS4A_EUNSUPPORTED
+    assert call(o=None) == L.DS4A_EINVAL
+    assert call(y=MIS) == L.DS4A_EINVAL
+    assert call(ws=None, wsb=0) == L.DS4A_ENOSPACE                    # decode needs split-K partials
+    cfg = L.OprojCfg(64, 512, 8, 1024, 4096)
+    assert L.ds4a_out_proj_workspace(cfg, 8) == 8 * 8192 * 4
+    assert L.ds4a_out_proj_workspace(cfg, 16384) == 0
+
+
 def test_workspace_queries():
     cfg = flash_cfg()
     assert L.ds4a_index_topk_workspace(cfg, 8, 1, 262144) == 8 * 262144 * 4

@@ -48,6 +48,11 @@ MUTANTS = {
                               "return (b >> np.uint32(16)).astype(np.uint16)")],
     "store_bf16 ties away from zero": [("return ((b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)",
                                         "return ((b + np.uint32(0x8000)) >> np.uint32(16)).astype(np.uint16)")],
+    "out_proj heads strided across groups": [("x = o.reshape(M, n_groups, -1)  # [M, g, (H/g) D], heads in order",
+                                              "x = o.reshape(M, -1, n_groups).transpose(0, 2, 1)")],
+    "out_proj weight transposed per group": [("np.concatenate([x[:, j] @ wa[j].T for j in range(n_groups)], axis=1)",
+                                              "np.concatenate([x[:, j] @ wa[j].reshape(-1, wa.shape[1]) for j in range(n_groups)], axis=1)")],
+    "out_proj second product unrounded": [("y = widen(store_bf16(mid)) @ widen(w_b).T", "y = mid @ widen(w_b).T")],
     "pool row ignores idx": [("rows = np.concatenate([widen(pool)[sel], window_rows",
                               "rows = np.concatenate([widen(pool)[: sel.size], window_rows")],
 }

@@ -95,6 +95,18 @@ def _csa_decode_layer(w, B, pos, n_c, dev, T, pre=""):
     ly.entry = (pos + 1) // c.ratio - 1  # the entry that closes at this token
     ly.state_kv = _ring_state(ly, ["kv_ca", "kv_cb", "kv_za", "kv_zb"], 2 * c.ratio, dev)
     ly.state_ix = _ring_state(ly, ["ix_ca", "ix_cb", "ix_za", "ix_zb"], 2 * c.ratio, dev)
+    ly.mx = w.storage == "mx"
+    if ly.mx:
+        # block-scaled caches made by the library's quantisers from the
+        # generated bf16 pools, which are then dropped
+        rb = L.ds4a_kv_fp8_row_bytes(c.head_dim, c.rope_dim)
+        ly.kv8 = torch.empty((B, n_c, rb), dtype=torch.uint8, device=dev)
+        L.ds4a_quantize_kv_fp8(ly.t["pool"].reshape(B * n_c, -1), c.rope_dim, ly.kv8.view(B * n_c, rb))
+        ly.ki4 = torch.empty((B, n_c, c.idx_dim // 2), dtype=torch.uint8, device=dev)
+        ly.ki4s = torch.empty((B, n_c, c.idx_dim // 32), dtype=torch.uint8, device=dev)
+        L.ds4a_quantize_idx_fp4(ly.t["ki"].reshape(B * n_c, -1), ly.ki4.view(B * n_c, -1), ly.ki4s.view(B * n_c, -1))
+        torch.cuda.synchronize()
+        del ly.t["pool"], ly.t["ki"]
     ly.step_inputs = ["q", "qi", "wi", "kv_ca_new", "kv_cb_new", "kv_za_new", "kv_zb_new", "ix_ca_new",
                       "ix_cb_new", "ix_za_new", "ix_zb_new"]
     return ly
@@ -117,6 +129,13 @@ def _hca_decode_layer(w, B, pos, n_c, dev, T, pre=""):
     ly.entry = (pos + 1) // h.ratio - 1
     ly.state_kv = _ring_state(ly, ["kv_c", "kv_z"], h.ratio, dev)
     ly.step_inputs = ["q", "kv_c_new", "kv_z_new"]
+    ly.mx = w.storage == "mx"
+    if ly.mx:
+        rb = L.ds4a_kv_fp8_row_bytes(h.head_dim, h.rope_dim)
+        ly.kv8 = torch.empty((B, n_c, rb), dtype=torch.uint8, device=dev)
+        L.ds4a_quantize_kv_fp8(ly.t["pool"].reshape(B * n_c, -1), h.rope_dim, ly.kv8.view(B * n_c, rb))
+        torch.cuda.synchronize()
+        del ly.t["pool"]
     return ly
 
 
@@ -191,7 +210,24 @@ def _run_layer(ly, stream=None):
 
     t = ly.t
     S = stream
-    if ly.kind == "csa":
+    if ly.kind == "csa" and ly.mx:
+        pos = ly.q_pos.view(-1)
+        L.ds4a_compress_append_mx(ly.cfg, pos, t["kv_ca_new"], t["kv_za_new"], t["kv_ba"], ly.state_kv,
+                                  L.DS4A_MX_KV_FP8, ly.kv8, cb=t["kv_cb_new"], zb=t["kv_zb_new"], bias_b=t["kv_bb"],
+                                  norm_g=t["kv_g"], stream=S)
+        L.ds4a_compress_append_mx(ly.cfg, pos, t["ix_ca_new"], t["ix_za_new"], t["ix_ba"], ly.state_ix,
+                                  L.DS4A_MX_IDX_FP4, ly.ki4, scales=ly.ki4s, cb=t["ix_cb_new"], zb=t["ix_zb_new"],
+                                  bias_b=t["ix_bb"], stream=S)
+        L.ds4a_index_topk_fp4(ly.cfg, ly.q_pos, t["qi"], t["wi"], ly.ki4, ly.ki4s, ly.n_c, ly.idx, ly.ws_index,
+                              stream=S)
+        L.ds4a_sparse_attend_fp8(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], ly.kv8, ly.n_c, ly.idx, t["win"],
+                                 t["win"].shape[1], t["sink"], ly.out, ly.ws_att, stream=S)
+    elif ly.kind == "hca" and ly.mx:
+        L.ds4a_compress_append_mx(ly.cfg, ly.q_pos.view(-1), t["kv_c_new"], t["kv_z_new"], t["kv_b"], ly.state_kv,
+                                  L.DS4A_MX_KV_FP8, ly.kv8, norm_g=t["kv_g"], stream=S)
+        L.ds4a_hca_attend_fp8(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], ly.kv8, ly.n_c, t["win"], t["win"].shape[1],
+                              t["sink"], ly.out, ly.ws_att, stream=S)
+    elif ly.kind == "csa":
         pos = ly.q_pos.view(-1)
         L.ds4a_compress_append(ly.cfg, pos, t["kv_ca_new"], t["kv_za_new"], t["kv_ba"], ly.state_kv, t["pool"],
                                cb=t["kv_cb_new"], zb=t["kv_zb_new"], bias_b=t["kv_bb"], norm_g=t["kv_g"], stream=S)
@@ -313,19 +349,24 @@ def kernel_work(state) -> dict:
             n_vis = min((pos + 1) // m, n_c)
             n_win = pos - max(0, pos - c.window + 1) + 1
             D, H = c.head_dim, c.n_heads
+            mx = getattr(ly, "mx", False)
+            row = (D - c.rope_dim) + 2 * c.rope_dim + (D - c.rope_dim) // 32 if mx else 2 * D  # bytes per K=V row
+            krow = c.idx_dim // 2 + c.idx_dim // 32 if mx else 2 * c.idx_dim  # bytes per indexer key
             # compressor: 2m (CSA) or m (HCA) tokens x (C + Z) + biases + gain, one entry out
             streams = (4 if ly.kind == "csa" else 2) * m
-            add("compress", B * (streams * D * 2 + 2 * m * D * 4 + D * 4 + D * 2))
+            add("compress", B * (streams * D * 2 + 2 * m * D * 4 + D * 4 + row))
             if ly.kind == "csa":
-                add("compress", B * (streams * c.idx_dim * 2 + 2 * m * c.idx_dim * 4 + c.idx_dim * 2))
+                add("compress", B * (streams * c.idx_dim * 2 + 2 * m * c.idx_dim * 4 + krow))
                 qb = c.idx_heads * c.idx_dim * 2 + c.idx_heads * 2
-                add("index_score", B * (n_vis * c.idx_dim * 2 + qb + n_vis * 4),
+                add("index_score", B * (n_vis * krow + qb + n_vis * 4),
                     2.0 * B * n_vis * c.idx_heads * c.idx_dim)
                 add("topk", B * (n_vis * 4 + c.topk * 4))
                 n_keys = min(c.topk, n_vis) + n_win
             else:
                 n_keys = n_vis + n_win
-            add("attend", B * (n_keys * D * 2 + 2 * H * D * 2 + H * 4 + D * 4), 4.0 * B * n_keys * H * D)
+            n_pool = n_keys - n_win
+            add("attend", B * (n_pool * row + n_win * D * 2 + 2 * H * D * 2 + H * 4 + D * 4),
+                4.0 * B * n_keys * H * D)
         else:  # prefill
             Tn, m, D, H = ly.T, ly.m, c.head_dim, c.n_heads
             n_c = ly.n_c

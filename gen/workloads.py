@@ -61,6 +61,7 @@ class Workload:
     n_csa: int  # compressed entries in the CSA pool
     n_hca: int
     n_layers: int = 0  # schedule_decode: layers of the Flash schedule
+    storage: str = "bf16"  # "mx": FP8 / BF16 K=V pools and FP4 indexer keys
 
     @property
     def seed(self) -> int:
@@ -110,6 +111,10 @@ WORKLOADS = {
     # rank 1024, hidden 4096) for a decode batch and for a prefill
     9: Workload(9, "outproj_decode_b8", "out_proj", 8, 0, FLASH_CSA, None, 0, 0),
     10: Workload(10, "outproj_prefill_t16k", "out_proj", 16384, 0, FLASH_CSA, None, 0, 0),
+    # the 1M mix with block-scaled caches: FP8 K=V pools (RoPE dims BF16) and
+    # FP4 indexer keys; the same generated values, quantised on the device
+    11: Workload(11, "mix_decode_b8_ctx1m_mx", "mix_decode", 8, 1048575, FLASH_CSA, FLASH_HCA, 262144, 8192,
+                 storage="mx"),
 }
 
 # Flash grouped output projection: groups of heads, rank per group, hidden

@@ -172,6 +172,64 @@ int ds4a_compress_append(const ds4a_layer_cfg* cfg, int B, int c, const int32_t*
                          const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
                          int64_t pool_bstride, ds4a_stream stream);
 
+/*
+ * Block-scaled cache storage ([V4-inside] "What does HCA change?", paper
+ * 2.3.4: the K=V cache keeps its RoPE dims in BF16 and the other dims in FP8;
+ * the indexer keys are FP4).  Element formats and block scaling after the
+ * OCP Microscaling (MX) formats: 32 consecutive values share one
+ * power-of-two scale stored as E8M0 (exponent + 127), the smallest power of
+ * two that keeps the block's largest magnitude within the element format;
+ * elements round to nearest even.  FP8 is E4M3 (largest 448), FP4 is E2M1
+ * (largest 6).
+ *
+ *   DS4A_MX_KV_FP8   one K=V entry of D dims (the last R in BF16) is a row of
+ *                    ds4a_kv_fp8_row_bytes(D, R) bytes:
+ *                      [0, D-R)          E4M3 codes of dims 0 .. D-R-1
+ *                      [D-R, D+R)        BF16 of dims D-R .. D-1, as stored
+ *                      [D+R, D+R+(D-R)/32)  E8M0 scales, one per 32 dims
+ *                      zero padding to a multiple of 16 (592 bytes at the
+ *                      Flash shape D = 512, R = 64)
+ *   DS4A_MX_IDX_FP4  one indexer key of D_I dims is D_I/2 bytes of E2M1 codes
+ *                    (element 2i in the low nibble) in a codes array, and
+ *                    D_I/32 E8M0 scales in a separate scales array
+ * Strides of block-scaled pools are in entries (rows).
+ */
+enum { DS4A_MX_KV_FP8 = 1, DS4A_MX_IDX_FP4 = 2 };
+
+/* Bytes of one DS4A_MX_KV_FP8 row (0 when D - R is not a multiple of 32 or
+ * R not a multiple of 8). */
+size_t ds4a_kv_fp8_row_bytes(int D, int R);
+
+/* bf16 K=V rows in[n][in_stride] -> DS4A_MX_KV_FP8 rows out (out_stride
+ * bytes apart, a multiple of 16).  Device pointers, 16-byte aligned. */
+int ds4a_quantize_kv_fp8(int n_rows, int D, int R, const ds4a_bf16* in, int64_t in_stride, uint8_t* out,
+                         int64_t out_stride, ds4a_stream stream);
+
+/* bf16 indexer keys in[n][in_stride] (D a multiple of 32) -> codes [n][D/2]
+ * and scales [n][D/32] (DS4A_MX_IDX_FP4).  Device pointers; in and codes
+ * 16-byte aligned. */
+int ds4a_quantize_idx_fp4(int n_rows, int D, const ds4a_bf16* in, int64_t in_stride, uint8_t* codes,
+                          uint8_t* scales, ds4a_stream stream);
+
+/*
+ * ds4a_compress_append_mx -- ds4a_compress_append writing the entries in a
+ * block-scaled format: the entry is computed as ds4a_compress_append does,
+ * rounded to bf16 (the ABI's storage type), then quantised.
+ *   format   DS4A_MX_KV_FP8 (K=V entries; R = cfg->rope_dim when norm_g is
+ *            given, else 0) or DS4A_MX_IDX_FP4 (indexer keys)
+ *   pool     device, entry i of sequence b at row b * pool_bstride + i of
+ *            the format's rows (FP8: row bytes; FP4: c/2 code bytes)
+ *   scales   FP4 only: device, c/32 bytes per entry, same row numbering
+ *   pool_bstride  entries between sequences (>= N_cap)
+ * c must be a multiple of 64 and c - R a multiple of 32 (DS4A_EUNSUPPORTED
+ * otherwise).  Everything else is as ds4a_compress_append.
+ */
+int ds4a_compress_append_mx(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
+                            const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                            const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                            const float* norm_g, ds4a_bf16* state, int N_cap, int format, uint8_t* pool,
+                            uint8_t* scales, int64_t pool_bstride, ds4a_stream stream);
+
 /* Bytes of workspace ds4a_index_topk needs for these sizes. */
 size_t ds4a_index_topk_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c);
 
@@ -197,6 +255,21 @@ int ds4a_index_topk(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_
                     const ds4a_bf16* q_idx, const ds4a_bf16* w_idx, const ds4a_bf16* k_idx,
                     int64_t k_bstride, int N_c, int32_t* idx_out, float* score_out, void* ws,
                     size_t ws_bytes, ds4a_stream stream);
+
+/*
+ * ds4a_index_topk_fp4 -- ds4a_index_topk over FP4 indexer keys
+ * (DS4A_MX_IDX_FP4): the score uses the keys' exact values (code times
+ * scale); queries and weights stay bf16.
+ *   k_codes   device, batch b's keys at k_codes + (b * k_bstride) * D_I/2
+ *   k_scales  device, batch b's keys at k_scales + (b * k_bstride) * D_I/32
+ *   k_bstride keys between sequences, a multiple of 4
+ * The Flash indexer shape only (64 heads x 128), N_c a multiple of 4
+ * (DS4A_EUNSUPPORTED otherwise); both arrays 16-byte aligned.
+ */
+int ds4a_index_topk_fp4(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                        const ds4a_bf16* q_idx, const ds4a_bf16* w_idx, const uint8_t* k_codes,
+                        const uint8_t* k_scales, int64_t k_bstride, int N_c, int32_t* idx_out,
+                        float* score_out, void* ws, size_t ws_bytes, ds4a_stream stream);
 
 /*
  * ds4a_index_topk_noalloc -- ds4a_index_topk for callers that cannot
@@ -318,6 +391,28 @@ int ds4a_out_proj(const ds4a_oproj_cfg* cfg, int M, const ds4a_bf16* o, const ds
  * completed) and exits, so ds4a_check then returns DS4A_ETIMEOUT and the
  * context stays usable.  No GPU fault is involved. */
 int ds4a_selftest_wait_timeout(int64_t limit_cycles, int32_t* status_out, ds4a_stream stream);
+
+/*
+ * ds4a_sparse_attend_fp8 / ds4a_hca_attend_fp8 -- ds4a_sparse_attend and
+ * ds4a_hca_attend over a DS4A_MX_KV_FP8 pool: every pool row enters the
+ * products with its exact values (E4M3 code times the block's scale, the
+ * RoPE dims as stored); window rows stay bf16.
+ *   pool          device, batch b's rows at pool + (b * pool_bstride) *
+ *                 ds4a_kv_fp8_row_bytes(D, R), 16-byte aligned
+ *   pool_bstride  rows between sequences (>= N_c)
+ * The Flash shape only (64 heads x 512, RoPE 64; DS4A_EUNSUPPORTED
+ * otherwise).  Everything else is as the bf16 calls.
+ */
+int ds4a_sparse_attend_fp8(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                           const ds4a_bf16* q, const float* q_norm_g, const uint8_t* pool,
+                           int64_t pool_bstride, int N_c, const int32_t* idx, const ds4a_bf16* win,
+                           int win_cap, int64_t win_bstride, const float* sink, ds4a_bf16* out,
+                           void* ws, size_t ws_bytes, ds4a_stream stream);
+int ds4a_hca_attend_fp8(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                        const ds4a_bf16* q, const float* q_norm_g, const uint8_t* pool,
+                        int64_t pool_bstride, int N_c, const ds4a_bf16* win, int win_cap,
+                        int64_t win_bstride, const float* sink, ds4a_bf16* out, void* ws,
+                        size_t ws_bytes, ds4a_stream stream);
 
 /* Synchronise the stream, then read and clear the current device's error
  * word.  Returns DS4A_OK, DS4A_EDEVICE (bad index / position),

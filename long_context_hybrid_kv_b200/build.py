@@ -16,8 +16,8 @@ OUT = os.path.join(PKG, "_lib", "libds4a.so")
 BUILD = os.path.join(ROOT, "_build", "ds4a")
 
 SOURCES = ["ds4a_api.cu", "ds4a_generic.cu", "ds4a_index_tc.cu", "ds4a_attend_tc.cu", "ds4a_noalloc.cu", "ds4a_topk.cu",
-           "ds4a_selftest.cu", "ds4a_outproj.cu"]
-HEADERS = ["ds4a_internal.cuh", "ds4a_tc.cuh"]
+           "ds4a_selftest.cu", "ds4a_outproj.cu", "ds4a_mx.cu"]
+HEADERS = ["ds4a_internal.cuh", "ds4a_tc.cuh", "ds4a_mx.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -1,6 +1,7 @@
 // extern "C" entry points of libds4a: argument checks (before any launch),
 // dispatch to the kernels, the device error word and the launch trace.
 #include "ds4a_internal.cuh"
+#include "ds4a_mx.cuh"
 
 #include <math.h>
 #include <stdio.h>
@@ -71,6 +72,8 @@ TraceScope::~TraceScope() {
 using namespace ds4a;
 
 namespace {
+
+constexpr int kMxBlockApi = kMxBlock;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -154,6 +157,7 @@ int ds4a_compress(const ds4a_layer_cfg* cfg, int B, int T_tok, int tok_begin, in
   a.entry_begin = entry_begin; a.entry_end = entry_end;
   a.pool = pool; a.pool_bstride = pool_bstride;
   a.app_pos = nullptr; a.ring = nullptr; a.ring_cap = 0; a.n_cap = 0;
+  a.qfmt = 0; a.qpool = nullptr; a.q_bstride = 0; a.q_row = 0; a.qscales = nullptr; a.qs_bstride = 0;
   fill_rope_theta(&a.rope, a.rope_dim, cfg->rope_base);
   a.err = err_word();
   if (!a.err) return DS4A_ECUDA;
@@ -166,28 +170,38 @@ size_t ds4a_compress_state_bytes(const ds4a_layer_cfg* cfg, int B, int c, int ov
   return (size_t)B * S * cap * (size_t)c * sizeof(uint16_t);
 }
 
-int ds4a_compress_append(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
-                         const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
-                         const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
-                         const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
-                         int64_t pool_bstride, ds4a_stream stream) {
+// the append call, bf16 (qfmt 0) or block-scaled output (qfmt 1, 2)
+static int compress_append_common(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
+                                  const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                                  const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                                  const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
+                                  int64_t pool_bstride, int qfmt, uint8_t* qpool, uint8_t* qscales,
+                                  int64_t q_bstride_rows, ds4a_stream stream) {
   if (!cfg || cfg->ratio < 1) return DS4A_EINVAL;
   if (B < 0 || N_cap < 0 || c < 2 || c > 1024 || (c % 2) != 0) return DS4A_EINVAL;
   if ((c % 8) != 0 && c > 512) return DS4A_EINVAL;
   if (B == 0) return DS4A_OK;
-  if (!pos || !ca || !za || !bias_a || !state || !pool) return DS4A_EINVAL;
+  if (!pos || !ca || !za || !bias_a || !state) return DS4A_EINVAL;
+  if (qfmt == 0 ? !pool : !qpool) return DS4A_EINVAL;
+  if (qfmt == 2 && !qscales) return DS4A_EINVAL;
   const bool overlap = cb != nullptr;
   if (overlap && (!zb || !bias_b)) return DS4A_EINVAL;
   if (!overlap && (zb || bias_b)) return DS4A_EINVAL;
   if (!aligned16(pos) || !aligned16(ca) || !aligned16(za) || !aligned16(bias_a) || !aligned16(state) ||
-      !aligned16(pool))
+      (pool && !aligned16(pool)) || (qpool && !aligned16(qpool)))
     return DS4A_EINVAL;
   if (overlap && (!aligned16(cb) || !aligned16(zb) || !aligned16(bias_b))) return DS4A_EINVAL;
   if (norm_g) {
     if (check_cfg(cfg) != DS4A_OK) return DS4A_EINVAL;
     if (cfg->rope_dim > c) return DS4A_EINVAL;
   }
-  if (pool_bstride < (int64_t)N_cap * c || (pool_bstride % 2) != 0) return DS4A_EINVAL;
+  const int R = norm_g ? cfg->rope_dim : 0;
+  if (qfmt == 0) {
+    if (pool_bstride < (int64_t)N_cap * c || (pool_bstride % 2) != 0) return DS4A_EINVAL;
+  } else {
+    // 64-channel warps hold whole 32-channel blocks
+    if (c % 64 != 0 || (c - R) % kMxBlockApi != 0 || q_bstride_rows < N_cap) return DS4A_EUNSUPPORTED;
+  }
   const int m = cfg->ratio;
   if ((int64_t)(overlap ? 2 * m : m) * c > (int64_t)1 << 24) return DS4A_EINVAL;
 
@@ -200,10 +214,57 @@ int ds4a_compress_append(const ds4a_layer_cfg* cfg, int B, int c, const int32_t*
   a.entry_begin = 0; a.entry_end = 1;
   a.pool = pool; a.pool_bstride = pool_bstride;
   a.app_pos = pos; a.ring = state; a.ring_cap = overlap ? 2 * m : m; a.n_cap = N_cap;
+  a.qfmt = qfmt; a.qpool = qpool; a.qscales = qscales;
+  a.q_row = qfmt == 1 ? kv_fp8_row_bytes(c, R) : c / 2;
+  a.q_bstride = q_bstride_rows * a.q_row;
+  a.qs_bstride = q_bstride_rows * (c / kMxBlockApi);
   fill_rope_theta(&a.rope, a.rope_dim, cfg->rope_base);
   a.err = err_word();
   if (!a.err) return DS4A_ECUDA;
   return cuda_rc(launch_compress(a, (cudaStream_t)stream));
+}
+
+int ds4a_compress_append(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
+                         const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                         const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                         const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
+                         int64_t pool_bstride, ds4a_stream stream) {
+  return compress_append_common(cfg, B, c, pos, ca, cb, za, zb, bias_a, bias_b, norm_g, state, N_cap, pool,
+                                pool_bstride, 0, nullptr, nullptr, 0, stream);
+}
+
+int ds4a_compress_append_mx(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
+                            const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                            const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                            const float* norm_g, ds4a_bf16* state, int N_cap, int format, uint8_t* pool,
+                            uint8_t* scales, int64_t pool_bstride, ds4a_stream stream) {
+  if (format != DS4A_MX_KV_FP8 && format != DS4A_MX_IDX_FP4) return DS4A_EINVAL;
+  return compress_append_common(cfg, B, c, pos, ca, cb, za, zb, bias_a, bias_b, norm_g, state, N_cap, nullptr, 0,
+                                format == DS4A_MX_KV_FP8 ? 1 : 2, pool, scales, pool_bstride, stream);
+}
+
+size_t ds4a_kv_fp8_row_bytes(int D, int R) {
+  if (D <= 0 || R < 0 || R > D || (D - R) % kMxBlockApi != 0 || (R % 8) != 0) return 0;
+  return (size_t)kv_fp8_row_bytes(D, R);
+}
+
+int ds4a_quantize_kv_fp8(int n_rows, int D, int R, const ds4a_bf16* in, int64_t in_stride, uint8_t* out,
+                         int64_t out_stride, ds4a_stream stream) {
+  if (n_rows < 0 || ds4a_kv_fp8_row_bytes(D, R) == 0) return DS4A_EINVAL;
+  if (n_rows == 0) return DS4A_OK;
+  if (!in || !out || !aligned16(in) || !aligned16(out)) return DS4A_EINVAL;
+  if (in_stride < D || in_stride % 8 != 0 || out_stride < kv_fp8_row_bytes(D, R) || out_stride % 16 != 0)
+    return DS4A_EINVAL;
+  return cuda_rc(launch_quant_kv_fp8(n_rows, D, R, in, in_stride, out, out_stride, (cudaStream_t)stream));
+}
+
+int ds4a_quantize_idx_fp4(int n_rows, int D, const ds4a_bf16* in, int64_t in_stride, uint8_t* codes,
+                          uint8_t* scales, ds4a_stream stream) {
+  if (n_rows < 0 || D <= 0 || D % kMxBlockApi != 0) return DS4A_EINVAL;
+  if (n_rows == 0) return DS4A_OK;
+  if (!in || !codes || !scales || !aligned16(in) || !aligned16(codes)) return DS4A_EINVAL;
+  if (in_stride < D || in_stride % 8 != 0) return DS4A_EINVAL;
+  return cuda_rc(launch_quant_idx_fp4(n_rows, D, in, in_stride, codes, scales, (cudaStream_t)stream));
 }
 
 size_t ds4a_index_topk_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c) {
@@ -232,6 +293,7 @@ int ds4a_index_topk(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_
   a.B = B; a.T_q = T_q; a.H = cfg->idx_heads; a.D = cfg->idx_dim; a.m = cfg->ratio;
   a.k = cfg->topk; a.N_c = N_c;
   a.q_pos = q_pos; a.q = q_idx; a.w = w_idx; a.kidx = k_idx; a.k_bstride = k_bstride;
+  a.kcodes = nullptr; a.kscales = nullptr;
   a.scores = reinterpret_cast<float*>(ws);
   a.idx_out = idx_out; a.score_out = score_out;
   a.err = err_word();
@@ -242,6 +304,37 @@ int ds4a_index_topk(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_
     e = index_scores_tc_supported(a) ? launch_index_scores_tc(a, s) : launch_index_scores_generic(a, s);
     if (e != cudaSuccess) return DS4A_ECUDA;
   }
+  return cuda_rc(launch_topk(a, s));
+}
+
+int ds4a_index_topk_fp4(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                        const ds4a_bf16* q_idx, const ds4a_bf16* w_idx, const uint8_t* k_codes,
+                        const uint8_t* k_scales, int64_t k_bstride, int N_c, int32_t* idx_out,
+                        float* score_out, void* ws, size_t ws_bytes, ds4a_stream stream) {
+  if (check_index_cfg(cfg) != DS4A_OK) return DS4A_EINVAL;
+  if (B < 0 || T_q < 0 || N_c < 0) return DS4A_EINVAL;
+  if (B == 0 || T_q == 0) return DS4A_OK;
+  if (!q_pos || !q_idx || !w_idx || !idx_out) return DS4A_EINVAL;
+  if (N_c > 0 && (!k_codes || !k_scales || !ws)) return DS4A_EINVAL;
+  if (!aligned16(q_pos) || !aligned16(q_idx) || !aligned16(w_idx) || !aligned16(idx_out)) return DS4A_EINVAL;
+  if ((k_codes && !aligned16(k_codes)) || (k_scales && !aligned16(k_scales)) ||
+      (score_out && !aligned16(score_out)) || (ws && !aligned16(ws)))
+    return DS4A_EINVAL;
+  if (N_c > 0 && k_bstride < N_c) return DS4A_EINVAL;
+  if (ws_bytes < index_ws_bytes(B, T_q, N_c)) return DS4A_ENOSPACE;
+  IndexArgs a;
+  a.B = B; a.T_q = T_q; a.H = cfg->idx_heads; a.D = cfg->idx_dim; a.m = cfg->ratio;
+  a.k = cfg->topk; a.N_c = N_c;
+  a.q_pos = q_pos; a.q = q_idx; a.w = w_idx; a.kidx = nullptr; a.k_bstride = k_bstride;
+  a.kcodes = k_codes; a.kscales = k_scales;
+  a.scores = reinterpret_cast<float*>(ws);
+  a.idx_out = idx_out; a.score_out = score_out;
+  // the tensor-core scorer with its FP4 converters is the only FP4 path
+  if (N_c > 0 && !index_scores_tc_supported(a)) return DS4A_EUNSUPPORTED;
+  a.err = err_word();
+  if (!a.err) return DS4A_ECUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (N_c > 0 && launch_index_scores_tc(a, s) != cudaSuccess) return DS4A_ECUDA;
   return cuda_rc(launch_topk(a, s));
 }
 
@@ -260,7 +353,16 @@ static int attend_common(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_
                          const ds4a_bf16* q, const float* q_norm_g, const ds4a_bf16* pool,
                          int64_t pool_bstride, int N_c, const int32_t* idx, const ds4a_bf16* win,
                          int win_cap, int64_t win_bstride, const float* sink, ds4a_bf16* out,
-                         void* ws, size_t ws_bytes, ds4a_stream stream, int sparse) {
+                         void* ws, size_t ws_bytes, ds4a_stream stream, int sparse,
+                         const uint8_t* pool8 = nullptr) {
+  const int64_t bstride8 = pool_bstride;  // rows, for FP8 pools
+  if (pool8) {
+    // mixed FP8 / BF16 rows: the tensor-core path of the Flash shape only
+    if (!cfg || cfg->n_heads != 64 || cfg->head_dim != 512 || cfg->rope_dim != 64) return DS4A_EUNSUPPORTED;
+    if (!aligned16(pool8) || (N_c > 0 && pool_bstride < N_c)) return DS4A_EINVAL;
+    pool = reinterpret_cast<const ds4a_bf16*>(pool8);  // for the checks below
+    pool_bstride = (int64_t)N_c * cfg->head_dim;
+  }
   if (check_cfg(cfg) != DS4A_OK) return DS4A_EINVAL;
   if (sparse && (cfg->topk < 1 || cfg->topk > 4096)) return DS4A_EINVAL;
   if (B < 0 || T_q < 0 || N_c < 0) return DS4A_EINVAL;
@@ -286,6 +388,8 @@ static int attend_common(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_
   a.m = cfg->ratio; a.k = cfg->topk; a.N_c = N_c; a.win_cap = win_cap; a.sparse = sparse;
   a.scale = cfg->sm_scale; a.rope_base = cfg->rope_base; a.eps = cfg->rms_eps;
   a.q_pos = q_pos; a.q = q; a.q_norm_g = q_norm_g; a.pool = pool; a.pool_bstride = pool_bstride;
+  a.pool8 = pool8;
+  if (pool8) a.pool_bstride = bstride8;
   a.idx = idx; a.win = win; a.win_bstride = win_bstride; a.sink = sink; a.out = out;
   a.ws = reinterpret_cast<float*>(ws);
   a.keys_max = (sparse ? cfg->topk : N_c) + cfg->window;
@@ -365,6 +469,26 @@ int ds4a_out_proj(const ds4a_oproj_cfg* cfg, int M, const ds4a_bf16* o, const ds
   // y[t][n] = W_b[n] . mid[t]
   e = launch_gemm(mid, n1, n1, w_b, M, cfg->hidden, n1, cfg->hidden, 0, y, cfg->hidden, acc, err, s);
   return cuda_rc(e);
+}
+
+int ds4a_sparse_attend_fp8(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                           const ds4a_bf16* q, const float* q_norm_g, const uint8_t* pool,
+                           int64_t pool_bstride, int N_c, const int32_t* idx, const ds4a_bf16* win,
+                           int win_cap, int64_t win_bstride, const float* sink, ds4a_bf16* out,
+                           void* ws, size_t ws_bytes, ds4a_stream stream) {
+  if (N_c > 0 && !pool) return DS4A_EINVAL;
+  return attend_common(cfg, B, T_q, q_pos, q, q_norm_g, nullptr, pool_bstride, N_c, idx, win, win_cap,
+                       win_bstride, sink, out, ws, ws_bytes, stream, 1, N_c > 0 ? pool : nullptr);
+}
+
+int ds4a_hca_attend_fp8(const ds4a_layer_cfg* cfg, int B, int T_q, const int32_t* q_pos,
+                        const ds4a_bf16* q, const float* q_norm_g, const uint8_t* pool,
+                        int64_t pool_bstride, int N_c, const ds4a_bf16* win, int win_cap,
+                        int64_t win_bstride, const float* sink, ds4a_bf16* out, void* ws,
+                        size_t ws_bytes, ds4a_stream stream) {
+  if (N_c > 0 && !pool) return DS4A_EINVAL;
+  return attend_common(cfg, B, T_q, q_pos, q, q_norm_g, nullptr, pool_bstride, N_c, nullptr, win, win_cap,
+                       win_bstride, sink, out, ws, ws_bytes, stream, 0, N_c > 0 ? pool : nullptr);
 }
 
 int ds4a_check(ds4a_stream stream, uint32_t* bits_out) {

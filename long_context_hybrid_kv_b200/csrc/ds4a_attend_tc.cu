@@ -32,6 +32,7 @@
 // Work items are (query, key split) pairs taken round-robin by the blocks;
 // with one split the block writes the final bf16 output, otherwise the
 // float partials (max, sum, accumulator) the combine kernel merges.
+#include "ds4a_mx.cuh"
 #include "ds4a_tc.cuh"
 
 namespace ds4a {
@@ -65,7 +66,15 @@ constexpr uint32_t kOffInv = kOffAlpha + 256;       // [64]
 constexpr uint32_t kOffSink = kOffInv + 256;        // [64] sink * log2(e)
 constexpr uint32_t kOffNext = kOffSink + 256;       // the softmax warps' next work item
 constexpr uint32_t kOffValid = kOffNext + 64;       // [2 tiles][128 keys] validity flags
-constexpr uint32_t kSmemBytes = kOffValid + 256 + 1024;  // + alignment slack
+// FP8 pools: codes of dims 384..447 staged per row, each row's 16-byte
+// scale run, and the E4M3 value of every code
+constexpr uint32_t kOffStage3 = kOffValid + 256;    // [128 keys][64 B]
+constexpr uint32_t kOffScale = kOffStage3 + 8192;   // [128 keys][16 B]
+constexpr uint32_t kOffLut8 = kOffScale + 2048;     // [256] floats
+constexpr uint32_t kSmemBytes = kOffValid + 256 + 1024;   // bf16 pools (+ alignment slack)
+constexpr uint32_t kSmemBytes8 = kOffLut8 + 1024 + 1024;  // FP8 pools
+constexpr int kRow8 = 592;                          // bytes of a mixed FP8 / BF16 row (D 512, R 64)
+constexpr int kNope8 = 448;                         // FP8 dims of a row
 
 enum Bar {
   kQFull = 0, kQEmpty, kKVFull0, kKVFull1, kKVFull2, kKVFull3, kKVEmpty0, kKVEmpty1, kKVEmpty2,
@@ -136,6 +145,7 @@ __device__ __forceinline__ Item make_item(const AttendArgs& a, int w) {
 }
 
 // row pointer of key j of an item, or nullptr (out of range / bad index)
+template <bool kFp8>
 __device__ __forceinline__ const uint16_t* key_ptr(const AttendArgs& a, const Item& it, int j,
                                                    bool* bad) {
   *bad = false;
@@ -146,6 +156,8 @@ __device__ __forceinline__ const uint16_t* key_ptr(const AttendArgs& a, const It
       *bad = true;
       return nullptr;
     }
+    if (kFp8)  // a mixed FP8 / BF16 row, addressed in bytes
+      return reinterpret_cast<const uint16_t*>(a.pool8 + ((int64_t)it.b * a.pool_bstride + e) * kRow8);
     return a.pool + (int64_t)it.b * a.pool_bstride + (int64_t)e * kD;
   }
   const int p = it.win_start + (j - it.n_sel);
@@ -166,7 +178,7 @@ struct DenseKV {
   int64_t pool_rows_b;
 };
 
-template <bool kCompact>
+template <bool kCompact, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap kvmap, DenseKV dkv, AttendArgs a, int n_items,
                      const uint8_t* qimg) {
@@ -596,6 +608,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pt = tid - kPG0;  // 0..127
     uint32_t gt = 0, active = 0;
     bool tma_used = false;
+    if (kFp8) {
+      float* lut = reinterpret_cast<float*>(smem + kOffLut8);
+      for (int c = pt; c < 256; c += 128) lut[c] = e4m3_value((uint32_t)c);
+      named_bar(2, 128);
+    }
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       const Item it = make_item(a, w);
       if (it.n_tiles == 0) continue;
@@ -604,11 +621,85 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto set_rowptr = [&](int tile) {
         named_bar(2, 128);
         bool bad = false;
-        const uint16_t* p = key_ptr(a, it, it.j0 + tile * kKT + pt, &bad);
+        const int j = it.j0 + tile * kKT + pt;
+        const uint16_t* p = key_ptr<kFp8>(a, it, j, &bad);
         if (bad) raise_err(err, DS4A_DEV_BAD_INDEX);
         rowptr[pt] = p;
-        vflag[(gt & 1u) * kKT + pt] = p != nullptr;
+        // 0: no row (zero-filled); 1: bf16 row; 2: FP8 pool row
+        vflag[(gt & 1u) * kKT + pt] = p == nullptr ? 0 : (kFp8 && j < it.n_sel ? 2 : 1);
         named_bar(2, 128);
+      };
+      // FP8 pools: chunk c of the tile.  bf16 rows (the window) and missing
+      // rows go as in issue_chunk; an FP8 row's codes of dims 128c .. 128c+127
+      // land in the row's own 128 bytes of block 2c+1 (chunks 0-2) or in the
+      // stage-3 area (chunk 3: dims 384..447), its RoPE dims 448..511 straight
+      // into block 7, its 16-byte scale run (chunk 0) in the scale area
+      auto issue_chunk8 = [&](int c) {
+        if (gt > 0) mbar_wait(bar(kKVEmpty0 + c), (gt - 1) & 1u, abort_flag, err);
+        const uint32_t blk = kv_base + (uint32_t)(2 * c + (piece >> 3)) * 16384u;
+        for (int i = 0; i < 16; ++i) {
+          const int row = (pt >> 4) + 8 * i;
+          const uint16_t* src = rowptr[row];
+          const uint8_t vf = vflag[(gt & 1u) * kKT + row];
+          const uint32_t dst = blk + sw128(row, piece & 7);
+          if (vf == 1) {
+            cp_async16(dst, src + c * 128 + piece * 8);
+          } else if (vf == 0) {
+            st_shared_zero16(dst);
+          } else {
+            const uint8_t* r8 = reinterpret_cast<const uint8_t*>(src);
+            if (c < 3) {
+              if (piece < 8)
+                cp_async16(kv_base + (uint32_t)(2 * c + 1) * 16384u + row * 128u + piece * 16u, r8 + c * 128 + piece * 16);
+            } else if (piece < 4) {
+              cp_async16(sbase + kOffStage3 + row * 64u + piece * 16u, r8 + 384 + piece * 16);
+            } else if (piece >= 8) {
+              cp_async16(dst, r8 + kNope8 + (piece - 8) * 16);  // RoPE dims, bf16
+            }
+            if (c == 0 && piece == 15) cp_async16(sbase + kOffScale + row * 16u, r8 + kNope8 + 128);
+          }
+        }
+        cp_async_commit();
+      };
+      // every producer's copies of chunk c have landed: thread pt expands its
+      // own FP8 row to bf16 (code value times the block's scale, exact)
+      auto convert_chunk8 = [&](int c) {
+        named_bar(2, 128);
+        if (vflag[(gt & 1u) * kKT + pt] != 2) return;
+        const float* lut = reinterpret_cast<const float*>(smem + kOffLut8);
+        const unsigned char* stg = c < 3 ? smem + kOffKV + (2 * c + 1) * 16384 + pt * 128 : smem + kOffStage3 + pt * 64;
+        const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(smem + kOffScale + pt * 16 + 4 * c);
+        // 16 codes = dims 128c + 16q .. + 15 (one scale block per two q) ->
+        // the 8-dim pieces 2q, 2q + 1 of the chunk
+        auto expand = [&](int q, const uint4 cw) {
+          const float sc = mx_scale((int)((sc4 >> (8 * (q >> 1))) & 255u));
+          const uint32_t wd[4] = {cw.x, cw.y, cw.z, cw.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t w = wd[k >> 1] >> (16 * (k & 1));
+            o[k] = f2_to_bf2x2(lut[w & 255u] * sc, lut[(w >> 8) & 255u] * sc);
+          }
+          const int p0 = 2 * q;
+          const uint32_t b0 = kv_base + (uint32_t)(2 * c + (p0 >> 3)) * 16384u;
+          st_shared16(b0 + sw128(pt, p0 & 7), o[0], o[1], o[2], o[3]);
+          st_shared16(b0 + sw128(pt, (p0 + 1) & 7), o[4], o[5], o[6], o[7]);
+        };
+        if (c == 3) {  // dims 384..447 from the stage-3 area into block 6
+#pragma unroll 1
+          for (int q = 0; q < 4; ++q) expand(q, reinterpret_cast<const uint4*>(stg)[q]);
+          return;
+        }
+        // the row's staged codes sit in its own bytes of block 2c+1: the
+        // upper half (q = 4..7, written into block 2c+1) is read first, the
+        // lower half is expanded into block 2c, then the upper half
+        uint4 hi[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) hi[q] = reinterpret_cast<const uint4*>(stg)[4 + q];
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) expand(q, reinterpret_cast<const uint4*>(stg)[q]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) expand(4 + q, hi[q]);
       };
       // one 128-dim chunk of the tile: 128 rows x 256 B, 16 cp.async each;
       // rows past the key list or with a bad index are zero-filled
@@ -659,6 +750,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           continue;
         }
         set_rowptr(tile);
+        if (kFp8) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            issue_chunk8(c);
+            if (c > 0) {
+              cp_async_wait<1>();
+              convert_chunk8(c - 1);
+              fence_async_smem();
+              mbar_arrive(bar(kKVFull0 + c - 1));
+            }
+          }
+          cp_async_wait<0>();
+          convert_chunk8(3);
+          fence_async_smem();
+          mbar_arrive(bar(kKVFull0 + 3));
+          continue;
+        }
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           issue_chunk(c);
@@ -793,9 +901,12 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   a.ws = reinterpret_cast<float*>(qimg + (size_t)rows * 65536u);
   const int n_items = rows * a.n_splits;
   const bool compact = n_items <= 148;  // every block takes at most one item
-  static std::atomic<int> cache[kMaxDevices], cache_c[kMaxDevices];
-  cudaError_t e = compact ? ensure_smem(attend_tc_kernel<true>, (int)kSmemBytes, cache_c)
-                          : ensure_smem(attend_tc_kernel<false>, (int)kSmemBytes, cache);
+  static std::atomic<int> cache[kMaxDevices], cache_c[kMaxDevices], cache8[kMaxDevices], cache8c[kMaxDevices];
+  const bool fp8 = a.pool8 != nullptr;
+  cudaError_t e = fp8 ? (compact ? ensure_smem(attend_tc_kernel<true, true>, (int)kSmemBytes8, cache8c)
+                                 : ensure_smem(attend_tc_kernel<false, true>, (int)kSmemBytes8, cache8))
+                      : (compact ? ensure_smem(attend_tc_kernel<true, false>, (int)kSmemBytes, cache_c)
+                                 : ensure_smem(attend_tc_kernel<false, false>, (int)kSmemBytes, cache));
   if (e != cudaSuccess) return e;
   if (!compact) {
     // decode-sized launches prepare q^ inside the attention kernel
@@ -813,7 +924,7 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   dkv.dense = 0;
   dkv.pool_rows_b = a.B > 1 ? a.pool_bstride / kD : 0;
   const int64_t pool_rows = (int64_t)(a.B - 1) * dkv.pool_rows_b + a.N_c;
-  if (!a.sparse && a.N_c >= kKT && (a.B == 1 || a.pool_bstride % kD == 0) && pool_rows < INT32_MAX) {
+  if (!a.pool8 && !a.sparse && a.N_c >= kKT && (a.B == 1 || a.pool_bstride % kD == 0) && pool_rows < INT32_MAX) {
     const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)pool_rows};
     const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)kKT};
@@ -828,10 +939,16 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   {
     TraceScope tr("attend_tc", s);
     const uint8_t* qi = qimg;
-    e = compact ? launch_pdl(attend_tc_kernel<true>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap,
-                             dkv, a, n_items, qi)
-                : launch_pdl(attend_tc_kernel<false>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap,
-                             dkv, a, n_items, qi);
+    if (fp8)
+      e = compact ? launch_pdl(attend_tc_kernel<true, true>, dim3(grid), dim3(kThreads), kSmemBytes8, s, kvmap, dkv,
+                               a, n_items, qi)
+                  : launch_pdl(attend_tc_kernel<false, true>, dim3(grid), dim3(kThreads), kSmemBytes8, s, kvmap, dkv,
+                               a, n_items, qi);
+    else
+      e = compact ? launch_pdl(attend_tc_kernel<true, false>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap, dkv,
+                               a, n_items, qi)
+                  : launch_pdl(attend_tc_kernel<false, false>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap,
+                               dkv, a, n_items, qi);
   }
   if (e != cudaSuccess || a.n_splits == 1) return e;
   return launch_attend_combine(a, s);

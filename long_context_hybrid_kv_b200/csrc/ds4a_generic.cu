@@ -5,6 +5,7 @@
 // take the tensor-core kernels of ds4a_index_tc.cu / ds4a_attend_tc.cu
 // where those apply.
 #include "ds4a_internal.cuh"
+#include "ds4a_mx.cuh"
 
 #include <cooperative_groups.h>
 #include <float.h>
@@ -109,6 +110,45 @@ __device__ __forceinline__ int append_token(const CompressArgs& a, int b, int ti
   return i;
 }
 
+// Store channels (ch, ch + 1) of entry i of sequence b: as bf16 at dst, or
+// (qfmt != 0) rounded to bf16 and then block-quantised (ds4a_mx.cuh).  In
+// the block-scaled case every lane of the warp calls it, the warp holding 64
+// consecutive channels that start at a multiple of 64 (two 32-channel
+// blocks, one per half-warp).
+__device__ __forceinline__ void store_entry_pair(const CompressArgs& a, int b, int i, int ch, float x0, float x1,
+                                                 uint16_t* dst) {
+  const unsigned int packed = f2_to_bf2x2(x0, x1);
+  if (a.qfmt == 0) {
+    *reinterpret_cast<unsigned int*>(dst) = packed;
+    return;
+  }
+  const float2 v = bf2x2_to_f2(packed);
+  float amax = fmaxf(fabsf(v.x), fabsf(v.y));
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const bool lead = (threadIdx.x & 15) == 0;
+  if (a.qfmt == 1) {
+    uint8_t* row = a.qpool + (int64_t)b * a.q_bstride + (int64_t)i * a.q_row;
+    const int R = a.rope_dim, n = a.c - R;
+    if (ch >= n) {  // RoPE dims stay bf16
+      *reinterpret_cast<unsigned int*>(row + n + 2 * (ch - n)) = packed;
+      return;
+    }
+    const int code = mx_scale_code<false>(amax);
+    const float inv = mx_inv_scale(code);
+    *reinterpret_cast<uint16_t*>(row + ch) = to_e4m3x2(v.x * inv, v.y * inv);
+    if (lead) row[n + 2 * R + ch / kMxBlock] = (uint8_t)code;
+    if (ch == 0)
+      for (int k = n + 2 * R + n / kMxBlock; k < (int)a.q_row; ++k) row[k] = 0;
+  } else {
+    uint8_t* row = a.qpool + (int64_t)b * a.q_bstride + (int64_t)i * (a.c / 2);
+    const int code = mx_scale_code<true>(amax);
+    const float inv = mx_inv_scale(code);
+    row[ch / 2] = (uint8_t)to_e2m1x2(v.x * inv, v.y * inv);
+    if (lead) a.qscales[(int64_t)b * a.qs_bstride + (int64_t)i * (a.c / kMxBlock) + ch / kMxBlock] = (uint8_t)code;
+  }
+}
+
 template <int V>
 __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs a) {
   extern __shared__ float csm[];
@@ -207,9 +247,14 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
     ss += v * v;
   }
   pdl_wait();
-  uint16_t* dst = a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c;
+  uint16_t* dst = a.qfmt ? nullptr : a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c;
   if (a.norm_g == nullptr) {
     __syncthreads();
+    if (a.qfmt) {
+      for (int p2 = tid; p2 < c / 2; p2 += kCompressThreads)
+        store_entry_pair(a, b, i, 2 * p2, s_v[2 * p2], s_v[2 * p2 + 1], nullptr);
+      return;
+    }
     for (int ch = tid; ch < c; ch += kCompressThreads) dst[ch] = f2bf(s_v[ch]);
     return;
   }
@@ -234,7 +279,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
       x0 = y0;
       x1 = y1;
     }
-    *reinterpret_cast<unsigned int*>(dst + ch) = f2_to_bf2x2(x0, x1);
+    store_entry_pair(a, b, i, ch, x0, x1, dst + ch);
   }
 }
 
@@ -372,9 +417,14 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
     ss += v * v;
   }
   pdl_wait();
-  uint16_t* dst = a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c + ch0;
+  uint16_t* dst = a.qfmt ? nullptr : a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c + ch0;
   if (a.norm_g == nullptr) {
     cl.sync();  // no block leaves while a peer may still read its partials
+    if (a.qfmt) {
+      for (int p2 = tid; p2 < cz / 2; p2 += kCompressThreads)
+        store_entry_pair(a, b, i, ch0 + 2 * p2, s_v[2 * p2], s_v[2 * p2 + 1], nullptr);
+      return;
+    }
     for (int k = tid; k < cz; k += kCompressThreads) dst[k] = f2bf(s_v[k]);
     return;
   }
@@ -405,7 +455,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
       x0 = y0;
       x1 = y1;
     }
-    *reinterpret_cast<unsigned int*>(dst + k) = f2_to_bf2x2(x0, x1);
+    store_entry_pair(a, b, i, ch, x0, x1, dst + k);
   }
 }
 

@@ -20,9 +20,16 @@
 //              warps per SM sub-partition hide each other's latencies.
 // Work: (query group, chunk of key tiles) pairs, taken round-robin by the
 // blocks; pairs past a group's visible entries are skipped.
+// FP4 keys (E2M1 codes and E8M0 scales per 32 dims): a bulk copy brings a
+// tile's packed codes and scales into a raw ring; four more warps (10-13)
+// expand them exactly into the same bf16 tile (a 256-entry table maps a code
+// byte to its two values, times the block's power-of-two scale), and the
+// products and the epilogue are unchanged.  Three stages instead of four
+// make room for the raw ring.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "ds4a_mx.cuh"
 #include "ds4a_tc.cuh"
 
 namespace ds4a {
@@ -41,15 +48,29 @@ constexpr int kEpiThreads = 256;
 constexpr int kRegBoundThreads = 384;
 constexpr int kMaxG = 4;
 
-constexpr uint32_t kOffK = 0;                       // kStages x 2 blocks x 16 KB
-constexpr uint32_t kOffQ = kStages * 32768;         // 2 blocks x (G*64 rows x 128 B)
-constexpr uint32_t kOffW = kOffQ + 2 * kMaxG * 8192;  // [G*64] floats
-constexpr uint32_t kOffBar = kOffW + kMaxG * kHI * 4;
-constexpr uint32_t kOffMisc = kOffBar + 256;
-constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+constexpr int kStagesFp4 = 3;
+constexpr int kConvThreads = 128;
+constexpr uint32_t kRawCodes = kKT * kDI / 2;  // 8 KiB of E2M1 codes per tile
+constexpr uint32_t kRawStage = kRawCodes + kKT * (kDI / kMxBlock);  // + 512 B of scales
 
-enum Bar { kKFull = 0, kKEmpty = kKFull + kStages, kQFull = kKEmpty + kStages, kQEmpty, kAccFull0,
-           kAccFull1, kAccEmpty0, kAccEmpty1, kDrain, kNumBars };
+// shared memory map (offsets from a 1024-aligned base) of either variant
+template <bool kFp4>
+struct Layout {
+  static constexpr int stages = kFp4 ? kStagesFp4 : kStages;
+  static constexpr uint32_t k = 0;                                  // stages x 2 blocks x 16 KB
+  static constexpr uint32_t raw = stages * 32768;                   // FP4: stages x kRawStage
+  static constexpr uint32_t q = (raw + (kFp4 ? stages * kRawStage : 0) + 1023) / 1024 * 1024;
+  static constexpr uint32_t w = q + 2 * kMaxG * 8192;               // [G*64] floats
+  static constexpr uint32_t lut = w + kMaxG * kHI * 4;              // FP4: 256 float2
+  static constexpr uint32_t bar = lut + (kFp4 ? 2048 : 0);
+  static constexpr uint32_t misc = bar + 256;
+  static constexpr uint32_t bytes = misc + 64 + 1024;
+  static constexpr int threads = kFp4 ? kThreads + kConvThreads : kThreads;
+};
+
+// barrier slots (FP4 adds the raw ring's full / empty barriers)
+constexpr int kKFull = 0, kKEmpty = 4, kQFull = 8, kQEmpty = 9, kAccFull0 = 10, kAccFull1 = 11,
+              kAccEmpty0 = 12, kAccEmpty1 = 13, kDrain = 14, kRawFull = 15, kRawEmpty = 19;
 
 struct TcIndexParams {
   IndexArgs a;
@@ -89,19 +110,22 @@ __device__ __forceinline__ Pair make_pair(const TcIndexParams& p, int w) {
   return q;
 }
 
-__global__ void __launch_bounds__(kRegBoundThreads, 1)
+template <bool kFp4>
+__global__ void __launch_bounds__(kFp4 ? 512 : kRegBoundThreads, 1)
     index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                     const TcIndexParams p) {
+  using Lay = Layout<kFp4>;
+  constexpr int kS = Lay::stages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t k_base = sbase + kOffK, q_base = sbase + kOffQ;
-  float* w_s = reinterpret_cast<float*>(smem + kOffW);
-  const uint32_t bar0 = sbase + kOffBar;
+  const uint32_t k_base = sbase + Lay::k, q_base = sbase + Lay::q;
+  float* w_s = reinterpret_cast<float*>(smem + Lay::w);
+  const uint32_t bar0 = sbase + Lay::bar;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::misc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::misc + 8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.G;
   const IndexArgs& a = p.a;
@@ -111,9 +135,13 @@ __global__ void __launch_bounds__(kRegBoundThreads, 1)
 
   if (tid == 0) {
     *abort_flag = 0;
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kKFull + s), 1);
+    for (int s = 0; s < kS; ++s) {
+      mbar_init(bar(kKFull + s), kFp4 ? kConvThreads : 1);
       mbar_init(bar(kKEmpty + s), 1);
+      if (kFp4) {
+        mbar_init(bar(kRawFull + s), 1);
+        mbar_init(bar(kRawEmpty + s), kConvThreads);
+      }
     }
     mbar_init(bar(kQFull), 1);
     mbar_init(bar(kQEmpty), 1);
@@ -165,15 +193,32 @@ __global__ void __launch_bounds__(kRegBoundThreads, 1)
           load_q(q);
         }
         for (int tile = q.tile0; tile < q.tile1; ++tile, ++kt) {
-          const uint32_t s = kt % kStages;
-          if (kt >= (uint32_t)kStages)
-            mbar_wait(bar(kKEmpty + s), ((kt / kStages) - 1) & 1u, abort_flag, err);
+          const uint32_t s = kt % kS;
+          if (kFp4) {
+            // the tile's packed codes and scales (rows past N_c are not read)
+            if (kt >= (uint32_t)kS) mbar_wait(bar(kRawEmpty + s), ((kt / kS) - 1) & 1u, abort_flag, err);
+            const int rows = min(kKT, a.N_c - tile * kKT);
+            const int64_t key0 = (int64_t)q.b * a.k_bstride + (int64_t)tile * kKT;
+            const uint32_t raw = sbase + Lay::raw + s * kRawStage;
+            mbar_expect_tx(bar(kRawFull + s), (uint32_t)rows * (kDI / 2 + kDI / kMxBlock));
+            bulk_g2s(raw, a.kcodes + key0 * (kDI / 2), (uint32_t)rows * (kDI / 2), bar(kRawFull + s));
+            bulk_g2s(raw + kRawCodes, a.kscales + key0 * (kDI / kMxBlock), (uint32_t)rows * (kDI / kMxBlock),
+                     bar(kRawFull + s));
+            continue;
+          }
+          if (kt >= (uint32_t)kS)
+            mbar_wait(bar(kKEmpty + s), ((kt / kS) - 1) & 1u, abort_flag, err);
           mbar_expect_tx(bar(kKFull + s), 32768u);
           const uint32_t dst = k_base + s * 32768u;
           tma_load_3d(dst, &kmap, 0, tile * kKT, q.b, bar(kKFull + s));
           tma_load_3d(dst + 16384u, &kmap, 64, tile * kKT, q.b, bar(kKFull + s));
         }
         ++active;
+      }
+      if (kFp4) {
+        // no bulk copy into this block's shared memory is left in flight
+        for (uint32_t j = kt > (uint32_t)kS ? kt - kS : 0; j < kt; ++j)
+          mbar_drain(bar(kRawFull + j % kS), (j / kS) & 1u);
       }
     }
     if (lane != 0) pdl_wait();
@@ -192,9 +237,9 @@ __global__ void __launch_bounds__(kRegBoundThreads, 1)
         mbar_wait(bar(kQFull), active & 1u, abort_flag, err);
         tc_fence_after();
         for (int tile = q.tile0; tile < q.tile1; ++tile, ++kt, ++at) {
-          const uint32_t s = kt % kStages;
+          const uint32_t s = kt % kS;
           const uint32_t ab = at & 1u;
-          mbar_wait(bar(kKFull + s), (kt / kStages) & 1u, abort_flag, err);
+          mbar_wait(bar(kKFull + s), (kt / kS) & 1u, abort_flag, err);
           if (at >= 2) mbar_wait(bar(kAccEmpty0 + ab), ((at >> 1) - 1) & 1u, abort_flag, err);
           tc_fence_after();
           const uint64_t a0 = k_desc0 + ((s * 32768u) >> 4);
@@ -215,6 +260,55 @@ __global__ void __launch_bounds__(kRegBoundThreads, 1)
       mbar_wait(bar(kDrain), 0, abort_flag, err);
     }
     __syncwarp();
+  } else if (kFp4 && warp >= 10) {
+    // =================== FP4 -> bf16 converters ===================
+    const int r = tid - kThreads;  // key row of the tile
+    float2* lut = reinterpret_cast<float2*>(smem + Lay::lut);
+    for (int c = r; c < 256; c += kConvThreads) lut[c] = make_float2(e2m1_value(c & 15u), e2m1_value(c >> 4));
+    named_bar(2, kConvThreads);
+    uint32_t kt = 0;
+    for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
+      const Pair q = make_pair(p, w);
+      for (int tile = q.tile0; tile < q.tile1; ++tile, ++kt) {
+        const uint32_t s = kt % kS;
+        mbar_wait(bar(kRawFull + s), (kt / kS) & 1u, abort_flag, err);
+        const unsigned char* raw = smem + Lay::raw + s * kRawStage;
+        const bool live = tile * kKT + r < a.N_c;
+        uint4 cw[4];
+        uint32_t sc4 = 0;
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cw[i] = reinterpret_cast<const uint4*>(raw + r * (kDI / 2))[i];
+          sc4 = *reinterpret_cast<const uint32_t*>(raw + kRawCodes + r * (kDI / kMxBlock));
+        }
+        mbar_arrive(bar(kRawEmpty + s));  // the raw slot may refill
+        if (kt >= (uint32_t)kS) mbar_wait(bar(kKEmpty + s), ((kt / kS) - 1) & 1u, abort_flag, err);
+        const uint32_t dst = k_base + s * 32768u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // 32 dims = one scale block
+          const float sc = mx_scale((int)((sc4 >> (8 * i)) & 255u));
+          const uint32_t words[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {  // 8 code bytes = 16 dims = two 16-byte pieces
+            uint32_t o[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t byte = (words[2 * h + (k >> 2)] >> (8 * (k & 3))) & 255u;
+              const float2 v = lut[byte];
+              o[k] = live ? f2_to_bf2x2(v.x * sc, v.y * sc) : 0u;
+            }
+            // dims 32 i + 16 h .. + 15: block (i >> 1), 16-byte chunks
+            const int d0 = 32 * i + 16 * h;
+            const uint32_t blk = dst + (uint32_t)(d0 >> 6) * 16384u;
+            const uint32_t c0 = (uint32_t)((d0 & 63) >> 3);
+            st_shared16(blk + sw128((uint32_t)r, c0), o[0], o[1], o[2], o[3]);
+            st_shared16(blk + sw128((uint32_t)r, c0 + 1), o[4], o[5], o[6], o[7]);
+          }
+        }
+        fence_async_smem();
+        mbar_arrive(bar(kKFull + s));
+      }
+    }
   } else {
     // =================== epilogue ===================
     const int et = tid - 64;                 // 0..255
@@ -316,6 +410,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 bool index_scores_tc_supported(const IndexArgs& a) {
   // Flash indexer width; the batch stride of the key pool must be a multiple
   // of 16 bytes for the tensor map
+  if (a.kcodes)  // FP4 keys: whole 16-byte runs of scales per 4 keys
+    return a.H == kHI && a.D == kDI && (a.k_bstride % 4) == 0 && (a.N_c % 4) == 0;
   return a.H == kHI && a.D == kDI && (a.k_bstride % 8) == 0 && a.N_c >= kKT && get_encode() != nullptr;
 }
 
@@ -339,7 +435,9 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s) {
   p.n_pairs = p.n_groups * p.chunks_per_group;
 
   CUtensorMap kmap, qmap;
-  {
+  memset(&kmap, 0, sizeof(kmap));
+  const bool fp4 = a.kcodes != nullptr;
+  if (!fp4) {
     const cuuint64_t dims[3] = {(cuuint64_t)kDI, (cuuint64_t)a.N_c, (cuuint64_t)a.B};
     const cuuint64_t strides[2] = {(cuuint64_t)kDI * 2, (cuuint64_t)a.k_bstride * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)kKT, 1};
@@ -359,12 +457,20 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  static std::atomic<int> cache[kMaxDevices];
-  cudaError_t e = ensure_smem(index_tc_kernel, (int)kSmemBytes, cache);
-  if (e != cudaSuccess) return e;
+  static std::atomic<int> cache[kMaxDevices], cache4[kMaxDevices];
   const int grid = min(p.n_pairs, 148);
+  if (fp4) {
+    cudaError_t e = ensure_smem(index_tc_kernel<true>, (int)Layout<true>::bytes, cache4);
+    if (e != cudaSuccess) return e;
+    TraceScope tr("index_score_tc_fp4", s);
+    return launch_pdl(index_tc_kernel<true>, dim3(grid), dim3(Layout<true>::threads), Layout<true>::bytes, s, kmap,
+                      qmap, p);
+  }
+  cudaError_t e = ensure_smem(index_tc_kernel<false>, (int)Layout<false>::bytes, cache);
+  if (e != cudaSuccess) return e;
   TraceScope tr("index_score_tc", s);
-  return launch_pdl(index_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, kmap, qmap, p);
+  return launch_pdl(index_tc_kernel<false>, dim3(grid), dim3(Layout<false>::threads), Layout<false>::bytes, s, kmap,
+                    qmap, p);
 }
 
 }  // namespace ds4a

@@ -229,6 +229,15 @@ struct CompressArgs {
   const int32_t* app_pos;
   uint16_t* ring;
   int ring_cap, n_cap;
+  // block-scaled output (qfmt 1: mixed FP8 / BF16 K=V rows of q_row bytes;
+  // 2: FP4 codes of c/2 bytes plus c/32 scales per entry) instead of bf16:
+  // entry i of sequence b at qpool + b * q_bstride + i * q_row (bytes), its
+  // FP4 scales at qscales + b * qs_bstride + i * (c/32)
+  int qfmt;
+  uint8_t* qpool;
+  int64_t q_bstride, q_row;
+  uint8_t* qscales;
+  int64_t qs_bstride;
   RopeTheta rope;
 };
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
@@ -237,6 +246,9 @@ struct IndexArgs {
   int B, T_q, H, D, m, k, N_c;
   const int32_t* q_pos;
   const uint16_t *q, *w, *kidx;
+  // FP4 keys (kcodes != nullptr): E2M1 codes [.., D/2] and E8M0 scales
+  // [.., D/32] per key; k_bstride then counts keys
+  const uint8_t *kcodes, *kscales;
   int64_t k_bstride;
   float* scores;  // workspace [B*T_q, N_c]
   int32_t* idx_out;
@@ -255,6 +267,9 @@ struct AttendArgs {
   const uint16_t* q;
   const float* q_norm_g;
   const uint16_t* pool;
+  // mixed FP8 / BF16 pool rows (DS4A_MX_KV_FP8), instead of pool when set;
+  // pool_bstride then counts rows
+  const uint8_t* pool8;
   int64_t pool_bstride;
   const int32_t* idx;
   const uint16_t* win;
@@ -275,6 +290,12 @@ cudaError_t launch_attend_generic(const AttendArgs& a, cudaStream_t s);
 bool attend_tc_supported(const AttendArgs& a);
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s);
+
+// bf16 rows -> block-scaled rows (ds4a_mx.cu)
+cudaError_t launch_quant_kv_fp8(int n_rows, int D, int R, const uint16_t* in, int64_t in_stride, uint8_t* out,
+                                int64_t out_stride, cudaStream_t s);
+cudaError_t launch_quant_idx_fp4(int n_rows, int D, const uint16_t* in, int64_t in_stride, uint8_t* codes,
+                                 uint8_t* scales, cudaStream_t s);
 
 // Tensor-core GEMM of the grouped output projection (ds4a_outproj.cu):
 // out[M][N] (row stride ldo) = A x B^T with B = bf16 [N][K]; output tile

@@ -17,11 +17,14 @@ __all__ = [
     "ds4a_compress_state_bytes", "ds4a_compress_append", "ds4a_index_topk_workspace", "ds4a_index_topk", "ds4a_index_topk_noalloc", "ds4a_attend_workspace", "ds4a_sparse_attend",
     "ds4a_hca_attend", "ds4a_check", "ds4a_strerror", "ds4a_trace_enable", "ds4a_trace_read",
     "ds4a_version", "ds4a_selftest_wait_timeout", "OprojCfg", "ds4a_out_proj_workspace", "ds4a_out_proj",
+    "DS4A_MX_KV_FP8", "DS4A_MX_IDX_FP4", "ds4a_kv_fp8_row_bytes", "ds4a_quantize_kv_fp8", "ds4a_quantize_idx_fp4",
+    "ds4a_compress_append_mx", "ds4a_index_topk_fp4", "ds4a_sparse_attend_fp8", "ds4a_hca_attend_fp8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libds4a.so")
 
 DS4A_OK, DS4A_EINVAL, DS4A_EUNSUPPORTED, DS4A_ECUDA, DS4A_EDEVICE, DS4A_ETIMEOUT, DS4A_ENOSPACE = range(7)
+DS4A_MX_KV_FP8, DS4A_MX_IDX_FP4 = 1, 2
 
 
 class Ds4aError(RuntimeError):
@@ -64,6 +67,13 @@ _SIGS = {
     "ds4a_compress_state_bytes": (_SZ, [_CFG, _I, _I, _I]),
     "ds4a_compress_append": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _I64, _P]),
     "ds4a_index_topk_workspace": (_SZ, [_CFG, _I, _I, _I]),
+    "ds4a_kv_fp8_row_bytes": (_SZ, [_I, _I]),
+    "ds4a_quantize_kv_fp8": (_I, [_I, _I, _I, _P, _I64, _P, _I64, _P]),
+    "ds4a_quantize_idx_fp4": (_I, [_I, _I, _P, _I64, _P, _P, _P]),
+    "ds4a_compress_append_mx": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _I64, _P]),
+    "ds4a_index_topk_fp4": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
+    "ds4a_sparse_attend_fp8": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _I, _I64, _P, _P, _P, _SZ, _P]),
+    "ds4a_hca_attend_fp8": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _I, _I64, _P, _P, _P, _SZ, _P]),
     "ds4a_index_topk": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
     "ds4a_index_topk_noalloc": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _I64, _I, _P, _P, _P]),
     "ds4a_attend_workspace": (_SZ, [_CFG, _I, _I, _I, _I]),
@@ -162,6 +172,77 @@ def ds4a_compress_append(cfg: LayerCfg, pos, ca, za, bias_a, state, pool, *, cb=
                                     _ptr(bias_a), _ptr(bias_b), _ptr(norm_g), _ptr(state), pool.shape[1],
                                     _ptr(pool), pool.stride(0), _stream(stream))
     _ok(rc, "ds4a_compress_append")
+
+
+def ds4a_kv_fp8_row_bytes(D: int, R: int) -> int:
+    return lib().ds4a_kv_fp8_row_bytes(D, R)
+
+
+def ds4a_quantize_kv_fp8(rows, R: int, out, *, stream=None):
+    """bf16 K=V rows [n, D] -> FP8 / BF16 rows out [n, row_bytes] (uint8)."""
+    _bf16(rows, "rows")
+    n, D = rows.reshape(-1, rows.shape[-1]).shape
+    rc = lib().ds4a_quantize_kv_fp8(n, D, R, _ptr(rows), D, _ptr(out), out.shape[-1], _stream(stream))
+    _ok(rc, "ds4a_quantize_kv_fp8")
+
+
+def ds4a_quantize_idx_fp4(keys, codes, scales, *, stream=None):
+    """bf16 indexer keys [n, D] -> E2M1 codes [n, D/2] and E8M0 scales [n, D/32] (uint8)."""
+    _bf16(keys, "keys")
+    n, D = keys.reshape(-1, keys.shape[-1]).shape
+    rc = lib().ds4a_quantize_idx_fp4(n, D, _ptr(keys), D, _ptr(codes), _ptr(scales), _stream(stream))
+    _ok(rc, "ds4a_quantize_idx_fp4")
+
+
+def ds4a_compress_append_mx(cfg: LayerCfg, pos, ca, za, bias_a, state, fmt: int, pool, *, scales=None, cb=None,
+                            zb=None, bias_b=None, norm_g=None, stream=None):
+    """ds4a_compress_append writing block-scaled entries: pool is uint8
+    [B, N_cap, row_bytes] (FP8 K=V) or [B, N_cap, c/2] (FP4 keys, with
+    scales [B, N_cap, c/32])."""
+    _bf16(ca, "ca"), _bf16(za, "za"), _bf16(cb, "cb"), _bf16(zb, "zb")
+    B, c = ca.shape
+    rc = lib().ds4a_compress_append_mx(ctypes.byref(cfg), B, c, _ptr(pos), _ptr(ca), _ptr(cb), _ptr(za), _ptr(zb),
+                                       _ptr(bias_a), _ptr(bias_b), _ptr(norm_g), _ptr(state), pool.shape[1], fmt,
+                                       _ptr(pool), _ptr(scales), pool.shape[1], _stream(stream))
+    _ok(rc, "ds4a_compress_append_mx")
+
+
+def ds4a_index_topk_fp4(cfg: LayerCfg, q_pos, q_idx, w_idx, k_codes, k_scales, N_c: int, idx_out, ws, *,
+                        score_out=None, stream=None):
+    """ds4a_index_topk over FP4 keys: k_codes [B, >=N_c, D/2], k_scales [B, >=N_c, D/32]."""
+    _bf16(q_idx, "q_idx"), _bf16(w_idx, "w_idx")
+    B, T_q = q_pos.shape
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = lib().ds4a_index_topk_fp4(ctypes.byref(cfg), B, T_q, _ptr(q_pos), _ptr(q_idx), _ptr(w_idx), _ptr(k_codes),
+                                   _ptr(k_scales), 0 if k_codes is None else k_codes.shape[1], N_c, _ptr(idx_out),
+                                   _ptr(score_out), _ptr(ws), ws_bytes, _stream(stream))
+    _ok(rc, "ds4a_index_topk_fp4")
+
+
+def ds4a_sparse_attend_fp8(cfg: LayerCfg, q_pos, q, q_norm_g, pool, N_c: int, idx, win, win_cap: int, sink, out,
+                           ws=None, *, stream=None):
+    """ds4a_sparse_attend over an FP8 / BF16 pool: uint8 [B, >=N_c, row_bytes]."""
+    _bf16(q, "q")
+    B, T_q = q_pos.shape
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = lib().ds4a_sparse_attend_fp8(ctypes.byref(cfg), B, T_q, _ptr(q_pos), _ptr(q), _ptr(q_norm_g), _ptr(pool),
+                                      0 if pool is None else pool.shape[1], N_c, _ptr(idx), _ptr(win), win_cap,
+                                      0 if win is None else win.stride(0), _ptr(sink), _ptr(out), _ptr(ws), ws_bytes,
+                                      _stream(stream))
+    _ok(rc, "ds4a_sparse_attend_fp8")
+
+
+def ds4a_hca_attend_fp8(cfg: LayerCfg, q_pos, q, q_norm_g, pool, N_c: int, win, win_cap: int, sink, out, ws=None,
+                        *, stream=None):
+    """ds4a_hca_attend over an FP8 / BF16 pool: uint8 [B, >=N_c, row_bytes]."""
+    _bf16(q, "q")
+    B, T_q = q_pos.shape
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = lib().ds4a_hca_attend_fp8(ctypes.byref(cfg), B, T_q, _ptr(q_pos), _ptr(q), _ptr(q_norm_g), _ptr(pool),
+                                   0 if pool is None else pool.shape[1], N_c, _ptr(win), win_cap,
+                                   0 if win is None else win.stride(0), _ptr(sink), _ptr(out), _ptr(ws), ws_bytes,
+                                   _stream(stream))
+    _ok(rc, "ds4a_hca_attend_fp8")
 
 
 def ds4a_index_topk_workspace(cfg: LayerCfg, B: int, T_q: int, N_c: int) -> int:

@@ -293,6 +293,133 @@ def out_proj(o, w_a, w_b, n_groups: int):
 
 
 # --------------------------------------------------------------------------
+# (6) block-scaled low-precision cache storage
+# [V4-inside] "What does HCA change?" (paper 2.3.4): the K=V cache keeps its
+# RoPE dims in BF16 and the other dims in FP8; the indexer keys are FP4.  The
+# element formats and the block scaling follow the OCP Microscaling Formats
+# (MX) specification v1.0: 32 consecutive values share one power-of-two
+# scale X stored as E8M0 (exponent + 127); each value is V / X rounded to the
+# nearest representable element (ties to the even code).  FP8 is E4M3 (bias
+# 7, largest 448), FP4 is E2M1 (bias 1, largest 6).  Readings: blocks of 32
+# along the channel axis; X is the smallest power of two with max |V| / X
+# within the element format's range (the specification's floor rule,
+# 2^(floor(log2 max|V|) - emax), would clip a block's largest values by up
+# to 12 %), so no element saturates; an all-zero block takes scale code 0.
+# --------------------------------------------------------------------------
+MX_BLOCK = 32
+_FMT = {"e4m3": dict(ebits=4, mbits=3, bias=7, ncodes=127),   # 0x7F is NaN
+        "e2m1": dict(ebits=2, mbits=1, bias=1, ncodes=8)}
+
+
+def format_values(fmt: str) -> np.ndarray:
+    """Magnitude of every non-negative code of an element format, by code."""
+    f = _FMT[fmt]
+    out = []
+    for code in range(f["ncodes"]):
+        e, m = code >> f["mbits"], code & ((1 << f["mbits"]) - 1)
+        if e == 0:  # subnormal
+            out.append(m / (1 << f["mbits"]) * 2.0 ** (1 - f["bias"]))
+        else:
+            out.append((1 + m / (1 << f["mbits"])) * 2.0 ** (e - f["bias"]))
+    return np.array(out)
+
+
+def round_to_format(x, fmt: str) -> np.ndarray:
+    """Codes (sign in the bit above the magnitude code) of x rounded to the
+    nearest value of the format, ties to the even code, magnitudes clamped
+    to the largest normal."""
+    f = _FMT[fmt]
+    grid = format_values(fmt)
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), grid[-1])
+    hi = np.clip(np.searchsorted(grid, a), 1, grid.size - 1)
+    lo = hi - 1
+    dlo, dhi = a - grid[lo], grid[hi] - a
+    code = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    sign_bit = 1 << (f["ebits"] + f["mbits"])
+    return (code + np.where(np.signbit(x) & (code > 0), sign_bit, 0)).astype(np.uint8)
+
+
+def format_value(codes, fmt: str) -> np.ndarray:
+    f = _FMT[fmt]
+    sign_bit = 1 << (f["ebits"] + f["mbits"])
+    codes = np.asarray(codes).astype(np.int64)
+    mag = format_values(fmt)[codes & (sign_bit - 1)]
+    return np.where(codes & sign_bit, -mag, mag)
+
+
+def mx_quantize(x, fmt: str):
+    """x [..., n] (n a multiple of 32) -> (element codes uint8 [..., n],
+    E8M0 scale codes uint8 [..., n/32])."""
+    x = np.asarray(x, dtype=np.float64)
+    blocks = x.reshape(*x.shape[:-1], -1, MX_BLOCK)
+    amax = np.abs(blocks).max(axis=-1)
+    # smallest s with amax <= largest * 2^s, exactly: with amax = f 2^k and
+    # largest = g 2^j (f, g in [0.5, 1)), s = k - j, plus one when f > g
+    f, k = np.frexp(amax)
+    g, j = np.frexp(format_values(fmt)[-1])
+    shared = np.clip(k - j + (f > g), -127, 127)
+    shared = np.where(amax > 0, shared, -127)
+    q = blocks / np.exp2(shared)[..., None]
+    codes = round_to_format(q, fmt).reshape(x.shape)
+    return codes, (shared + 127).astype(np.uint8)
+
+
+def mx_dequantize(codes, scales, fmt: str) -> np.ndarray:
+    v = format_value(codes, fmt)
+    v = v.reshape(*v.shape[:-1], -1, MX_BLOCK)
+    return (v * np.exp2(np.asarray(scales, dtype=np.float64) - 127.0)[..., None]).reshape(np.shape(codes))
+
+
+def kv_fp8_row_bytes(D: int, R: int) -> int:
+    """Bytes of one mixed K=V row: D - R FP8 codes, R BF16 values, (D - R)/32
+    scales, padded to a multiple of 16."""
+    n = D - R
+    return (n + 2 * R + n // MX_BLOCK + 15) // 16 * 16
+
+
+def quantize_kv_fp8(rows, D: int, R: int) -> np.ndarray:
+    """bf16 K=V rows (uint16 bits or floats) [..., D] -> byte rows: FP8 codes
+    of the first D - R dims, the last R dims as stored bf16 (little endian),
+    the E8M0 scales, zero padding."""
+    bits = np.asarray(rows)
+    if bits.dtype != np.uint16:
+        bits = store_bf16(bits)
+    n = D - R
+    codes, scales = mx_quantize(widen(bits[..., :n]), "e4m3")
+    out = np.zeros(bits.shape[:-1] + (kv_fp8_row_bytes(D, R),), np.uint8)
+    out[..., :n] = codes
+    out[..., n:n + 2 * R] = np.ascontiguousarray(bits[..., n:]).view(np.uint8).reshape(bits.shape[:-1] + (2 * R,))
+    out[..., n + 2 * R:n + 2 * R + n // MX_BLOCK] = scales
+    return out
+
+
+def dequantize_kv_fp8(qrows, D: int, R: int) -> np.ndarray:
+    q = np.asarray(qrows, dtype=np.uint8)
+    n = D - R
+    nope = mx_dequantize(q[..., :n], q[..., n + 2 * R:n + 2 * R + n // MX_BLOCK], "e4m3")
+    rope_bits = np.ascontiguousarray(q[..., n:n + 2 * R]).view(np.uint16)
+    return np.concatenate([nope, widen(rope_bits)], axis=-1)
+
+
+def quantize_idx_fp4(keys):
+    """bf16 indexer keys [..., D] -> (packed E2M1 codes uint8 [..., D/2], even
+    element in the low nibble; E8M0 scales uint8 [..., D/32])."""
+    bits = np.asarray(keys)
+    if bits.dtype != np.uint16:
+        bits = store_bf16(bits)
+    codes, scales = mx_quantize(widen(bits), "e2m1")
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    return packed, scales
+
+
+def dequantize_idx_fp4(packed, scales) -> np.ndarray:
+    p = np.asarray(packed, dtype=np.uint8)
+    codes = np.stack([p & 15, p >> 4], axis=-1).reshape(*p.shape[:-1], 2 * p.shape[-1])
+    return mx_dequantize(codes, scales, "e2m1")
+
+
+# --------------------------------------------------------------------------
 # batch drivers (loops over sequences and queries)
 # --------------------------------------------------------------------------
 def index_topk_batch(qi, wi, ki, q_pos, m: int, k: int, n_c: int, rows=None):

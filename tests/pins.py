@@ -567,4 +567,84 @@ def pin_out_proj_groups_are_separate(O):
     _close(y, O.widen(O.store_bf16(mid)), 0.0, "identity W_b")
 
 
+# --------------------------------------------------------------------------
+# block-scaled FP8 / FP4 storage
+# --------------------------------------------------------------------------
+def pin_e4m3_rounding_vs_torch(O):
+    """E4M3 round-to-nearest-even (subnormals, ties, the top of the range)
+    equals torch's float32 -> float8_e4m3fn conversion for every value torch
+    keeps finite."""
+    rng = np.random.default_rng(19)
+    x = (rng.standard_normal(20000) * np.exp2(rng.integers(-14, 9, 20000))).astype(np.float32)
+    grid = np.concatenate([O.format_values("e4m3"), -O.format_values("e4m3")])
+    mids = ((grid[:-1] + grid[1:]) / 2).astype(np.float32)  # exact ties between neighbours
+    x = np.concatenate([x, grid.astype(np.float32), mids, np.float32([448.0, 460.0, 464.0, -464.0])])
+    x = x[np.abs(x) <= 464.0]
+    ours = O.format_value(O.round_to_format(x, "e4m3"), "e4m3")
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).double().numpy()
+    bad = np.flatnonzero(ours != ref)
+    assert bad.size == 0, f"e4m3 differs from torch at {x[bad[:4]]}: {ours[bad[:4]]} vs {ref[bad[:4]]}"
+    assert O.format_value(O.round_to_format(np.array([1e6, -1e6]), "e4m3"), "e4m3").tolist() == [448.0, -448.0]
+
+
+def pin_e2m1_table(O):
+    """E2M1: the eight magnitudes, nearest-even rounding at the midpoints
+    (OCP MX specification's element format) and clamping at 6."""
+    assert O.format_values("e2m1").tolist() == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    x = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.2, 0.3, 5.1, 7.0, -1.25, -5.0])
+    want = [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 0.0, 0.5, 6.0, 6.0, -1.0, -4.0]
+    assert O.format_value(O.round_to_format(x, "e2m1"), "e2m1").tolist() == want
+
+
+def pin_mx_block_scale(O):
+    """The block scale is the smallest power of two that keeps the block's
+    largest magnitude in range: on-grid blocks survive a round trip exactly,
+    a block max just above the largest element doubles the scale, and every
+    value lands within half a step of itself."""
+    for fmt, top in (("e4m3", 448.0), ("e2m1", 6.0)):
+        grid = O.format_values(fmt)
+        for s in (-20, -3, 0, 5):
+            blk = np.resize(grid, 32) * 2.0 ** s
+            blk[7] = top * 2.0 ** s
+            codes, sc = O.mx_quantize(blk, fmt)
+            assert int(sc[0]) == 127 + s, (fmt, s, sc)
+            _close(O.mx_dequantize(codes, sc, fmt), blk, 0.0, f"{fmt} on-grid round trip")
+            nxt = np.nextafter(top, np.inf) * 2.0 ** s
+            _, sc2 = O.mx_quantize(np.concatenate([[nxt], np.zeros(31)]), fmt)
+            assert int(sc2[0]) == 128 + s
+        rng = np.random.default_rng(20)
+        x = rng.standard_normal((50, 64)) * np.exp2(rng.integers(-6, 6, (50, 1)))
+        codes, sc = O.mx_quantize(x, fmt)
+        d = O.mx_dequantize(codes, sc, fmt)
+        step = np.exp2(sc.astype(np.float64) - 127.0).repeat(32, axis=-1)
+        # half of the largest gap of the format (1 for E4M3 near 448 is 16, scaled)
+        half_gap = {"e4m3": 16.0, "e2m1": 1.0}[fmt]
+        assert np.all(np.abs(d - x) <= half_gap * step + 1e-300)
+    codes, sc = O.mx_quantize(np.zeros(32), "e4m3")
+    assert int(sc[0]) == 0 and not codes.any()
+
+
+def pin_kv_fp8_row_layout(O):
+    """A mixed K=V row: FP8 codes of the first D - R dims, the last R dims as
+    the stored bf16 bits, the scales, zero padding to 16 bytes; 592 bytes at
+    the Flash shape; FP4 indexer keys pack the even element in the low
+    nibble."""
+    assert O.kv_fp8_row_bytes(512, 64) == 592
+    rng = np.random.default_rng(21)
+    rows = O.store_bf16(rng.standard_normal((4, 512)))
+    q = O.quantize_kv_fp8(rows, 512, 64)
+    assert q.shape == (4, 592) and not q[:, 590:].any()
+    assert np.array_equal(q[:, 448:576].view(np.uint16), rows[:, 448:])
+    d = O.dequantize_kv_fp8(q, 512, 64)
+    assert np.array_equal(d[:, 448:], O.widen(rows[:, 448:]))
+    codes, sc = O.mx_quantize(O.widen(rows[:, :448]), "e4m3")
+    assert np.array_equal(q[:, :448], codes) and np.array_equal(q[:, 576:590], sc)
+    keys = O.store_bf16(rng.standard_normal((3, 128)))
+    packed, scales = O.quantize_idx_fp4(keys)
+    c4, s4 = O.mx_quantize(O.widen(keys), "e2m1")
+    assert np.array_equal(packed & 15, c4[:, 0::2]) and np.array_equal(packed >> 4, c4[:, 1::2])
+    assert np.array_equal(scales, s4)
+    _close(O.dequantize_idx_fp4(packed, scales), O.mx_dequantize(c4, s4, "e2m1"), 0.0, "fp4 unpack")
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -53,6 +53,15 @@ MUTANTS = {
     "out_proj weight transposed per group": [("np.concatenate([x[:, j] @ wa[j].T for j in range(n_groups)], axis=1)",
                                               "np.concatenate([x[:, j] @ wa[j].reshape(-1, wa.shape[1]) for j in range(n_groups)], axis=1)")],
     "out_proj second product unrounded": [("y = widen(store_bf16(mid)) @ widen(w_b).T", "y = mid @ widen(w_b).T")],
+    "mx rounding ties away from zero": [("code = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))",
+                                         "code = np.where(dlo < dhi, lo, hi)")],
+    "mx scale floor rule (clips)": [("shared = np.clip(k - j + (f > g), -127, 127)", "shared = np.clip(k - j, -127, 127)")],
+    "fp4 nibbles swapped": [("packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)",
+                             "packed = (codes[..., 1::2] | (codes[..., 0::2] << 4)).astype(np.uint8)")],
+    "fp8 rope dims quantised too": [("out[..., n:n + 2 * R] = np.ascontiguousarray(bits[..., n:]).view(np.uint8).reshape(bits.shape[:-1] + (2 * R,))",
+                                     "out[..., n:n + 2 * R] = np.ascontiguousarray(store_bf16(np.round(widen(bits[..., n:])))).view(np.uint8).reshape(bits.shape[:-1] + (2 * R,))")],
+    "e4m3 subnormal exponent off by one": [("out.append(m / (1 << f[\"mbits\"]) * 2.0 ** (1 - f[\"bias\"]))",
+                                            "out.append(m / (1 << f[\"mbits\"]) * 2.0 ** (0 - f[\"bias\"]))")],
     "pool row ignores idx": [("rows = np.concatenate([widen(pool)[sel], window_rows",
                               "rows = np.concatenate([widen(pool)[: sel.size], window_rows")],
 }

@@ -115,6 +115,11 @@ WORKLOADS = {
     # FP4 indexer keys; the same generated values, quantised on the device
     11: Workload(11, "mix_decode_b8_ctx1m_mx", "mix_decode", 8, 1048575, FLASH_CSA, FLASH_HCA, 262144, 8192,
                  storage="mx"),
+    # the mix at a 128K context: a few hundred MB on the device, still far
+    # above L2 -- the size for multi-pass profiler captures (not bench lines)
+    12: Workload(12, "mix_decode_b8_ctx128k", "mix_decode", 8, 131071, FLASH_CSA, FLASH_HCA, 32768, 1024),
+    13: Workload(13, "mix_decode_b8_ctx128k_mx", "mix_decode", 8, 131071, FLASH_CSA, FLASH_HCA, 32768, 1024,
+                 storage="mx"),
 }
 
 # Flash grouped output projection: groups of heads, rank per group, hidden

@@ -327,7 +327,8 @@ def format_values(fmt: str) -> np.ndarray:
 def round_to_format(x, fmt: str) -> np.ndarray:
     """Codes (sign in the bit above the magnitude code) of x rounded to the
     nearest value of the format, ties to the even code, magnitudes clamped
-    to the largest normal."""
+    to the largest normal.  As in IEEE rounding, the sign is kept: a
+    negative value that rounds to zero gives negative zero."""
     f = _FMT[fmt]
     grid = format_values(fmt)
     x = np.asarray(x, dtype=np.float64)
@@ -337,7 +338,7 @@ def round_to_format(x, fmt: str) -> np.ndarray:
     dlo, dhi = a - grid[lo], grid[hi] - a
     code = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
     sign_bit = 1 << (f["ebits"] + f["mbits"])
-    return (code + np.where(np.signbit(x) & (code > 0), sign_bit, 0)).astype(np.uint8)
+    return (code + np.where(np.signbit(x), sign_bit, 0)).astype(np.uint8)
 
 
 def format_value(codes, fmt: str) -> np.ndarray:

@@ -584,6 +584,9 @@ def pin_e4m3_rounding_vs_torch(O):
     ref = torch.from_numpy(x).to(torch.float8_e4m3fn).double().numpy()
     bad = np.flatnonzero(ours != ref)
     assert bad.size == 0, f"e4m3 differs from torch at {x[bad[:4]]}: {ours[bad[:4]]} vs {ref[bad[:4]]}"
+    # the codes themselves, the sign of a value that rounds to zero included
+    codes = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.round_to_format(x, "e4m3"), codes), "e4m3 codes differ from torch's"
     assert O.format_value(O.round_to_format(np.array([1e6, -1e6]), "e4m3"), "e4m3").tolist() == [448.0, -448.0]
 
 
@@ -594,6 +597,8 @@ def pin_e2m1_table(O):
     x = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.2, 0.3, 5.1, 7.0, -1.25, -5.0])
     want = [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 0.0, 0.5, 6.0, 6.0, -1.0, -4.0]
     assert O.format_value(O.round_to_format(x, "e2m1"), "e2m1").tolist() == want
+    # codes: sign in bit 3, kept for a negative value that rounds to zero
+    assert O.round_to_format(np.array([-0.1, 0.1, -6.0, -0.0]), "e2m1").tolist() == [8, 0, 15, 8]
 
 
 def pin_mx_block_scale(O):

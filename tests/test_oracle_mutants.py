@@ -62,6 +62,8 @@ MUTANTS = {
                                      "out[..., n:n + 2 * R] = np.ascontiguousarray(store_bf16(np.round(widen(bits[..., n:])))).view(np.uint8).reshape(bits.shape[:-1] + (2 * R,))")],
     "e4m3 subnormal exponent off by one": [("out.append(m / (1 << f[\"mbits\"]) * 2.0 ** (1 - f[\"bias\"]))",
                                             "out.append(m / (1 << f[\"mbits\"]) * 2.0 ** (0 - f[\"bias\"]))")],
+    "mx drops the sign of zero": [("return (code + np.where(np.signbit(x), sign_bit, 0)).astype(np.uint8)",
+                                   "return (code + np.where(np.signbit(x) & (code > 0), sign_bit, 0)).astype(np.uint8)")],
     "pool row ignores idx": [("rows = np.concatenate([widen(pool)[sel], window_rows",
                               "rows = np.concatenate([widen(pool)[: sel.size], window_rows")],
 }

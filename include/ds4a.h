@@ -357,9 +357,10 @@ typedef struct ds4a_oproj_cfg {
   int32_t n_heads, head_dim, n_groups, group_rank, hidden;
 } ds4a_oproj_cfg;
 
-/* Bytes of workspace ds4a_out_proj needs for M tokens (float partial sums
- * when M is too small for the row and output tiles to fill the SMs, else
- * 0). */
+/* Bytes of workspace ds4a_out_proj needs for M tokens: when M is too small
+ * for the row and output tiles to fill the SMs, K is split and each split's
+ * float partial sums are kept apart and added in split order (the result
+ * does not depend on scheduling); else 0. */
 size_t ds4a_out_proj_workspace(const ds4a_oproj_cfg* cfg, int M);
 
 /*

@@ -67,12 +67,11 @@ constexpr uint32_t kOffSink = kOffInv + 256;        // [64] sink * log2(e)
 constexpr uint32_t kOffNext = kOffSink + 256;       // the softmax warps' next work item
 constexpr uint32_t kOffValid = kOffNext + 64;       // [2 tiles][128 keys] validity flags
 // FP8 pools: codes of dims 384..447 staged per row, each row's 16-byte
-// scale run, and the E4M3 value of every code
+// scale run
 constexpr uint32_t kOffStage3 = kOffValid + 256;    // [128 keys][64 B]
 constexpr uint32_t kOffScale = kOffStage3 + 8192;   // [128 keys][16 B]
-constexpr uint32_t kOffLut8 = kOffScale + 2048;     // [256] floats
 constexpr uint32_t kSmemBytes = kOffValid + 256 + 1024;   // bf16 pools (+ alignment slack)
-constexpr uint32_t kSmemBytes8 = kOffLut8 + 1024 + 1024;  // FP8 pools
+constexpr uint32_t kSmemBytes8 = kOffScale + 2048 + 1024;  // FP8 pools
 constexpr int kRow8 = 592;                          // bytes of a mixed FP8 / BF16 row (D 512, R 64)
 constexpr int kNope8 = 448;                         // FP8 dims of a row
 
@@ -608,11 +607,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pt = tid - kPG0;  // 0..127
     uint32_t gt = 0, active = 0;
     bool tma_used = false;
-    if (kFp8) {
-      float* lut = reinterpret_cast<float*>(smem + kOffLut8);
-      for (int c = pt; c < 256; c += 128) lut[c] = e4m3_value((uint32_t)c);
-      named_bar(2, 128);
-    }
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       const Item it = make_item(a, w);
       if (it.n_tiles == 0) continue;
@@ -666,7 +660,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto convert_chunk8 = [&](int c) {
         named_bar(2, 128);
         if (vflag[(gt & 1u) * kKT + pt] != 2) return;
-        const float* lut = reinterpret_cast<const float*>(smem + kOffLut8);
         const unsigned char* stg = c < 3 ? smem + kOffKV + (2 * c + 1) * 16384 + pt * 128 : smem + kOffStage3 + pt * 64;
         const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(smem + kOffScale + pt * 16 + 4 * c);
         // 16 codes = dims 128c + 16q .. + 15 (one scale block per two q) ->
@@ -677,8 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t o[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const uint32_t w = wd[k >> 1] >> (16 * (k & 1));
-            o[k] = f2_to_bf2x2(lut[w & 255u] * sc, lut[(w >> 8) & 255u] * sc);
+            const float2 v = mul_f2(e4m3x2_to_f2(wd[k >> 1] >> (16 * (k & 1))), make_float2(sc, sc));
+            o[k] = f2_to_bf2x2(v.x, v.y);
           }
           const int p0 = 2 * q;
           const uint32_t b0 = kv_base + (uint32_t)(2 * c + (p0 >> 3)) * 16384u;

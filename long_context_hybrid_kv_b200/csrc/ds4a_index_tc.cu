@@ -22,7 +22,7 @@
 // blocks; pairs past a group's visible entries are skipped.
 // FP4 keys (E2M1 codes and E8M0 scales per 32 dims): a bulk copy brings a
 // tile's packed codes and scales into a raw ring; four more warps (10-13)
-// expand them exactly into the same bf16 tile (a 256-entry table maps a code
+// expand them exactly into the same bf16 tile (the hardware unpacks a code
 // byte to its two values, times the block's power-of-two scale), and the
 // products and the epilogue are unchanged.  Three stages instead of four
 // make room for the raw ring.
@@ -61,8 +61,7 @@ struct Layout {
   static constexpr uint32_t raw = stages * 32768;                   // FP4: stages x kRawStage
   static constexpr uint32_t q = (raw + (kFp4 ? stages * kRawStage : 0) + 1023) / 1024 * 1024;
   static constexpr uint32_t w = q + 2 * kMaxG * 8192;               // [G*64] floats
-  static constexpr uint32_t lut = w + kMaxG * kHI * 4;              // FP4: 256 float2
-  static constexpr uint32_t bar = lut + (kFp4 ? 2048 : 0);
+  static constexpr uint32_t bar = w + kMaxG * kHI * 4;
   static constexpr uint32_t misc = bar + 256;
   static constexpr uint32_t bytes = misc + 64 + 1024;
   static constexpr int threads = kFp4 ? kThreads + kConvThreads : kThreads;
@@ -263,9 +262,6 @@ __global__ void __launch_bounds__(kFp4 ? 512 : kRegBoundThreads, 1)
   } else if (kFp4 && warp >= 10) {
     // =================== FP4 -> bf16 converters ===================
     const int r = tid - kThreads;  // key row of the tile
-    float2* lut = reinterpret_cast<float2*>(smem + Lay::lut);
-    for (int c = r; c < 256; c += kConvThreads) lut[c] = make_float2(e2m1_value(c & 15u), e2m1_value(c >> 4));
-    named_bar(2, kConvThreads);
     uint32_t kt = 0;
     for (int w = blockIdx.x; w < p.n_pairs; w += gridDim.x) {
       const Pair q = make_pair(p, w);
@@ -294,8 +290,8 @@ __global__ void __launch_bounds__(kFp4 ? 512 : kRegBoundThreads, 1)
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               const uint32_t byte = (words[2 * h + (k >> 2)] >> (8 * (k & 3))) & 255u;
-              const float2 v = lut[byte];
-              o[k] = live ? f2_to_bf2x2(v.x * sc, v.y * sc) : 0u;
+              const float2 v = mul_f2(e2m1x2_to_f2(byte), make_float2(sc, sc));
+              o[k] = live ? f2_to_bf2x2(v.x, v.y) : 0u;
             }
             // dims 32 i + 16 h .. + 15: block (i >> 1), 16-byte chunks
             const int d0 = 32 * i + 16 * h;

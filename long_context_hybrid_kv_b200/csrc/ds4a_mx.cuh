@@ -68,6 +68,28 @@ __device__ __forceinline__ uint32_t to_e2m1x2(float a, float b) {
   return r & 0xFFu;
 }
 
+// Two codes -> their two values as float32, exactly (the hardware unpacks to
+// f16x2; every E4M3 / E2M1 value is exact in f16), low code first.
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t two) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(two & 0xFFFFu)));
+  float2 r;
+  asm("{\n .reg .f16 lo, hi;\n mov.b32 {lo, hi}, %2;\n cvt.f32.f16 %0, lo;\n cvt.f32.f16 %1, hi;\n}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(h2));
+  return r;
+}
+
+__device__ __forceinline__ float2 e2m1x2_to_f2(uint32_t byte) {
+  uint32_t h2;
+  asm("{\n .reg .b8 t;\n cvt.u8.u32 t, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}" : "=r"(h2) : "r"(byte & 0xFFu));
+  float2 r;
+  asm("{\n .reg .f16 lo, hi;\n mov.b32 {lo, hi}, %2;\n cvt.f32.f16 %0, lo;\n cvt.f32.f16 %1, hi;\n}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(h2));
+  return r;
+}
+
 // value of an E4M3 code (exact; 0x7F / 0xFF are NaN and never produced)
 __device__ __forceinline__ float e4m3_value(uint32_t code) {
   const uint32_t e = (code >> 3) & 15u, m = code & 7u;

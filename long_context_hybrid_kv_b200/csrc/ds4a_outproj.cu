@@ -21,8 +21,9 @@
 //   warp 0     lane 0: TMA producer (A and B tiles of every k step)
 //   warp 1     TMEM allocation; lane 0 issues the MMAs
 //   warps 2-5  epilogue: warp w reads TMEM lane quarter w % 4 (32 rows of
-//              the tile), converts to bf16 and stores, or with split K adds
-//              float partials into a workspace that a second kernel rounds.
+//              the tile), converts to bf16 and stores, or with split K
+//              stores its split's float partial sums, which a second kernel
+//              adds in split order (deterministic) and rounds.
 // Work units: (row tile, output tile, K split), rastered in bands of eight
 // row tiles so the A and B tiles that concurrent blocks read stay in L2.
 #include <cuda.h>
@@ -56,7 +57,7 @@ struct GemmParams {
   int m_tiles, n_tiles, ksplit, steps_per_split, n_units;
   uint16_t* out;          // bf16 [M][ldo] (ksplit == 1)
   int64_t ldo;
-  float* acc;             // float [M][N] partial sums (ksplit > 1), zeroed before the launch
+  float* acc;             // float [ksplit][M][N] partial sums (ksplit > 1)
   unsigned int* err;
 };
 
@@ -184,7 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(bar(kAccFull0 + ab), (at >> 1) & 1u, abort_flag, err);
       tc_fence_after();
       const int row = w.m0 + r;
-      const bool live = row < p.M && w.k1 > w.k0;
+      const bool live = row < p.M;
+      const bool empty = w.k1 <= w.k0;  // a split with no k steps: its partial is 0
+      const int ks = u % p.ksplit;
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         float v[32];
@@ -199,10 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[q] = make_uint4(f2_to_bf2x2(v[8 * q], v[8 * q + 1]), f2_to_bf2x2(v[8 * q + 2], v[8 * q + 3]),
                                 f2_to_bf2x2(v[8 * q + 4], v[8 * q + 5]), f2_to_bf2x2(v[8 * q + 6], v[8 * q + 7]));
         } else {
-          float4* dst = reinterpret_cast<float4*>(p.acc + (int64_t)row * p.N + col);
+          float4* dst = reinterpret_cast<float4*>(p.acc + ((int64_t)ks * p.M + row) * p.N + col);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            atomicAdd(dst + q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+            dst[q] = empty ? make_float4(0.f, 0.f, 0.f, 0.f)
+                           : make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
       }
       tc_fence_before();
@@ -216,17 +220,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// float partial sums -> bf16 (split-K products), 8 values per thread
-__global__ void __launch_bounds__(256) round_bf16_kernel(const float* __restrict__ acc, int M, int N,
+// split-K partial sums [ksplit][M][N] -> their sum, in split order, as
+// bf16; 8 values per thread
+__global__ void __launch_bounds__(256) round_bf16_kernel(const float* __restrict__ acc, int M, int N, int ksplit,
                                                          uint16_t* __restrict__ out, int64_t ldo) {
   pdl_trigger();
   pdl_wait();
-  const int64_t n8 = (int64_t)M * N / 8;
+  const int64_t n8 = (int64_t)M * N / 8, plane = (int64_t)M * N / 4;  // float4 per split
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t e = i * 8;
     const int row = (int)(e / N), col = (int)(e % N);
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    for (int k = 1; k < ksplit; ++k) {
+      const float4 c = reinterpret_cast<const float4*>(acc)[k * plane + 2 * i];
+      const float4 d = reinterpret_cast<const float4*>(acc)[k * plane + 2 * i + 1];
+      a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
+      b.x += d.x; b.y += d.y; b.z += d.z; b.w += d.w;
+    }
     *reinterpret_cast<uint4*>(out + (int64_t)row * ldo + col) =
         make_uint4(f2_to_bf2x2(a.x, a.y), f2_to_bf2x2(a.z, a.w), f2_to_bf2x2(b.x, b.y), f2_to_bf2x2(b.z, b.w));
   }
@@ -259,7 +270,8 @@ int gemm_ksplit(int M, int N, int K) {
 }
 
 size_t gemm_acc_bytes(int M, int N, int K) {
-  return gemm_ksplit(M, N, K) > 1 ? (size_t)M * N * sizeof(float) : 0;
+  const int ks = gemm_ksplit(M, N, K);
+  return ks > 1 ? (size_t)ks * M * N * sizeof(float) : 0;
 }
 
 // One product: out[M][N] (row stride ldo) = A[M][...] x B[N][K]^T, where
@@ -284,11 +296,7 @@ cudaError_t launch_gemm(const uint16_t* a, int64_t a_cols, int64_t a_ld, const u
   static std::atomic<int> cache[kMaxDevices];
   cudaError_t e = ensure_smem(gemm_tc_kernel, (int)kSmemBytes, cache);
   if (e != cudaSuccess) return e;
-  if (p.ksplit > 1) {
-    if (!acc) return cudaErrorInvalidValue;
-    e = cudaMemsetAsync(acc, 0, (size_t)M * N * sizeof(float), s);
-    if (e != cudaSuccess) return e;
-  }
+  if (p.ksplit > 1 && !acc) return cudaErrorInvalidValue;
   {
     TraceScope tr("out_proj_gemm", s);
     e = launch_pdl(gemm_tc_kernel, dim3(min(p.n_units, 148)), dim3(kThreads), kSmemBytes, s, amap, bmap, p);
@@ -298,7 +306,7 @@ cudaError_t launch_gemm(const uint16_t* a, int64_t a_cols, int64_t a_ld, const u
   const int64_t blocks = (n8 + 255) / 256;
   const int grid = (int)(blocks < 148 * 8 ? blocks : 148 * 8);
   TraceScope tr("out_proj_round", s);
-  return launch_pdl(round_bf16_kernel, dim3(grid), dim3(256), 0, s, (const float*)acc, M, N, out, ldo);
+  return launch_pdl(round_bf16_kernel, dim3(grid), dim3(256), 0, s, (const float*)acc, M, N, p.ksplit, out, ldo);
 }
 
 }  // namespace ds4a

@@ -187,7 +187,8 @@ def test_out_proj_rejects_bad_args():
     assert call(y=MIS) == L.DS4A_EINVAL
     assert call(ws=None, wsb=0) == L.DS4A_ENOSPACE                    # decode needs split-K partials
     cfg = L.OprojCfg(64, 512, 8, 1024, 4096)
-    assert L.ds4a_out_proj_workspace(cfg, 8) == 8 * 8192 * 4
+    # 4 K splits of the first product (8 x 8192 floats each), 8 of the second (8 x 4096)
+    assert L.ds4a_out_proj_workspace(cfg, 8) == 4 * 8 * 8192 * 4 == 8 * 8 * 4096 * 4
     assert L.ds4a_out_proj_workspace(cfg, 16384) == 0
 
 

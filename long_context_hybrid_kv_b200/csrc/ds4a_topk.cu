@@ -14,9 +14,10 @@
 //   topk_cluster_kernel  one 8-block cluster per row (rows up to 262144):
 //                        each block stages a slice; histograms and the
 //                        compaction offsets are summed over the cluster
-//                        through distributed shared memory; a first select
-//                        over the per-thread maxima gives a floor below
-//                        which the main select need not count
+//                        through distributed shared memory; a 2048-bin
+//                        histogram of the per-thread maxima gives a floor
+//                        below which the select need not count, and the
+//                        select takes 11-bit digits (three passes)
 //   topk_global_kernel   one block per row, every pass reading the scores
 //                        from global memory (any length)
 #include <cooperative_groups.h>
@@ -93,6 +94,28 @@ __device__ __forceinline__ void find_digit(const unsigned int* hist, int remaini
       above += cnt[j];
     }
   }
+}
+
+// Digit of a pass over 2048 bins (11-bit digits), blocks of 1024 threads:
+// the bin holding the remaining-th largest key, counting from the top bin,
+// and the count of keys in higher bins.  Every thread must call it.
+__device__ __forceinline__ void find_digit2048(const unsigned int* hist, int remaining, int* s_warp,
+                                               unsigned int* s_digit, int* s_above) {
+  const int t = threadIdx.x;  // bins 2047 - 2t (first) and 2046 - 2t
+  const int c0 = (int)hist[2047 - 2 * t], c1 = (int)hist[2046 - 2 * t];
+  int tot;
+  const int incl = block_incl_scan(c0 + c1, s_warp, &tot);
+  const int excl = incl - (c0 + c1);
+  if (excl < remaining && incl >= remaining) {
+    if (excl + c0 >= remaining) {
+      *s_digit = 2047u - 2u * t;
+      *s_above = excl;
+    } else {
+      *s_digit = 2046u - 2u * t;
+      *s_above = excl + c0;
+    }
+  }
+  __syncthreads();
 }
 
 // Shared-memory slot of key i: XOR-swizzled inside each group of 32 so that
@@ -207,13 +230,12 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThreads)
     topk_cluster_kernel(IndexArgs a) {
   extern __shared__ unsigned int keys[];  // [kClusterSlice]
-  __shared__ unsigned int hist[256];
-  __shared__ unsigned int hist_all[256];
+  __shared__ unsigned int hist[2048];
+  __shared__ unsigned int hist_all[2048];
   __shared__ int s_warp[33];
   __shared__ int s_tot[2];  // this block's tie count, kept count
   __shared__ unsigned int s_digit;
   __shared__ int s_above;
-  __shared__ unsigned int tmaxs[kClusterThreads];
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
   const int row = blockIdx.x / kCluster, tid = threadIdx.x;
@@ -234,51 +256,51 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   const int slice = (n_vis + kCluster - 1) / kCluster;
   const int lo = min(n_vis, rank * slice), hi = min(n_vis, lo + slice);
   const int n = hi - lo;
-  // stage the slice; thread t's keys are t, t + 1024, ...: keep their max
-  tmaxs[tid] = stage_keys<8>(sc + lo, n, keys);
-  // Radix select over the cluster (k-th largest of vals[0..nv) in every
-  // block, counting only values >= floor): the key T and how many of the
-  // values equal to T are needed.
-  auto cluster_select = [&](const unsigned int* vals, bool swz, int nv, unsigned int floor, unsigned int* T_out,
-                            int* need_out) {
-    unsigned int prefix = 0, mask = 0;
-    int remaining = a.k;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
-      __syncthreads();
-      for (int i = tid; i < nv; i += blockDim.x) {
-        const unsigned int u = vals[swz ? kpos(i) : i];
-        if (u >= floor && (u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
-      }
-      cl.sync();  // every block's histogram is complete
-      if (tid < 256) {
-        unsigned int sum = 0;
+  for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  // stage the slice; thread t's keys are t, t + 1024, ...: their maximum
+  const unsigned int tmax = stage_keys<8>(sc + lo, n, keys);
+  // Histogram (cluster-wide, one 2048-bin pass) of the top 11 bits of the
+  // cluster's 8192 per-thread maxima: the lowest key of the bin holding the
+  // k-th largest maximum is a floor with at least k keys at or above it
+  // (each of those maxima is one), so the select over the keys can skip
+  // everything below it and counts about a thousand keys.
+  atomicAdd(&hist[tmax >> 21], 1u);
+  auto reduce_hist = [&]() {
+    cl.sync();  // every block's histogram is complete
+    for (int b = tid; b < 2048; b += blockDim.x) {
+      unsigned int sum = 0;
 #pragma unroll
-        for (int r = 0; r < kCluster; ++r) sum += cl.map_shared_rank(hist, r)[tid];
-        hist_all[tid] = sum;
-      }
-      __syncthreads();
-      find_digit(hist_all, remaining, &s_digit, &s_above);
-      cl.sync();  // peers are done reading this block's histogram
-      prefix |= s_digit << shift;
-      mask |= 255u << shift;
-      remaining -= s_above;
+      for (int r = 0; r < kCluster; ++r) sum += cl.map_shared_rank(hist, r)[b];
+      hist_all[b] = sum;
     }
-    *T_out = prefix;
-    *need_out = remaining;
+    __syncthreads();
   };
-  // The k-th largest of the cluster's 8192 per-thread maxima is a floor
-  // with at least k keys at or above it (each of those k threads holds
-  // one), so the k-th largest key is at or above it too and the select over
-  // the keys can skip everything below: its histogram passes then count
-  // about a thousand keys instead of the whole row.
-  unsigned int floor_key;
-  int unused;
-  cluster_select(tmaxs, false, (int)blockDim.x, 0u, &floor_key, &unused);
-  unsigned int prefix;
-  int remaining;
-  cluster_select(keys, true, n, floor_key, &prefix, &remaining);
+  reduce_hist();
+  find_digit2048(hist_all, a.k, s_warp, &s_digit, &s_above);
+  const unsigned int floor_key = s_digit << 21;
+  // Radix select over the keys >= floor with 11-, 11- and 10-bit digits:
+  // the k-th largest key T and how many of the keys equal to T are needed.
+  unsigned int prefix = 0, mask = 0;
+  int remaining = a.k;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const unsigned int dmask = pass < 2 ? 2047u : 1023u;
+    cl.sync();  // peers are done reading this block's previous histogram
+    for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += blockDim.x) {
+      const unsigned int u = keys[kpos(i)];
+      if (u >= floor_key && (u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+    }
+    reduce_hist();
+    find_digit2048(hist_all, remaining, s_warp, &s_digit, &s_above);
+    prefix |= s_digit << shift;
+    mask |= dmask << shift;
+    remaining -= s_above;
+  }
+  cl.sync();  // no peer still reads this block's histogram
   const unsigned int T = prefix;
   const int need = remaining;
   // ordered compaction across the cluster: block r holds indices

@@ -665,14 +665,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 16 codes = dims 128c + 16q .. + 15 (one scale block per two q) ->
         // the 8-dim pieces 2q, 2q + 1 of the chunk
         auto expand = [&](int q, const uint4 cw) {
-          const float sc = mx_scale((int)((sc4 >> (8 * (q >> 1))) & 255u));
+          const int code = (int)((sc4 >> (8 * (q >> 1))) & 255u);
+          const float sc = mx_scale(code);
           const uint32_t wd[4] = {cw.x, cw.y, cw.z, cw.w};
           uint32_t o[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float2 v = mul_f2(e4m3x2_to_f2(wd[k >> 1] >> (16 * (k & 1))), make_float2(sc, sc));
-            o[k] = f2_to_bf2x2(v.x, v.y);
-          }
+          for (int k = 0; k < 8; ++k) o[k] = e4m3x2_scaled_bf16x2(wd[k >> 1], k & 1, code - 127, sc);
           const int p0 = 2 * q;
           const uint32_t b0 = kv_base + (uint32_t)(2 * c + (p0 >> 3)) * 16384u;
           st_shared16(b0 + sw128(pt, p0 & 7), o[0], o[1], o[2], o[3]);

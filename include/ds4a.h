@@ -297,13 +297,10 @@ int ds4a_index_topk_noalloc(const ds4a_layer_cfg* cfg, int B, int T_q, const int
                             const ds4a_bf16* k_idx, int64_t k_bstride, int N_c,
                             int32_t* idx_out, float* score_out, ds4a_stream stream);
 
-/* Bytes of workspace the attend calls can use for these sizes.  For the
- * Flash head shape (64 heads x 512, tensor cores) it holds one prepared
- * query (64 KiB) per query plus the partial results of key splits (used
- * when few queries are given).  Passing less is allowed down to
- * B * T_q * 64 KiB (the work is then split less); below that the call
- * returns DS4A_ENOSPACE.  Other head shapes run on CUDA cores and use the
- * workspace only for key splits (any size, NULL included, is accepted). */
+/* Bytes of workspace the attend calls can use for these sizes: the float
+ * partial results of key splits, which spread the keys of few queries over
+ * more SMs.  Passing less (NULL included) is allowed: the work is then split
+ * less, down to one split per query, which needs none. */
 size_t ds4a_attend_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c, int sparse);
 
 /*

@@ -20,15 +20,14 @@
 //              normalisation with the sink, de-rotation of the rope slice
 //              by -pos, stores straight from registers.
 //   warp 8     TMEM allocation; lane 0 issues every tcgen05.mma / commit.
-//   warps 9-12 producers: q^ as one 64 KB bulk copy of the image that
-//              qhat_prep_kernel wrote, then the KV rows by cp.async, one
-//              128-dim chunk (32 KB) at a time, each chunk released by the
-//              PV products that read it.
-// qhat_prep_kernel computes q^ = RoPE_pos(RMSNorm(q) * g) for every query
-// (one warp per head, coalesced) straight into that shared-memory image
-// (K-major, 128-byte swizzle, 64 KB per query) in the workspace.  Decode-
-// sized launches (kCompact) skip it: their softmax warps compute q^ into
-// shared memory themselves, before waiting for the preceding kernels.
+//   warps 9-12 producers: the query's 64 heads x 512 by eight TMA tile
+//              loads straight into the operand layout (K-major, 128-byte
+//              swizzle), normalised and rotated in place (q^ =
+//              RoPE_pos(RMSNorm(q) * g)) while the previous item finishes;
+//              then the KV rows by cp.async, one 128-dim chunk (32 KB) at a
+//              time, each chunk released by the PV products that read it.
+// Decode-sized launches (kCompact) prepare q^ in the softmax warps instead,
+// before waiting for the preceding kernels.
 // Work items are (query, key split) pairs taken round-robin by the blocks;
 // with one split the block writes the final bf16 output, otherwise the
 // float partials (max, sum, accumulator) the combine kernel merges.
@@ -66,18 +65,20 @@ constexpr uint32_t kOffInv = kOffAlpha + 256;       // [64]
 constexpr uint32_t kOffSink = kOffInv + 256;        // [64] sink * log2(e)
 constexpr uint32_t kOffNext = kOffSink + 256;       // the softmax warps' next work item
 constexpr uint32_t kOffValid = kOffNext + 64;       // [2 tiles][128 keys] validity flags
+constexpr uint32_t kOffG = kOffValid + 256;        // [512] query RMSNorm gains (prefill form)
+constexpr uint32_t kOffRope = kOffG + 2048;         // [<= 64] (cos, sin) of the item's position
 // FP8 pools: codes of dims 384..447 staged per row, each row's 16-byte
 // scale run
-constexpr uint32_t kOffStage3 = kOffValid + 256;    // [128 keys][64 B]
+constexpr uint32_t kOffStage3 = kOffRope + 512;     // [128 keys][64 B]
 constexpr uint32_t kOffScale = kOffStage3 + 8192;   // [128 keys][16 B]
-constexpr uint32_t kSmemBytes = kOffValid + 256 + 1024;   // bf16 pools (+ alignment slack)
+constexpr uint32_t kSmemBytes = kOffRope + 512 + 1024;     // bf16 pools (+ alignment slack)
 constexpr uint32_t kSmemBytes8 = kOffScale + 2048 + 1024;  // FP8 pools
 constexpr int kRow8 = 592;                          // bytes of a mixed FP8 / BF16 row (D 512, R 64)
 constexpr int kNope8 = 448;                         // FP8 dims of a row
 
 enum Bar {
   kQFull = 0, kQEmpty, kKVFull0, kKVFull1, kKVFull2, kKVFull3, kKVEmpty0, kKVEmpty1, kKVEmpty2,
-  kKVEmpty3, kSFull, kPFull, kPVDone, kEpiDone, kDrain, kNumBars
+  kKVEmpty3, kSFull, kPFull, kPVDone, kEpiDone, kDrain, kQRaw, kNumBars
 };
 
 constexpr uint32_t kIdescQK = idesc_bf16(128, 64, 0, 0);
@@ -180,7 +181,7 @@ struct DenseKV {
 template <bool kCompact, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap kvmap, DenseKV dkv, AttendArgs a, int n_items,
-                     const uint8_t* qimg) {
+                     const __grid_constant__ CUtensorMap qmap) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -209,8 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // decode-sized launches (kCompact): the softmax warps prepare q^ in the
     // kernel and all 256 arrive; otherwise one bulk copy of the prepared
     // image arrives with its bytes
-    mbar_init(bar(kQFull), kCompact ? 256 : 1);
+    mbar_init(bar(kQFull), kCompact ? 256 : 128);
     mbar_init(bar(kQEmpty), 1);
+    mbar_init(bar(kQRaw), 1);
     for (int c = 0; c < 4; ++c) {
       mbar_init(bar(kKVFull0 + c), 128);
       mbar_init(bar(kKVEmpty0 + c), 1);
@@ -605,8 +607,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // =================== producers ===================
     const int pt = tid - kPG0;  // 0..127
-    uint32_t gt = 0, active = 0;
+    uint32_t gt = 0, active = 0, q_loads = 0;
     bool tma_used = false;
+    if (!kCompact) {
+      float* gs = reinterpret_cast<float*>(smem + kOffG);
+      for (int d = pt; d < kD; d += 128) gs[d] = a.q_norm_g[d];
+      named_bar(2, 128);
+    }
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       const Item it = make_item(a, w);
       if (it.n_tiles == 0) continue;
@@ -707,12 +714,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cp_async_commit();
       };
-      // ---- q^ (prepared by qhat_prep_kernel in the shared-memory image
-      // layout): one 64 KB bulk copy once the previous item's QK is done ----
-      if (!kCompact && pt == 0) {
-        if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
-        mbar_expect_tx(bar(kQFull), 65536u);
-        bulk_g2s(q_base, qimg + (size_t)it.row * 65536u, 65536u, bar(kQFull));
+      // ---- q^ (prefill form): once the previous item's QK products are
+      // done, eight TMA tile loads bring the query's 64 heads x 512 into
+      // the operand layout (blocks of 64 dims, 128-byte swizzle); the
+      // producers then normalise and rotate it in place while the previous
+      // item's last softmax, PV and epilogue run ----
+      if (!kCompact) {
+        named_bar(2, 128);  // every producer is done with the previous item's q^ and angles
+        if (pt == 0) {
+          if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
+          mbar_expect_tx(bar(kQRaw), 65536u);
+#pragma unroll 1
+          for (int blk = 0; blk < 8; ++blk)
+            tma_load_2d(q_base + (uint32_t)blk * 8192u, &qmap, blk * 64, it.row * kH, bar(kQRaw));
+          q_loads = active + 1;
+        }
+        float2* rope_s = reinterpret_cast<float2*>(smem + kOffRope);
+        if (pt < a.R / 2) {
+          float cs, sn;
+          rope_cos_sin(it.pos, a.rope.t[pt], &cs, &sn);
+          rope_s[pt] = make_float2(cs, sn);
+        }
+        mbar_wait(bar(kQRaw), active & 1u, abort_flag, err);
+        named_bar(2, 128);
+        // thread pt: head pt / 2, dims 256 (pt & 1) .. + 255 (blocks 4 (pt & 1)
+        // .. + 3); RMS over the head's 512 dims with its partner lane
+        const int h = pt >> 1, half = pt & 1;
+        const float* gs = reinterpret_cast<const float*>(smem + kOffG);
+        float ss = 0.f;
+#pragma unroll 1
+        for (int q = 0; q < 32; ++q) {
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + kOffQ + (4 * half + (q >> 3)) * 8192 +
+                                                          sw128((uint32_t)h, (uint32_t)(q & 7)));
+          const unsigned int wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = bf2x2_to_f2(wv[k]);
+            ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+          }
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        const float rstd = rsqrtf(ss / (float)kD + a.eps);
+        const int R = a.R;
+#pragma unroll 1
+        for (int q = 0; q < 32; ++q) {
+          unsigned char* p = smem + kOffQ + (4 * half + (q >> 3)) * 8192 + sw128((uint32_t)h, (uint32_t)(q & 7));
+          const uint4 v = *reinterpret_cast<const uint4*>(p);
+          const unsigned int wv[4] = {v.x, v.y, v.z, v.w};
+          const int d0 = 256 * half + 8 * q;
+          uint32_t o[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = bf2x2_to_f2(wv[k]);
+            const int d = d0 + 2 * k;
+            float x0 = f.x * rstd * gs[d], x1 = f.y * rstd * gs[d + 1];
+            if (d >= kD - R) {
+              const float2 t = rope_s[(d - (kD - R)) >> 1];
+              const float y0 = x0 * t.x - x1 * t.y, y1 = x0 * t.y + x1 * t.x;
+              x0 = y0;
+              x1 = y1;
+            }
+            o[k] = f2_to_bf2x2(x0, x1);
+          }
+          *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_async_smem();
+        mbar_arrive(bar(kQFull));
       }
       // ---- K=V tiles: each chunk goes out when the PV products of the
       // previous tile have released it ----
@@ -776,95 +843,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_wait<0>();  // nothing of this block is in flight at exit
     if (pt == 0 && tma_used)
       for (int c = 0; c < 4; ++c) mbar_drain(bar(kKVFull0 + c), (gt - 1) & 1u);
+    if (pt == 0 && q_loads > 0) mbar_drain(bar(kQRaw), (q_loads - 1) & 1u);
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
-}
-
-// q^ = RoPE_pos(RMSNorm(q_h) * g) for every query, written as the
-// shared-memory image attend_tc_kernel copies in: 8 blocks of 64 dims, each
-// [64 heads][128 B] with the 128-byte swizzle.  Block = (query, 16 heads),
-// warp = two heads, lane = dims 8l..8l+7 and 256+8l..256+8l+7.
-__global__ void __launch_bounds__(256) qhat_prep_kernel(AttendArgs a, uint8_t* qimg) {
-  __shared__ float2 rt[64];
-  const int row = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_trigger();
-  // every load goes out before any of them is used: the two heads' rows
-  // (heads 16 y + w and 16 y + 8 + w), this lane's gains, the position --
-  // all inputs that no kernel of the chain writes, so they go out before
-  // the wait for the preceding kernels, which only the image writes need
-  // (the previous attention may still be reading the image)
-  const uint16_t* qrow = a.q + (int64_t)row * kH * kD;
-  uint4 v[2][2];
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int h = blockIdx.y * 16 + 8 * u + warp;
-    v[u][0] = *reinterpret_cast<const uint4*>(qrow + h * kD + 8 * lane);
-    v[u][1] = *reinterpret_cast<const uint4*>(qrow + h * kD + 256 + 8 * lane);
-  }
-  float g[16];
-  {
-    const float4 g0 = *reinterpret_cast<const float4*>(a.q_norm_g + 8 * lane);
-    const float4 g1 = *reinterpret_cast<const float4*>(a.q_norm_g + 8 * lane + 4);
-    const float4 g2 = *reinterpret_cast<const float4*>(a.q_norm_g + 256 + 8 * lane);
-    const float4 g3 = *reinterpret_cast<const float4*>(a.q_norm_g + 256 + 8 * lane + 4);
-    const float t[16] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w, g2.x, g2.y, g2.z, g2.w, g3.x, g3.y, g3.z, g3.w};
-#pragma unroll
-    for (int i = 0; i < 16; ++i) g[i] = t[i];
-  }
-  const int pos = a.q_pos[row];
-  const int R = a.R;
-  for (int j = threadIdx.x; j < R / 2; j += blockDim.x) {
-    float cs, sn;
-    rope_cos_sin(pos < 0 ? 0 : pos, a.rope.t[j], &cs, &sn);
-    rt[j] = make_float2(cs, sn);
-  }
-  __syncthreads();
-  pdl_wait();
-  uint8_t* img = qimg + (size_t)row * 65536u;
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int h = blockIdx.y * 16 + 8 * u + warp;
-    float x[16];
-    const unsigned int wa[4] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w};
-    const unsigned int wb[4] = {v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 fa = bf2x2_to_f2(wa[q]), fb = bf2x2_to_f2(wb[q]);
-      x[2 * q] = fa.x;
-      x[2 * q + 1] = fa.y;
-      x[8 + 2 * q] = fb.x;
-      x[8 + 2 * q + 1] = fb.y;
-    }
-    float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) ss += x[i] * x[i];
-    ss = warp_sum(ss);
-    const float rstd = rsqrtf(ss / (float)kD + a.eps);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = x[i] * rstd * g[i];
-#pragma unroll
-    for (int pr = 0; pr < 8; ++pr) {
-      const int i = 2 * pr;
-      const int d = i < 8 ? 8 * lane + i : 256 + 8 * lane + (i - 8);
-      if (d >= kD - R) {
-        const float2 t = rt[(d - (kD - R)) >> 1];
-        const float x0 = x[i], x1 = x[i + 1];
-        x[i] = x0 * t.x - x1 * t.y;
-        x[i + 1] = x0 * t.y + x1 * t.x;
-      }
-    }
-    const uint32_t offA = (uint32_t)(lane >> 3) * 8192u + sw128(h, lane & 7);
-    const uint32_t offB = (uint32_t)(4 + (lane >> 3)) * 8192u + sw128(h, lane & 7);
-    *reinterpret_cast<uint4*>(img + offA) = make_uint4(f2_to_bf2x2(x[0], x[1]), f2_to_bf2x2(x[2], x[3]),
-                                                       f2_to_bf2x2(x[4], x[5]), f2_to_bf2x2(x[6], x[7]));
-    *reinterpret_cast<uint4*>(img + offB) = make_uint4(f2_to_bf2x2(x[8], x[9]), f2_to_bf2x2(x[10], x[11]),
-                                                       f2_to_bf2x2(x[12], x[13]), f2_to_bf2x2(x[14], x[15]));
-  }
 }
 
 }  // namespace
@@ -887,9 +872,6 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   AttendArgs a = a0;
   const int rows = a.B * a.T_q;
   if (rows <= 0) return cudaSuccess;
-  // workspace: [rows x 64 KB q^ images][split partials]
-  uint8_t* qimg = reinterpret_cast<uint8_t*>(a.ws);
-  a.ws = reinterpret_cast<float*>(qimg + (size_t)rows * 65536u);
   const int n_items = rows * a.n_splits;
   const bool compact = n_items <= 148;  // every block takes at most one item
   static std::atomic<int> cache[kMaxDevices], cache_c[kMaxDevices], cache8[kMaxDevices], cache8c[kMaxDevices];
@@ -899,14 +881,21 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
                       : (compact ? ensure_smem(attend_tc_kernel<true, false>, (int)kSmemBytes, cache_c)
                                  : ensure_smem(attend_tc_kernel<false, false>, (int)kSmemBytes, cache));
   if (e != cudaSuccess) return e;
-  if (!compact) {
-    // decode-sized launches prepare q^ inside the attention kernel
-    TraceScope tr("qhat_prep", s);
-    e = launch_pdl(qhat_prep_kernel, dim3(rows, kH / 16), dim3(256), 0, s, a, qimg);
-    if (e != cudaSuccess) return e;
-  }
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
   if (!encode) return cudaErrorNotSupported;
+  // the queries as rows of 512 (one per head), for the prefill form's TMA
+  // loads into the operand layout
+  CUtensorMap qmap;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows * kH};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kH};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.q), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   // HCA keys are consecutive pool entries: a row view of the pool for TMA
   // tile loads (when the sequences are a whole number of rows apart)
   CUtensorMap kvmap;
@@ -929,17 +918,16 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
   const int grid = min(n_items, 148);
   {
     TraceScope tr("attend_tc", s);
-    const uint8_t* qi = qimg;
     if (fp8)
       e = compact ? launch_pdl(attend_tc_kernel<true, true>, dim3(grid), dim3(kThreads), kSmemBytes8, s, kvmap, dkv,
-                               a, n_items, qi)
+                               a, n_items, qmap)
                   : launch_pdl(attend_tc_kernel<false, true>, dim3(grid), dim3(kThreads), kSmemBytes8, s, kvmap, dkv,
-                               a, n_items, qi);
+                               a, n_items, qmap);
     else
       e = compact ? launch_pdl(attend_tc_kernel<true, false>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap, dkv,
-                               a, n_items, qi)
+                               a, n_items, qmap)
                   : launch_pdl(attend_tc_kernel<false, false>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap,
-                               dkv, a, n_items, qi);
+                               dkv, a, n_items, qmap);
   }
   if (e != cudaSuccess || a.n_splits == 1) return e;
   return launch_attend_combine(a, s);

@@ -848,15 +848,12 @@ int attend_splits(int B, int T_q, int keys_max, int H, int D, bool tc, size_t ws
   const int rows = B * T_q;
   const size_t per = (size_t)rows * (2 * H + (size_t)H * D) * sizeof(float);
   if (tc) {
-    // the tensor-core path keeps one 64 KB prepared q^ per query in front
-    // of the split partials; without room for those it cannot run (0)
-    const size_t qimg = (size_t)rows * 65536u;
+    // the tensor-core path needs workspace only for the partials of key
+    // splits; with less than they want it splits less (one split: none)
     int want = attend_tc_splits(B, T_q, keys_max);
-    if (need) *need = qimg + (want > 1 ? per * want : 0);
-    if (ws_bytes < qimg) return 0;
-    const size_t avail = ws_bytes - qimg;
-    if (want > 1 && per > 0 && avail < per * want) {
-      want = (int)(avail / per);
+    if (need) *need = want > 1 ? per * want : 0;
+    if (want > 1 && per > 0 && ws_bytes < per * want) {
+      want = (int)(ws_bytes / per);
       if (want < 2) want = 1;
     }
     return want;

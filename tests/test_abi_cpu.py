@@ -80,14 +80,6 @@ def test_attend_rejects_bad_args(bad):
     assert attend(flash_cfg(), **bad) == L.DS4A_EINVAL
 
 
-def test_flash_shape_needs_the_prepared_query_workspace():
-    # the tensor-core path has no silent CUDA-core fallback: too little
-    # workspace is an error, reported before any launch
-    assert attend(flash_cfg()) == L.DS4A_ENOSPACE
-    assert attend(flash_cfg(), ws=A, wsb=65536 - 16) == L.DS4A_ENOSPACE
-    assert attend(flash_cfg(), B=2, ws=A, wsb=65536) == L.DS4A_ENOSPACE
-
-
 def test_selftest_rejects_bad_limits():
     lib = L.lib()
     assert lib.ds4a_selftest_wait_timeout(0, A, None) == L.DS4A_EINVAL
@@ -198,9 +190,8 @@ def test_workspace_queries():
     assert L.ds4a_index_topk_workspace(cfg, 1, 1, 0) == 0
     # few queries: split over more blocks -> partials need workspace
     assert L.ds4a_attend_workspace(cfg, 1, 1, 2048, True) > 0
-    # many queries on the tensor-core path: one prepared query (64 KiB) each,
-    # no split partials
-    assert L.ds4a_attend_workspace(cfg, 1, 16384, 4096, True) == 16384 * 65536
+    # many queries on the tensor-core path: one split each, no workspace
+    assert L.ds4a_attend_workspace(cfg, 1, 16384, 4096, True) == 0
     # the CUDA-core path (another head width) needs none for many queries
     assert L.ds4a_attend_workspace(flash_cfg(head_dim=256, rope_dim=32), 1, 16384, 4096, True) == 0
 

@@ -127,12 +127,50 @@ __device__ __forceinline__ int kpos(int i) { return i ^ ((i >> 5) & 31); }
 
 // Stage scores [0, n) of `src` as keys in shared memory (slot kpos(i)),
 // every thread's loads in flight together (coalesced, kBatch per thread per
-// round), and return the largest key this thread staged.
+// round), and return the largest key this thread staged.  A 16-byte aligned
+// source goes four keys per load: keys 4j .. 4j+3 share one XOR pattern
+// (kpos flips bits 0-4 by the group index), so they land permuted inside
+// one 16-byte slot and take one 128-bit store.
 template <int kBatch>
 __device__ __forceinline__ unsigned int stage_keys(const float* __restrict__ src, int n, unsigned int* keys) {
   unsigned int tmax = 0u;
   const int nt = blockDim.x, tid = threadIdx.x;
-  for (int base = 0; base < n; base += kBatch * nt) {
+  int done = 0;
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+    const float4* src4 = reinterpret_cast<const float4*>(src);
+    const int n4 = n >> 2;
+    for (int base = 0; base < n4; base += kBatch * nt) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = base + u * nt + tid;
+        v[u] = j < n4 ? src4[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = base + u * nt + tid;
+        if (j < n4) {
+          const unsigned int k0 = f2key(v[u].x), k1 = f2key(v[u].y), k2 = f2key(v[u].z), k3 = f2key(v[u].w);
+          tmax = max(tmax, max(max(k0, k1), max(k2, k3)));
+          const int i = 4 * j;
+          const unsigned int x = (unsigned int)(i >> 5) & 31u;  // kpos(i + e) = i ^ x ^ e
+          const unsigned int m = x & 3u;
+          // slot e holds key 4j + (e ^ m): swap pairs when bit 0 of m is
+          // set, swap halves when bit 1 is
+          const unsigned int a0 = (m & 1u) ? k1 : k0, a1 = (m & 1u) ? k0 : k1;
+          const unsigned int a2 = (m & 1u) ? k3 : k2, a3 = (m & 1u) ? k2 : k3;
+          uint4 w;
+          w.x = (m & 2u) ? a2 : a0;
+          w.y = (m & 2u) ? a3 : a1;
+          w.z = (m & 2u) ? a0 : a2;
+          w.w = (m & 2u) ? a1 : a3;
+          *reinterpret_cast<uint4*>(keys + (i ^ (int)(x & ~3u))) = w;
+        }
+      }
+    }
+    done = n4 << 2;
+  }
+  for (int base = done; base < n; base += kBatch * nt) {
     float v[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -204,6 +242,7 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
   const int run = (n_vis + blockDim.x - 1) / blockDim.x;
   const int i0 = min(n_vis, tid * run), i1 = min(n_vis, i0 + run);
   int gt = 0, eq = 0;
+#pragma unroll 8
   for (int i = i0; i < i1; ++i) {
     const unsigned int u = keys[kpos(i)];
     gt += u > T;
@@ -308,6 +347,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   const int run = (n + blockDim.x - 1) / blockDim.x;
   const int i0 = min(n, tid * run), i1 = min(n, i0 + run);
   int gt = 0, eq = 0;
+#pragma unroll 8
   for (int i = i0; i < i1; ++i) {
     const unsigned int u = keys[kpos(i)];
     gt += u > T;

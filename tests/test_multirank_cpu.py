@@ -57,3 +57,21 @@ def test_single_rank_env_defaults(monkeypatch):
         monkeypatch.delenv(k, raising=False)
     assert bench.dist_env() == (0, 1, 0)
     assert bench.max_over_ranks(2.5, 1) == 2.5
+
+
+def test_reference_arm_line_and_other_ranks(monkeypatch, capsys):
+    # the oracle arm: rank 0 prints one line with the contract's keys; any
+    # other rank exits 0 without work
+    import json
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3", "--workloads", "2"]) == 0
+    assert capsys.readouterr().out.strip() == ""
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3", "--workloads", "2"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"] == "csa_decode_b1_ctx8k"

@@ -107,9 +107,29 @@ def _csa_decode_layer(w, B, pos, n_c, dev, T, pre=""):
         L.ds4a_quantize_idx_fp4(ly.t["ki"].reshape(B * n_c, -1), ly.ki4.view(B * n_c, -1), ly.ki4s.view(B * n_c, -1))
         torch.cuda.synchronize()
         del ly.t["pool"], ly.t["ki"]
+    _csa_jobs(ly)
     ly.step_inputs = ["q", "qi", "wi", "kv_ca_new", "kv_cb_new", "kv_za_new", "kv_zb_new", "ix_ca_new",
                       "ix_cb_new", "ix_za_new", "ix_zb_new"]
     return ly
+
+
+def _csa_jobs(ly):
+    """The two compressor jobs of a CSA decode layer (K=V entries and indexer
+    keys), rebuilt whenever the step's input tensors move."""
+    import long_context_hybrid_kv_b200 as L
+
+    t = ly.t
+    if ly.mx:
+        kv = L.append_job(t["kv_ca_new"], t["kv_za_new"], t["kv_ba"], ly.state_kv, ly.kv8, cb=t["kv_cb_new"],
+                          zb=t["kv_zb_new"], bias_b=t["kv_bb"], norm_g=t["kv_g"], fmt=L.DS4A_MX_KV_FP8)
+        ix = L.append_job(t["ix_ca_new"], t["ix_za_new"], t["ix_ba"], ly.state_ix, ly.ki4, cb=t["ix_cb_new"],
+                          zb=t["ix_zb_new"], bias_b=t["ix_bb"], fmt=L.DS4A_MX_IDX_FP4, scales=ly.ki4s)
+    else:
+        kv = L.append_job(t["kv_ca_new"], t["kv_za_new"], t["kv_ba"], ly.state_kv, t["pool"], cb=t["kv_cb_new"],
+                          zb=t["kv_zb_new"], bias_b=t["kv_bb"], norm_g=t["kv_g"])
+        ix = L.append_job(t["ix_ca_new"], t["ix_za_new"], t["ix_ba"], ly.state_ix, t["ki"], cb=t["ix_cb_new"],
+                          zb=t["ix_zb_new"], bias_b=t["ix_bb"])
+    ly.jobs = [kv, ix]
 
 
 def _hca_decode_layer(w, B, pos, n_c, dev, T, pre=""):
@@ -211,13 +231,8 @@ def _run_layer(ly, stream=None):
     t = ly.t
     S = stream
     if ly.kind == "csa" and ly.mx:
-        pos = ly.q_pos.view(-1)
-        L.ds4a_compress_append_mx(ly.cfg, pos, t["kv_ca_new"], t["kv_za_new"], t["kv_ba"], ly.state_kv,
-                                  L.DS4A_MX_KV_FP8, ly.kv8, cb=t["kv_cb_new"], zb=t["kv_zb_new"], bias_b=t["kv_bb"],
-                                  norm_g=t["kv_g"], stream=S)
-        L.ds4a_compress_append_mx(ly.cfg, pos, t["ix_ca_new"], t["ix_za_new"], t["ix_ba"], ly.state_ix,
-                                  L.DS4A_MX_IDX_FP4, ly.ki4, scales=ly.ki4s, cb=t["ix_cb_new"], zb=t["ix_zb_new"],
-                                  bias_b=t["ix_bb"], stream=S)
+        # the layer's two compressors in one call (one launch)
+        L.ds4a_compress_append_jobs(ly.cfg, ly.q_pos.view(-1), ly.n_c, ly.jobs, stream=S)
         L.ds4a_index_topk_fp4(ly.cfg, ly.q_pos, t["qi"], t["wi"], ly.ki4, ly.ki4s, ly.n_c, ly.idx, ly.ws_index,
                               stream=S)
         L.ds4a_sparse_attend_fp8(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], ly.kv8, ly.n_c, ly.idx, t["win"],
@@ -228,11 +243,8 @@ def _run_layer(ly, stream=None):
         L.ds4a_hca_attend_fp8(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], ly.kv8, ly.n_c, t["win"], t["win"].shape[1],
                               t["sink"], ly.out, ly.ws_att, stream=S)
     elif ly.kind == "csa":
-        pos = ly.q_pos.view(-1)
-        L.ds4a_compress_append(ly.cfg, pos, t["kv_ca_new"], t["kv_za_new"], t["kv_ba"], ly.state_kv, t["pool"],
-                               cb=t["kv_cb_new"], zb=t["kv_zb_new"], bias_b=t["kv_bb"], norm_g=t["kv_g"], stream=S)
-        L.ds4a_compress_append(ly.cfg, pos, t["ix_ca_new"], t["ix_za_new"], t["ix_ba"], ly.state_ix, t["ki"],
-                               cb=t["ix_cb_new"], zb=t["ix_zb_new"], bias_b=t["ix_bb"], stream=S)
+        # the layer's two compressors in one call (one launch)
+        L.ds4a_compress_append_jobs(ly.cfg, ly.q_pos.view(-1), ly.n_c, ly.jobs, stream=S)
         L.ds4a_index_topk(ly.cfg, ly.q_pos, t["qi"], t["wi"], t["ki"], ly.n_c, ly.idx, ly.ws_index, stream=S)
         L.ds4a_sparse_attend(ly.cfg, ly.q_pos, t["q"], t["q_norm_g"], t["pool"], ly.n_c, ly.idx, t["win"],
                              t["win"].shape[1], t["sink"], ly.out, ly.ws_att, stream=S)
@@ -870,6 +882,9 @@ def stage_inputs(st):
         view.copy_(t)
         hbuf[o:o + nb].copy_(t.reshape(-1).view(torch.uint8).cpu())
         ly.t[n] = view
+    for ly in st.layers:
+        if ly.kind == "csa":
+            _csa_jobs(ly)
     return dbuf, hbuf
 
 

@@ -230,6 +230,31 @@ int ds4a_compress_append_mx(const ds4a_layer_cfg* cfg, int B, int c, const int32
                             const float* norm_g, ds4a_bf16* state, int N_cap, int format, uint8_t* pool,
                             uint8_t* scales, int64_t pool_bstride, ds4a_stream stream);
 
+/*
+ * ds4a_compress_append_jobs -- one decode step of up to two compressors of
+ * the same layer (a CSA layer's K=V entries and its indexer keys) in one
+ * call: each job is exactly ds4a_compress_append (format 0) or
+ * ds4a_compress_append_mx (format DS4A_MX_*) with the fields below, and
+ * the same B, positions and N_cap.  Two CSA-shaped jobs (overlap, c a
+ * multiple of 8) run in one launch, so the second does not wait for the
+ * first; otherwise the jobs run one after the other.  (No counterpart on
+ * the pages: a launch-count choice.)
+ */
+typedef struct ds4a_append_job {
+  int32_t c;                          /* channels */
+  int32_t format;                     /* 0 (bf16 entries), DS4A_MX_KV_FP8 or DS4A_MX_IDX_FP4 */
+  const ds4a_bf16 *ca, *cb, *za, *zb; /* the new token's rows [B, c]; cb NULL: HCA form */
+  const float *bias_a, *bias_b;       /* [m, c] */
+  const float* norm_g;                /* [c] or NULL */
+  ds4a_bf16* state;                   /* ds4a_compress_state_bytes(cfg, B, c, cb != NULL) bytes */
+  void* pool;                         /* bf16 entries, or the block-scaled rows */
+  uint8_t* scales;                    /* FP4 scales, else NULL */
+  int64_t pool_bstride;               /* elements (bf16) or entries (block-scaled) between sequences */
+} ds4a_append_job;
+
+int ds4a_compress_append_jobs(const ds4a_layer_cfg* cfg, int B, const int32_t* pos, int N_cap,
+                              const ds4a_append_job* jobs, int n_jobs, ds4a_stream stream);
+
 /* Bytes of workspace ds4a_index_topk needs for these sizes. */
 size_t ds4a_index_topk_workspace(const ds4a_layer_cfg* cfg, int B, int T_q, int N_c);
 

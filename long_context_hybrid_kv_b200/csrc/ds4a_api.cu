@@ -170,13 +170,16 @@ size_t ds4a_compress_state_bytes(const ds4a_layer_cfg* cfg, int B, int c, int ov
   return (size_t)B * S * cap * (size_t)c * sizeof(uint16_t);
 }
 
-// the append call, bf16 (qfmt 0) or block-scaled output (qfmt 1, 2)
-static int compress_append_common(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
-                                  const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
-                                  const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
-                                  const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
-                                  int64_t pool_bstride, int qfmt, uint8_t* qpool, uint8_t* qscales,
-                                  int64_t q_bstride_rows, ds4a_stream stream) {
+// the arguments of one append job, bf16 (qfmt 0) or block-scaled output
+// (qfmt 1, 2), checked; DS4A_OK with *a filled, or an error (nothing to do:
+// DS4A_OK with a->B == 0)
+static int build_append_args(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
+                             const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                             const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                             const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
+                             int64_t pool_bstride, int qfmt, uint8_t* qpool, uint8_t* qscales,
+                             int64_t q_bstride_rows, CompressArgs* out) {
+  out->B = 0;
   if (!cfg || cfg->ratio < 1) return DS4A_EINVAL;
   if (B < 0 || N_cap < 0 || c < 2 || c > 1024 || (c % 2) != 0) return DS4A_EINVAL;
   if ((c % 8) != 0 && c > 512) return DS4A_EINVAL;
@@ -221,7 +224,43 @@ static int compress_append_common(const ds4a_layer_cfg* cfg, int B, int c, const
   fill_rope_theta(&a.rope, a.rope_dim, cfg->rope_base);
   a.err = err_word();
   if (!a.err) return DS4A_ECUDA;
+  *out = a;
+  return DS4A_OK;
+}
+
+static int compress_append_common(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,
+                                  const ds4a_bf16* ca, const ds4a_bf16* cb, const ds4a_bf16* za,
+                                  const ds4a_bf16* zb, const float* bias_a, const float* bias_b,
+                                  const float* norm_g, ds4a_bf16* state, int N_cap, ds4a_bf16* pool,
+                                  int64_t pool_bstride, int qfmt, uint8_t* qpool, uint8_t* qscales,
+                                  int64_t q_bstride_rows, ds4a_stream stream) {
+  CompressArgs a;
+  const int rc = build_append_args(cfg, B, c, pos, ca, cb, za, zb, bias_a, bias_b, norm_g, state, N_cap, pool,
+                                   pool_bstride, qfmt, qpool, qscales, q_bstride_rows, &a);
+  if (rc != DS4A_OK || a.B == 0) return rc;
   return cuda_rc(launch_compress(a, (cudaStream_t)stream));
+}
+
+int ds4a_compress_append_jobs(const ds4a_layer_cfg* cfg, int B, const int32_t* pos, int N_cap,
+                              const ds4a_append_job* jobs, int n_jobs, ds4a_stream stream) {
+  if (n_jobs < 0 || n_jobs > 2 || (n_jobs > 0 && !jobs)) return DS4A_EINVAL;
+  CompressArgs a[2];
+  int n = 0;
+  for (int j = 0; j < n_jobs; ++j) {
+    const ds4a_append_job& J = jobs[j];
+    int qfmt = 0;
+    if (J.format == DS4A_MX_KV_FP8) qfmt = 1;
+    else if (J.format == DS4A_MX_IDX_FP4) qfmt = 2;
+    else if (J.format != 0) return DS4A_EINVAL;
+    const int rc = build_append_args(
+        cfg, B, J.c, pos, J.ca, J.cb, J.za, J.zb, J.bias_a, J.bias_b, J.norm_g, J.state, N_cap,
+        qfmt ? nullptr : static_cast<ds4a_bf16*>(J.pool), J.pool_bstride, qfmt,
+        qfmt ? static_cast<uint8_t*>(J.pool) : nullptr, J.scales, J.pool_bstride, &a[n]);
+    if (rc != DS4A_OK) return rc;
+    if (a[n].B > 0) ++n;
+  }
+  if (n == 0) return DS4A_OK;
+  return cuda_rc(launch_compress_jobs(a, n, (cudaStream_t)stream));
 }
 
 int ds4a_compress_append(const ds4a_layer_cfg* cfg, int B, int c, const int32_t* pos,

@@ -741,22 +741,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         // .. + 3); RMS over the head's 512 dims with its partner lane
         const int h = pt >> 1, half = pt & 1;
         const float* gs = reinterpret_cast<const float*>(smem + kOffG);
-        float ss = 0.f;
+        // eight 16-byte reads in flight, four independent sums
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-        for (int q = 0; q < 32; ++q) {
-          const uint4 v = *reinterpret_cast<const uint4*>(smem + kOffQ + (4 * half + (q >> 3)) * 8192 +
-                                                          sw128((uint32_t)h, (uint32_t)(q & 7)));
-          const unsigned int wv[4] = {v.x, v.y, v.z, v.w};
+        for (int q0 = 0; q0 < 32; q0 += 8) {
+          uint4 v[8];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = bf2x2_to_f2(wv[k]);
-            ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+          for (int u = 0; u < 8; ++u)
+            v[u] = *reinterpret_cast<const uint4*>(smem + kOffQ + (4 * half + ((q0 + u) >> 3)) * 8192 +
+                                                   sw128((uint32_t)h, (uint32_t)((q0 + u) & 7)));
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const unsigned int wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 f = bf2x2_to_f2(wv[k]);
+              s4[k] = fmaf(f.x, f.x, fmaf(f.y, f.y, s4[k]));
+            }
           }
         }
+        float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
         const float rstd = rsqrtf(ss / (float)kD + a.eps);
         const int R = a.R;
-#pragma unroll 1
+#pragma unroll 4
         for (int q = 0; q < 32; ++q) {
           unsigned char* p = smem + kOffQ + (4 * half + (q >> 3)) * 8192 + sw128((uint32_t)h, (uint32_t)(q & 7));
           const uint4 v = *reinterpret_cast<const uint4*>(p);

@@ -150,7 +150,7 @@ __device__ __forceinline__ void store_entry_pair(const CompressArgs& a, int b, i
 }
 
 template <int V>
-__global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs a) {
+__device__ __forceinline__ void compress_body(const CompressArgs& a) {
   extern __shared__ float csm[];
   const int c = a.c, m = a.m;
   const int NC = c / V;
@@ -281,6 +281,22 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressArgs
     }
     store_entry_pair(a, b, i, ch, x0, x1, dst + ch);
   }
+}
+
+template <int V>
+__global__ void __launch_bounds__(kCompressThreads) compress_kernel(const __grid_constant__ CompressArgs a) {
+  compress_body<V>(a);
+}
+
+// Two append-mode compressions in one launch (blockIdx.z picks the job):
+// one decode step of a CSA layer's K=V and indexer-key compressors, which
+// would otherwise each wait for the kernel before them.
+struct CompressPair {
+  CompressArgs j[2];
+};
+template <int V>
+__global__ void __launch_bounds__(kCompressThreads) compress_pair_kernel(const __grid_constant__ CompressPair p) {
+  compress_body<V>(p.j[blockIdx.z]);
 }
 
 // Long entries (HCA: m' = 128 terms) when there are few of them (decode):
@@ -457,6 +473,38 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
     }
     store_entry_pair(a, b, i, ch, x0, x1, dst + k);
   }
+}
+
+// whether a job runs in the one-block-per-entry kernel with 8-wide loads
+static bool plain8(const CompressArgs& a) {
+  const int n_terms = a.cb != nullptr ? 2 * a.m : a.m;
+  return a.c % 8 == 0 && n_terms < 64;
+}
+
+cudaError_t launch_compress_jobs(const CompressArgs* jobs, int n_jobs, cudaStream_t s) {
+  if (n_jobs == 2 && jobs[0].app_pos && jobs[1].app_pos && plain8(jobs[0]) && plain8(jobs[1]) &&
+      jobs[0].B == jobs[1].B && jobs[0].B > 0) {
+    size_t smem = 0;
+    for (int j = 0; j < 2; ++j) {
+      const int NC = jobs[j].c / 8;
+      const int G = NC >= kCompressThreads ? 1 : kCompressThreads / NC;
+      const size_t b = (size_t)(3 * G * jobs[j].c + jobs[j].c) * sizeof(float);
+      smem = b > smem ? b : smem;
+    }
+    static std::atomic<int> cache[kMaxDevices];
+    cudaError_t e = ensure_smem(compress_pair_kernel<8>, (int)smem, cache);
+    if (e != cudaSuccess) return e;
+    CompressPair p;
+    p.j[0] = jobs[0];
+    p.j[1] = jobs[1];
+    TraceScope tr("compress", s);
+    return launch_pdl(compress_pair_kernel<8>, dim3(1, jobs[0].B, 2), dim3(kCompressThreads), smem, s, p);
+  }
+  for (int j = 0; j < n_jobs; ++j) {
+    const cudaError_t e = launch_compress(jobs[j], s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {

@@ -303,22 +303,24 @@ __global__ void __launch_bounds__(kFp4 ? 512 : kRegBoundThreads, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {  // 8 code bytes = 16 dims = two 16-byte pieces
             uint32_t o[8];
+            if (fast) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t byte = (words[2 * h + (k >> 2)] >> (8 * (k & 3))) & 255u;
-              uint32_t w;
-              if (fast) {
+              for (int k = 0; k < 8; ++k) {
+                const uint32_t byte = (words[2 * h + (k >> 2)] >> (8 * (k & 3))) & 255u;
                 // selector nibbles: byte 0 <- low code, byte 2 <- high code
                 // (low bytes), shifted by one nibble for the high bytes
                 const uint32_t sel = (byte & 7u) | ((byte & 0x70u) << 4);
-                w = __byte_perm(tl0, tl1, sel) | __byte_perm(th0, th1, sel << 4) |
-                    ((byte & 0x08u) << 12) | ((byte & 0x80u) << 24);
-              } else {
-                const float2 v = mul_f2(e2m1x2_to_f2(byte), make_float2(sc, sc));
-                w = f2_to_bf2x2(v.x, v.y);
+                o[k] = __byte_perm(tl0, tl1, sel) | __byte_perm(th0, th1, sel << 4) |
+                       ((byte & 0x08u) << 12) | ((byte & 0x80u) << 24);
               }
-              o[k] = live ? w : 0u;
+            } else {
+#pragma unroll 1
+              for (int k = 0; k < 8; ++k)
+                o[k] = e2m1x2_bf16x2_by_cvt((words[2 * h + (k >> 2)] >> (8 * (k & 3))) & 255u, sc);
             }
+            if (!live)
+#pragma unroll
+              for (int k = 0; k < 8; ++k) o[k] = 0u;
             // dims 32 i + 16 h .. + 15: block (i >> 1), 16-byte chunks
             const int d0 = 32 * i + 16 * h;
             const uint32_t blk = dst + (uint32_t)(d0 >> 6) * 16384u;

@@ -241,6 +241,8 @@ struct CompressArgs {
   RopeTheta rope;
 };
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
+// several append-mode jobs of the same batch; two plain jobs share a launch
+cudaError_t launch_compress_jobs(const CompressArgs* jobs, int n_jobs, cudaStream_t s);
 
 struct IndexArgs {
   int B, T_q, H, D, m, k, N_c;

@@ -218,7 +218,8 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
     write_identity(a, n_vis, sc, out, so);
     return;
   }
-  stage_keys<8>(sc, n_vis, keys);
+  // several blocks share an SM here: two 16-byte loads per thread in flight
+  stage_keys<2>(sc, n_vis, keys);
   unsigned int prefix = 0, mask = 0;
   int remaining = a.k;
   for (int pass = 0; pass < 4; ++pass) {

@@ -19,6 +19,7 @@ __all__ = [
     "ds4a_version", "ds4a_selftest_wait_timeout", "OprojCfg", "ds4a_out_proj_workspace", "ds4a_out_proj",
     "DS4A_MX_KV_FP8", "DS4A_MX_IDX_FP4", "ds4a_kv_fp8_row_bytes", "ds4a_quantize_kv_fp8", "ds4a_quantize_idx_fp4",
     "ds4a_compress_append_mx", "ds4a_index_topk_fp4", "ds4a_sparse_attend_fp8", "ds4a_hca_attend_fp8",
+    "AppendJob", "append_job", "ds4a_compress_append_jobs",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libds4a.so")
@@ -47,6 +48,14 @@ class OprojCfg(ctypes.Structure):
                 ("group_rank", ctypes.c_int32), ("hidden", ctypes.c_int32)]
 
 
+class AppendJob(ctypes.Structure):
+    _fields_ = [("c", ctypes.c_int32), ("format", ctypes.c_int32),
+                ("ca", ctypes.c_void_p), ("cb", ctypes.c_void_p), ("za", ctypes.c_void_p), ("zb", ctypes.c_void_p),
+                ("bias_a", ctypes.c_void_p), ("bias_b", ctypes.c_void_p), ("norm_g", ctypes.c_void_p),
+                ("state", ctypes.c_void_p), ("pool", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("pool_bstride", ctypes.c_int64)]
+
+
 def layer_cfg(c) -> LayerCfg:
     """LayerCfg from any object with the fields of ds4a_layer_cfg
     (sm_scale defaults to 1/sqrt(head_dim))."""
@@ -67,6 +76,7 @@ _SIGS = {
     "ds4a_compress_state_bytes": (_SZ, [_CFG, _I, _I, _I]),
     "ds4a_compress_append": (_I, [_CFG, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _I64, _P]),
     "ds4a_index_topk_workspace": (_SZ, [_CFG, _I, _I, _I]),
+    "ds4a_compress_append_jobs": (_I, [_CFG, _I, _P, _I, ctypes.POINTER(AppendJob), _I, _P]),
     "ds4a_kv_fp8_row_bytes": (_SZ, [_I, _I]),
     "ds4a_quantize_kv_fp8": (_I, [_I, _I, _I, _P, _I64, _P, _I64, _P]),
     "ds4a_quantize_idx_fp4": (_I, [_I, _I, _P, _I64, _P, _P, _P]),
@@ -243,6 +253,24 @@ def ds4a_hca_attend_fp8(cfg: LayerCfg, q_pos, q, q_norm_g, pool, N_c: int, win, 
                                    0 if win is None else win.stride(0), _ptr(sink), _ptr(out), _ptr(ws), ws_bytes,
                                    _stream(stream))
     _ok(rc, "ds4a_hca_attend_fp8")
+
+
+def append_job(ca, za, bias_a, state, pool, *, cb=None, zb=None, bias_b=None, norm_g=None, fmt: int = 0,
+               scales=None) -> AppendJob:
+    """One job of ds4a_compress_append_jobs (pool: bf16 [B, N_cap, c], or the
+    block-scaled uint8 rows of fmt)."""
+    _bf16(ca, "ca"), _bf16(za, "za"), _bf16(cb, "cb"), _bf16(zb, "zb")
+    bstride = pool.stride(0) if fmt == 0 else pool.shape[1]
+    return AppendJob(ca.shape[1], fmt, _ptr(ca), _ptr(cb), _ptr(za), _ptr(zb), _ptr(bias_a), _ptr(bias_b),
+                     _ptr(norm_g), _ptr(state), _ptr(pool), _ptr(scales), bstride)
+
+
+def ds4a_compress_append_jobs(cfg: LayerCfg, pos, N_cap: int, jobs, *, stream=None):
+    """Up to two compressors of one layer, one decode step, one launch when both are CSA-shaped."""
+    arr = (AppendJob * len(jobs))(*jobs)
+    rc = lib().ds4a_compress_append_jobs(ctypes.byref(cfg), pos.shape[0], _ptr(pos), N_cap, arr, len(jobs),
+                                         _stream(stream))
+    _ok(rc, "ds4a_compress_append_jobs")
 
 
 def ds4a_index_topk_workspace(cfg: LayerCfg, B: int, T_q: int, N_c: int) -> int:

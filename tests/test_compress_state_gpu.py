@@ -91,3 +91,38 @@ def test_append_reports_full_pool_and_bad_position():
     rc, b = L.ds4a_check()
     assert rc == L.DS4A_EDEVICE and (b & 2), (rc, b)
     assert float(pool.float().abs().max()) == 0.0
+
+
+def test_append_jobs_equal_separate_calls():
+    # a CSA layer's two compressors in one ds4a_compress_append_jobs launch
+    # give the same bits as two ds4a_compress_append calls
+    B, T = 3, 96
+    cfg = L.LayerCfg(64, 512, 64, 128, 64, 128, 512, 4, 512 ** -0.5, 10000.0, 1e-6)
+    outs = []
+    for mode in ("jobs", "separate"):
+        pools, states, args = [], [], []
+        for name, c, norm in (("jkv", 512, True), ("jix", 128, False)):
+            st = {s: bf(host.normal_bf16(SEED, f"{name}.{s}", (B, T, c))) for s in ("ca", "cb", "za", "zb")}
+            ba = f32(host.normal_f32(SEED, f"{name}.ba", (4, c), 0.5))
+            bb = f32(host.normal_f32(SEED, f"{name}.bb", (4, c), 0.5))
+            g = f32(host.normal_f32(SEED, f"{name}.g", (c,), 0.1, 1.0)) if norm else None
+            state = torch.zeros(L.ds4a_compress_state_bytes(cfg, B, c, True) // 2, dtype=torch.bfloat16,
+                                device="cuda")
+            pool = torch.zeros((B, T // 4, c), dtype=torch.bfloat16, device="cuda")
+            pools.append(pool)
+            args.append((st, ba, bb, g, state, pool))
+        for t in range(T):
+            pos = torch.full((B,), t, dtype=torch.int32, device="cuda")
+            rows = [{k: v[:, t].contiguous() for k, v in a[0].items()} for a in args]
+            if mode == "jobs":
+                jobs = [L.append_job(r["ca"], r["za"], a[1], a[4], a[5], cb=r["cb"], zb=r["zb"], bias_b=a[2],
+                                     norm_g=a[3]) for r, a in zip(rows, args)]
+                L.ds4a_compress_append_jobs(cfg, pos, T // 4, jobs)
+            else:
+                for r, a in zip(rows, args):
+                    L.ds4a_compress_append(cfg, pos, r["ca"], r["za"], a[1], a[4], a[5], cb=r["cb"], zb=r["zb"],
+                                           bias_b=a[2], norm_g=a[3])
+        check_ok()
+        outs.append([p.view(torch.int16).cpu().numpy() for p in pools])
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)

@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(512) topk_smem_kernel(IndexArgs a) {
 
 // ---------------------------------------------------------------------------
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThreads)
-    topk_cluster_kernel(IndexArgs a) {
+    topk_cluster_wide_kernel(IndexArgs a) {
   extern __shared__ unsigned int keys[];  // [kClusterSlice]
   __shared__ unsigned int hist[2048];
   __shared__ unsigned int hist_all[2048];
@@ -383,6 +383,173 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
 }
 
 // ---------------------------------------------------------------------------
+// Block-level radix select (1024 threads) over vals[0..n) (slot(i) maps an
+// index to its shared-memory slot), counting only values >= floor, 11-, 11-
+// and 10-bit digits: the k-th largest value and how many equal to it are
+// needed.  hist: 2048 counters of shared memory.
+template <typename Slot>
+__device__ __forceinline__ void block_select(const unsigned int* vals, int n, Slot slot, unsigned int floor_v, int k,
+                                             unsigned int* hist, int* s_warp, unsigned int* s_digit, int* s_above,
+                                             unsigned int* T_out, int* need_out) {
+  unsigned int prefix = 0, mask = 0;
+  int remaining = k;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const unsigned int dmask = pass < 2 ? 2047u : 1023u;
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const unsigned int u = vals[slot(i)];
+      if (u >= floor_v && (u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    find_digit2048(hist, remaining, s_warp, s_digit, s_above);
+    prefix |= *s_digit << shift;
+    mask |= dmask << shift;
+    remaining -= *s_above;
+    __syncthreads();  // every thread has read the digit before the next pass writes it
+  }
+  *T_out = prefix;
+  *need_out = remaining;
+}
+
+// Ordered compaction (1024 threads): thread t walks [t*run, t*run + run) of
+// vals and keeps every value > T and the first `need` values == T in index
+// order; keep(i, o) stores kept i at output position o.  Returns the count.
+template <typename Slot, typename Keep>
+__device__ __forceinline__ int block_compact(const unsigned int* vals, int n, Slot slot, unsigned int T, int need,
+                                             int* s_warp, Keep keep) {
+  const int run = (n + blockDim.x - 1) / blockDim.x;
+  const int i0 = min(n, (int)threadIdx.x * run), i1 = min(n, i0 + run);
+  int gt = 0, eq = 0;
+#pragma unroll 8
+  for (int i = i0; i < i1; ++i) {
+    const unsigned int u = vals[slot(i)];
+    gt += u > T;
+    eq += u == T;
+  }
+  int tot;
+  const int eq_before = block_incl_scan(eq, s_warp, &tot) - eq;
+  const int take_eq = max(0, min(eq, need - eq_before));
+  const int sel_before = block_incl_scan(gt + take_eq, s_warp, &tot) - (gt + take_eq);
+  int o = sel_before, tr = eq_before;
+  for (int i = i0; i < i1; ++i) {
+    const unsigned int u = vals[slot(i)];
+    bool k_ = u > T;
+    if (u == T) k_ = tr++ < need;
+    if (k_) keep(i, o++);
+  }
+  return tot;
+}
+
+constexpr int kLocalK = 2048;  // largest k of the local-candidate cluster kernel
+
+// One 8-block cluster per row (rows up to 262144 entries, k <= 2048): each
+// block stages a slice and selects its own k best with block barriers only
+// (a floor from a histogram of its per-thread maxima, then 11-bit digits),
+// keeping them in index order; after one cluster barrier, block 0 gathers
+// the 8 candidate lists through distributed shared memory (in rank order,
+// so in index order) and selects the row's k among them.  The row's top k
+// lies in the union of the blocks' top k (same tie rule), so the result is
+// exact.
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThreads)
+    topk_cluster_kernel(IndexArgs a) {
+  extern __shared__ unsigned int keys[];  // [kClusterSlice]; block 0 reuses it for the gathered lists
+  __shared__ unsigned int hist[2048];
+  __shared__ unsigned int cand_key[kLocalK];
+  __shared__ int cand_idx[kLocalK];
+  __shared__ int s_warp[33];
+  __shared__ int s_count;
+  __shared__ unsigned int s_digit;
+  __shared__ int s_above;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int row = blockIdx.x / kCluster, tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
+  const int pos = a.q_pos[row];
+  const int n_vis = pos < 0 ? 0 : min((pos + 1) / a.m, a.N_c);
+  const float* sc = a.scores + (int64_t)row * a.N_c;
+  int32_t* out = a.idx_out + (int64_t)row * a.k;
+  float* so = a.score_out ? a.score_out + (int64_t)row * a.k : nullptr;
+  if (n_vis <= a.k) {  // the same branch in every block of the cluster
+    if (rank == 0) {
+      if (pos < 0 && tid == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
+      write_identity(a, n_vis, sc, out, so);
+    }
+    return;
+  }
+  const int k = a.k;
+  // slices start on a multiple of 4 (16-byte aligned loads when the row is)
+  const int slice = ((n_vis + kCluster - 1) / kCluster + 3) & ~3;
+  const int lo = min(n_vis, rank * slice), hi = min(n_vis, lo + slice);
+  const int n = hi - lo;
+  for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const unsigned int tmax = stage_keys<8>(sc + lo, n, keys);
+  auto kslot = [](int i) { return kpos(i); };
+  if (n <= k) {
+    // the whole slice is a candidate list
+    for (int i = tid; i < n; i += blockDim.x) {
+      cand_key[i] = keys[kpos(i)];
+      cand_idx[i] = lo + i;
+    }
+    if (tid == 0) s_count = n;
+  } else {
+    // floor: the lowest key of the 2048-bin bucket holding the k-th largest
+    // per-thread maximum (each thread's maximum is one of its keys, so at
+    // least k keys lie at or above it); no floor when k exceeds the threads
+    unsigned int floor_v = 0u;
+    if (k <= (int)blockDim.x) {
+      atomicAdd(&hist[tmax >> 21], 1u);
+      __syncthreads();
+      find_digit2048(hist, k, s_warp, &s_digit, &s_above);
+      floor_v = s_digit << 21;
+    }
+    unsigned int T;
+    int need;
+    block_select(keys, n, kslot, floor_v, k, hist, s_warp, &s_digit, &s_above, &T, &need);
+    const int cnt = block_compact(keys, n, kslot, T, need, s_warp, [&](int i, int o) {
+      cand_key[o] = keys[kpos(i)];
+      cand_idx[o] = lo + i;
+    });
+    if (tid == 0) s_count = cnt;
+  }
+  cl.sync();  // every block's candidate list is complete
+  if (rank == 0) {
+    // gather the lists in rank order into keys[0 .. total) and the indices
+    // into keys[16384 ..] (total <= 8 k <= 16384)
+    int offs[kCluster + 1];
+    offs[0] = 0;
+#pragma unroll
+    for (int r = 0; r < kCluster; ++r) offs[r + 1] = offs[r] + *cl.map_shared_rank(&s_count, r);
+    const int total = offs[kCluster];
+    int* gidx = reinterpret_cast<int*>(keys + 16384);
+#pragma unroll 1
+    for (int r = 0; r < kCluster; ++r) {
+      const unsigned int* rk = cl.map_shared_rank(cand_key, r);
+      const int* ri = cl.map_shared_rank(cand_idx, r);
+      for (int i = tid; i < offs[r + 1] - offs[r]; i += blockDim.x) {
+        keys[offs[r] + i] = rk[i];
+        gidx[offs[r] + i] = ri[i];
+      }
+    }
+    __syncthreads();
+    auto plain = [](int i) { return i; };
+    unsigned int T;
+    int need;
+    block_select(keys, total, plain, 0u, k, hist, s_warp, &s_digit, &s_above, &T, &need);
+    block_compact(keys, total, plain, T, need, s_warp, [&](int i, int o) {
+      const int e = gidx[i];
+      out[o] = e;
+      if (so) so[o] = sc[e];
+    });
+  }
+  cl.sync();  // no block leaves while block 0 may still read its list
+}
+
+// ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) topk_global_kernel(IndexArgs a) {
   __shared__ unsigned int hist[256];
   __shared__ int s_warp[33];
@@ -456,11 +623,18 @@ cudaError_t launch_topk(const IndexArgs& a, cudaStream_t s) {
   }
   if (a.N_c <= kCluster * kClusterSlice) {
     const size_t smem = (size_t)kClusterSlice * sizeof(unsigned int);
-    static std::atomic<int> cache[kMaxDevices];
-    cudaError_t e = ensure_smem(topk_cluster_kernel, (int)smem, cache);
+    if (a.k <= kLocalK) {
+      static std::atomic<int> cache[kMaxDevices];
+      cudaError_t e = ensure_smem(topk_cluster_kernel, (int)smem, cache);
+      if (e != cudaSuccess) return e;
+      TraceScope tr("topk_cluster", s);
+      return launch_pdl(topk_cluster_kernel, dim3(rows * kCluster), dim3(kClusterThreads), smem, s, a);
+    }
+    static std::atomic<int> cache_w[kMaxDevices];
+    cudaError_t e = ensure_smem(topk_cluster_wide_kernel, (int)smem, cache_w);
     if (e != cudaSuccess) return e;
     TraceScope tr("topk_cluster", s);
-    return launch_pdl(topk_cluster_kernel, dim3(rows * kCluster), dim3(kClusterThreads), smem, s, a);
+    return launch_pdl(topk_cluster_wide_kernel, dim3(rows * kCluster), dim3(kClusterThreads), smem, s, a);
   }
   TraceScope tr("topk_global", s);
   return launch_pdl(topk_global_kernel, dim3(rows), dim3(1024), 0, s, a);

@@ -672,12 +672,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 16 codes = dims 128c + 16q .. + 15 (one scale block per two q) ->
         // the 8-dim pieces 2q, 2q + 1 of the chunk
         auto expand = [&](int q, const uint4 cw) {
-          const int code = (int)((sc4 >> (8 * (q >> 1))) & 255u);
-          const float sc = mx_scale(code);
+          const float sc = mx_scale((int)((sc4 >> (8 * (q >> 1))) & 255u));
           const uint32_t wd[4] = {cw.x, cw.y, cw.z, cw.w};
           uint32_t o[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) o[k] = e4m3x2_scaled_bf16x2(wd[k >> 1], k & 1, code - 127, sc);
+          for (int k = 0; k < 8; ++k) {
+            const float2 v = mul_f2(e4m3x2_to_f2(wd[k >> 1] >> (16 * (k & 1))), make_float2(sc, sc));
+            o[k] = f2_to_bf2x2(v.x, v.y);
+          }
           const int p0 = 2 * q;
           const uint32_t b0 = kv_base + (uint32_t)(2 * c + (p0 >> 3)) * 16384u;
           st_shared16(b0 + sw128(pt, p0 & 7), o[0], o[1], o[2], o[3]);
@@ -721,6 +723,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // item's last softmax, PV and epilogue run ----
       if (!kCompact) {
         named_bar(2, 128);  // every producer is done with the previous item's q^ and angles
+        if (pt == 0 && w + (int)gridDim.x < n_items) {
+          // the next item's query into L2 now, so that its TMA loads (issued
+          // when this item's last QK is done) come from L2
+          const int rn = (w + (int)gridDim.x) / a.n_splits;
+          prefetch_l2_bulk(a.q + (int64_t)rn * kH * kD, (uint32_t)(kH * kD * 2));
+        }
         if (pt == 0) {
           if (active > 0) mbar_wait(bar(kQEmpty), (active - 1) & 1u, abort_flag, err);
           mbar_expect_tx(bar(kQRaw), 65536u);

@@ -282,45 +282,17 @@ __global__ void __launch_bounds__(kFp4 ? 512 : kRegBoundThreads, 1)
         const uint32_t dst = k_base + s * 32768u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {  // 32 dims = one scale block
-          const int code = (int)((sc4 >> (8 * i)) & 255u);
-          const float sc = mx_scale(code);
+          const float sc = mx_scale((int)((sc4 >> (8 * i)) & 255u));
           const uint32_t words[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
-          // the bf16 bits of the 8 E2M1 magnitudes times 2^s, as byte tables
-          // for prmt: the exponent add is exact while every result stays a
-          // normal bf16 (s in [-125, 125]); otherwise the cvt path
-          const int sx = code - 127;
-          const bool fast = sx >= -125 && sx <= 125;
-          uint32_t tl0 = 0, tl1 = 0, th0 = 0, th1 = 0;
-          {
-            const uint32_t add = (uint32_t)(sx * 128);
-            const uint32_t u1 = 0x3F00u + add, u2 = 0x3F80u + add, u3 = 0x3FC0u + add, u4 = 0x4000u + add,
-                           u5 = 0x4040u + add, u6 = 0x4080u + add, u7 = 0x40C0u + add;
-            tl0 = ((u1 & 255u) << 8) | ((u2 & 255u) << 16) | ((u3 & 255u) << 24);
-            tl1 = (u4 & 255u) | ((u5 & 255u) << 8) | ((u6 & 255u) << 16) | ((u7 & 255u) << 24);
-            th0 = (u1 & 0xFF00u) | ((u2 & 0xFF00u) << 8) | ((u3 & 0xFF00u) << 16);
-            th1 = ((u4 >> 8) & 255u) | (u5 & 0xFF00u) | ((u6 & 0xFF00u) << 8) | ((u7 & 0xFF00u) << 16);
-          }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {  // 8 code bytes = 16 dims = two 16-byte pieces
             uint32_t o[8];
-            if (fast) {
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const uint32_t byte = (words[2 * h + (k >> 2)] >> (8 * (k & 3))) & 255u;
-                // selector nibbles: byte 0 <- low code, byte 2 <- high code
-                // (low bytes), shifted by one nibble for the high bytes
-                const uint32_t sel = (byte & 7u) | ((byte & 0x70u) << 4);
-                o[k] = __byte_perm(tl0, tl1, sel) | __byte_perm(th0, th1, sel << 4) |
-                       ((byte & 0x08u) << 12) | ((byte & 0x80u) << 24);
-              }
-            } else {
-#pragma unroll 1
-              for (int k = 0; k < 8; ++k)
-                o[k] = e2m1x2_bf16x2_by_cvt((words[2 * h + (k >> 2)] >> (8 * (k & 3))) & 255u, sc);
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t byte = (words[2 * h + (k >> 2)] >> (8 * (k & 3))) & 255u;
+              const float2 v = mul_f2(e2m1x2_to_f2(byte), make_float2(sc, sc));
+              o[k] = live ? f2_to_bf2x2(v.x, v.y) : 0u;
             }
-            if (!live)
-#pragma unroll
-              for (int k = 0; k < 8; ++k) o[k] = 0u;
             // dims 32 i + 16 h .. + 15: block (i >> 1), 16-byte chunks
             const int d0 = 32 * i + 16 * h;
             const uint32_t blk = dst + (uint32_t)(d0 >> 6) * 16384u;

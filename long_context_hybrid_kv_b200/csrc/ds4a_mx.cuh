@@ -90,41 +90,6 @@ __device__ __forceinline__ float2 e2m1x2_to_f2(uint32_t byte) {
   return r;
 }
 
-// Two E4M3 codes (bytes 0, 1 of w when pair is 0, bytes 2, 3 when 1) times
-// 2^sx as bf16x2, low code in the low half, exactly.  A normal code's bits
-// shift into place and its exponent moves by 120 + sx (valid while sx is in
-// [-120, 119]); a zero or subnormal code in the pair, or a scale outside
-// that range, takes the hardware conversion (sc = 2^sx as a float).
-// the rare cases of the two unpackings below, kept out of line so that the
-// common path is a branch, not a predicated copy of both
-static __device__ __noinline__ uint32_t e4m3x2_bf16x2_by_cvt(uint32_t two, float sc) {
-  float2 v = e4m3x2_to_f2(two);
-  v.x *= sc;
-  v.y *= sc;
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(v.y), "f"(v.x));
-  return r;
-}
-
-static __device__ __noinline__ uint32_t e2m1x2_bf16x2_by_cvt(uint32_t byte, float sc) {
-  float2 v = e2m1x2_to_f2(byte);
-  v.x *= sc;
-  v.y *= sc;
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(v.y), "f"(v.x));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t w, int pair, int sx, float sc) {
-  const uint32_t x = __byte_perm(w, 0u, pair ? 0x4342u : 0x4140u);
-  const uint32_t mag = x & 0x007F007Fu;
-  if (sx >= -120 && sx <= 119 && (mag & 0x0078u) != 0u && (mag & 0x00780000u) != 0u) {
-    const uint32_t off = (uint32_t)((120 + sx) << 7);
-    return ((mag << 4) + (off | (off << 16))) | ((x & 0x00800080u) << 8);
-  }
-  return e4m3x2_bf16x2_by_cvt(pair ? (w >> 16) : w, sc);
-}
-
 // value of an E4M3 code (exact; 0x7F / 0xFF are NaN and never produced)
 __device__ __forceinline__ float e4m3_value(uint32_t code) {
   const uint32_t e = (code >> 3) & 15u, m = code & 7u;

@@ -69,9 +69,10 @@ constexpr uint32_t kOffG = kOffValid + 256;        // [512] query RMSNorm gains 
 constexpr uint32_t kOffRope = kOffG + 2048;         // [<= 64] (cos, sin) of the item's position
 // FP8 pools: codes of dims 384..447 staged per row, each row's 16-byte
 // scale run
-constexpr uint32_t kOffStage3 = kOffRope + 512;     // [128 keys][64 B]
+constexpr uint32_t kOffRstd = kOffRope + 512;       // [64] 1 / RMS of each head of the query (prefill form)
+constexpr uint32_t kOffStage3 = kOffRstd + 256;     // [128 keys][64 B]
 constexpr uint32_t kOffScale = kOffStage3 + 8192;   // [128 keys][16 B]
-constexpr uint32_t kSmemBytes = kOffRope + 512 + 1024;     // bf16 pools (+ alignment slack)
+constexpr uint32_t kSmemBytes = kOffRstd + 256 + 1024;     // bf16 pools (+ alignment slack)
 constexpr uint32_t kSmemBytes8 = kOffScale + 2048 + 1024;  // FP8 pools
 constexpr int kRow8 = 592;                          // bytes of a mixed FP8 / BF16 row (D 512, R 64)
 constexpr int kNope8 = 448;                         // FP8 dims of a row
@@ -719,8 +720,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- q^ (prefill form): once the previous item's QK products are
       // done, eight TMA tile loads bring the query's 64 heads x 512 into
       // the operand layout (blocks of 64 dims, 128-byte swizzle); the
-      // producers then normalise and rotate it in place while the previous
-      // item's last softmax, PV and epilogue run ----
+      // producers normalise and rotate it in place (prep_qhat) after they
+      // have sent out the first two chunks of the item's first tile, so that
+      // the transform overlaps those copies ----
       if (!kCompact) {
         named_bar(2, 128);  // every producer is done with the previous item's q^ and angles
         if (pt == 0 && w + (int)gridDim.x < n_items) {
@@ -737,66 +739,91 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(q_base + (uint32_t)blk * 8192u, &qmap, blk * 64, it.row * kH, bar(kQRaw));
           q_loads = active + 1;
         }
-        float2* rope_s = reinterpret_cast<float2*>(smem + kOffRope);
+        float2* rope_w = reinterpret_cast<float2*>(smem + kOffRope);
         if (pt < a.R / 2) {
           float cs, sn;
           rope_cos_sin(it.pos, a.rope.t[pt], &cs, &sn);
-          rope_s[pt] = make_float2(cs, sn);
+          rope_w[pt] = make_float2(cs, sn);
         }
+      }
+      float2* rope_s = reinterpret_cast<float2*>(smem + kOffRope);
+      float* rstd_s = reinterpret_cast<float*>(smem + kOffRstd);
+      auto prep_qhat = [&]() {
         mbar_wait(bar(kQRaw), active & 1u, abort_flag, err);
         named_bar(2, 128);
-        // thread pt: head pt / 2, dims 256 (pt & 1) .. + 255 (blocks 4 (pt & 1)
-        // .. + 3); RMS over the head's 512 dims with its partner lane
-        const int h = pt >> 1, half = pt & 1;
-        const float* gs = reinterpret_cast<const float*>(smem + kOffG);
-        // eight 16-byte reads in flight, four independent sums
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        // RMS: thread pt takes head pt / 2, dims 256 (pt & 1) .. + 255
+        // (blocks 4 (pt & 1) .. + 3), and adds its partner lane's half
+        {
+          const int h = pt >> 1, half = pt & 1;
+          // eight 16-byte reads in flight, four independent sums
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-        for (int q0 = 0; q0 < 32; q0 += 8) {
-          uint4 v[8];
+          for (int q0 = 0; q0 < 32; q0 += 8) {
+            uint4 v[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            v[u] = *reinterpret_cast<const uint4*>(smem + kOffQ + (4 * half + ((q0 + u) >> 3)) * 8192 +
-                                                   sw128((uint32_t)h, (uint32_t)((q0 + u) & 7)));
+            for (int u = 0; u < 8; ++u)
+              v[u] = *reinterpret_cast<const uint4*>(smem + kOffQ + (4 * half + ((q0 + u) >> 3)) * 8192 +
+                                                     sw128((uint32_t)h, (uint32_t)((q0 + u) & 7)));
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const unsigned int wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            for (int u = 0; u < 8; ++u) {
+              const unsigned int wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float2 f = bf2x2_to_f2(wv[k]);
+                s4[k] = fmaf(f.x, f.x, fmaf(f.y, f.y, s4[k]));
+              }
+            }
+          }
+          float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          if (half == 0) rstd_s[h] = rsqrtf(ss / (float)kD + a.eps);
+        }
+        named_bar(2, 128);
+        // normalise and rotate in place: thread pt takes the 8-dim piece
+        // j = pt % 64 of every other head (pt / 64, + 2, ...), so its gains
+        // and angles stay in registers; a warp's 32 pieces of one head are
+        // 512 contiguous bytes of the row (no bank conflict)
+        {
+          const int j = pt & 63, hs = pt >> 6;
+          const float* gs = reinterpret_cast<const float*>(smem + kOffG);
+          const float4 ga = *reinterpret_cast<const float4*>(gs + 8 * j);
+          const float4 gb = *reinterpret_cast<const float4*>(gs + 8 * j + 4);
+          const float g8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          const int R = a.R;
+          float2 cs4[4];
+          bool rot[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int d = 8 * j + 2 * k;
+            rot[k] = d >= kD - R;
+            cs4[k] = rot[k] ? rope_s[(d - (kD - R)) >> 1] : make_float2(1.f, 0.f);
+          }
+          const uint32_t pbase = kOffQ + (uint32_t)(j >> 3) * 8192u;
+#pragma unroll 4
+          for (int i = 0; i < 32; ++i) {
+            const int h = hs + 2 * i;
+            unsigned char* p = smem + pbase + sw128((uint32_t)h, (uint32_t)(j & 7));
+            const uint4 v = *reinterpret_cast<const uint4*>(p);
+            const float rs = rstd_s[h];
+            const unsigned int wv[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const float2 f = bf2x2_to_f2(wv[k]);
-              s4[k] = fmaf(f.x, f.x, fmaf(f.y, f.y, s4[k]));
+              float x0 = f.x * rs * g8[2 * k], x1 = f.y * rs * g8[2 * k + 1];
+              if (rot[k]) {
+                const float y0 = x0 * cs4[k].x - x1 * cs4[k].y, y1 = x0 * cs4[k].y + x1 * cs4[k].x;
+                x0 = y0;
+                x1 = y1;
+              }
+              o[k] = f2_to_bf2x2(x0, x1);
             }
+            *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
           }
-        }
-        float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        const float rstd = rsqrtf(ss / (float)kD + a.eps);
-        const int R = a.R;
-#pragma unroll 4
-        for (int q = 0; q < 32; ++q) {
-          unsigned char* p = smem + kOffQ + (4 * half + (q >> 3)) * 8192 + sw128((uint32_t)h, (uint32_t)(q & 7));
-          const uint4 v = *reinterpret_cast<const uint4*>(p);
-          const unsigned int wv[4] = {v.x, v.y, v.z, v.w};
-          const int d0 = 256 * half + 8 * q;
-          uint32_t o[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = bf2x2_to_f2(wv[k]);
-            const int d = d0 + 2 * k;
-            float x0 = f.x * rstd * gs[d], x1 = f.y * rstd * gs[d + 1];
-            if (d >= kD - R) {
-              const float2 t = rope_s[(d - (kD - R)) >> 1];
-              const float y0 = x0 * t.x - x1 * t.y, y1 = x0 * t.y + x1 * t.x;
-              x0 = y0;
-              x1 = y1;
-            }
-            o[k] = f2_to_bf2x2(x0, x1);
-          }
-          *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_async_smem();
         mbar_arrive(bar(kQFull));
-      }
+      };
       // ---- K=V tiles: each chunk goes out when the PV products of the
       // previous tile have released it ----
       // Two chunks stay in flight: chunk c goes out, then chunk c-1 is
@@ -821,6 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive(bar(kKVFull0 + c));
             }
           }
+          if (!kCompact && tile == 0) prep_qhat();
           continue;
         }
         set_rowptr(tile);
@@ -828,6 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             issue_chunk8(c);
+            if (!kCompact && tile == 0 && c == 1) prep_qhat();
             if (c > 0) {
               cp_async_wait<1>();
               convert_chunk8(c - 1);
@@ -844,6 +873,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           issue_chunk(c);
+          if (!kCompact && tile == 0 && c == 1) prep_qhat();
           if (c > 0) {
             cp_async_wait<1>();
             fence_async_smem();

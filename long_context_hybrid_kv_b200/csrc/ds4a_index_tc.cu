@@ -79,6 +79,7 @@ struct TcIndexParams {
   int chunk_tiles;     // key tiles per work pair
   int chunks_per_group;
   int n_pairs;
+  int keys_once;       // one group per batch: every key tile is read once
 };
 
 struct Pair {
@@ -169,6 +170,7 @@ __global__ void __launch_bounds__(kFp4 ? 512 : kRegBoundThreads, 1)
     // =================== TMA producer ===================
     if (lane == 0) {
       uint32_t kt = 0, active = 0;
+      const uint64_t pol = l2_evict_first_policy();
       auto load_q = [&](const Pair& q) {
         mbar_expect_tx(bar(kQFull), q_bytes);
         const int qrow = (q.b * a.T_q + q.t0) * kHI;
@@ -200,17 +202,28 @@ __global__ void __launch_bounds__(kFp4 ? 512 : kRegBoundThreads, 1)
             const int64_t key0 = (int64_t)q.b * a.k_bstride + (int64_t)tile * kKT;
             const uint32_t raw = sbase + Lay::raw + s * kRawStage;
             mbar_expect_tx(bar(kRawFull + s), (uint32_t)rows * (kDI / 2 + kDI / kMxBlock));
-            bulk_g2s(raw, a.kcodes + key0 * (kDI / 2), (uint32_t)rows * (kDI / 2), bar(kRawFull + s));
-            bulk_g2s(raw + kRawCodes, a.kscales + key0 * (kDI / kMxBlock), (uint32_t)rows * (kDI / kMxBlock),
-                     bar(kRawFull + s));
+            if (p.keys_once) {
+              bulk_g2s_hint(raw, a.kcodes + key0 * (kDI / 2), (uint32_t)rows * (kDI / 2), bar(kRawFull + s), pol);
+              bulk_g2s_hint(raw + kRawCodes, a.kscales + key0 * (kDI / kMxBlock),
+                            (uint32_t)rows * (kDI / kMxBlock), bar(kRawFull + s), pol);
+            } else {
+              bulk_g2s(raw, a.kcodes + key0 * (kDI / 2), (uint32_t)rows * (kDI / 2), bar(kRawFull + s));
+              bulk_g2s(raw + kRawCodes, a.kscales + key0 * (kDI / kMxBlock), (uint32_t)rows * (kDI / kMxBlock),
+                       bar(kRawFull + s));
+            }
             continue;
           }
           if (kt >= (uint32_t)kS)
             mbar_wait(bar(kKEmpty + s), ((kt / kS) - 1) & 1u, abort_flag, err);
           mbar_expect_tx(bar(kKFull + s), 32768u);
           const uint32_t dst = k_base + s * 32768u;
-          tma_load_3d(dst, &kmap, 0, tile * kKT, q.b, bar(kKFull + s));
-          tma_load_3d(dst + 16384u, &kmap, 64, tile * kKT, q.b, bar(kKFull + s));
+          if (p.keys_once) {
+            tma_load_3d_hint(dst, &kmap, 0, tile * kKT, q.b, bar(kKFull + s), pol);
+            tma_load_3d_hint(dst + 16384u, &kmap, 64, tile * kKT, q.b, bar(kKFull + s), pol);
+          } else {
+            tma_load_3d(dst, &kmap, 0, tile * kKT, q.b, bar(kKFull + s));
+            tma_load_3d(dst + 16384u, &kmap, 64, tile * kKT, q.b, bar(kKFull + s));
+          }
         }
         ++active;
       }
@@ -429,6 +442,7 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s) {
   p.chunk_tiles = chunk;
   p.chunks_per_group = (max_tiles + chunk - 1) / chunk;
   p.n_pairs = p.n_groups * p.chunks_per_group;
+  p.keys_once = p.groups_per_b == 1;
 
   CUtensorMap kmap, qmap;
   memset(&kmap, 0, sizeof(kmap));

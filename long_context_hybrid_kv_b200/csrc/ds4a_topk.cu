@@ -11,13 +11,14 @@
 // ascending without a sort.
 //   topk_smem_kernel     one thread block per row, the row's keys staged in
 //                        shared memory once (rows up to 12288 entries)
-//   topk_cluster_kernel  one 8-block cluster per row (rows up to 262144):
-//                        each block stages a slice; histograms and the
-//                        compaction offsets are summed over the cluster
-//                        through distributed shared memory; a 2048-bin
-//                        histogram of the per-thread maxima gives a floor
-//                        below which the select need not count, and the
-//                        select takes 11-bit digits (three passes)
+//   topk_cluster_kernel  one 8-block cluster per row (rows up to 262144,
+//                        k <= 2048): each block stages a slice; a floor from
+//                        the cluster's histogram of per-thread maxima
+//                        leaves a short candidate list per block, which
+//                        block 0 gathers through distributed shared memory
+//                        and selects from (11-bit digits, three passes)
+//   topk_cluster_wide_kernel  the same rows for k > 2048: histograms and
+//                        compaction offsets summed over the cluster
 //   topk_global_kernel   one block per row, every pass reading the scores
 //                        from global memory (any length)
 #include <cooperative_groups.h>
@@ -445,22 +446,29 @@ __device__ __forceinline__ int block_compact(const unsigned int* vals, int n, Sl
 
 constexpr int kLocalK = 2048;  // largest k of the local-candidate cluster kernel
 
-// One 8-block cluster per row (rows up to 262144 entries, k <= 2048): each
-// block stages a slice and selects its own k best with block barriers only
-// (a floor from a histogram of its per-thread maxima, then 11-bit digits),
-// keeping them in index order; after one cluster barrier, block 0 gathers
-// the 8 candidate lists through distributed shared memory (in rank order,
-// so in index order) and selects the row's k among them.  The row's top k
-// lies in the union of the blocks' top k (same tie rule), so the result is
-// exact.
+// One 8-block cluster per row (rows up to 262144 entries, k <= 2048).
+// Every block stages a slice and histograms its threads' maxima (2048 bins
+// of the top 11 key bits); after one cluster barrier each block sums the 8
+// histograms and takes the floor F = the lowest key of the bin holding the
+// k-th largest maximum.  At least k keys of the row lie at or above F (the
+// maxima are distinct keys), so the row's k-th largest T >= F and every key
+// the selection can keep is >= F.  Each block writes its keys >= F in index
+// order; after a second barrier block 0 gathers the lists (rank order, so
+// index order) and selects the row's k among them.  When some block has
+// more than kLocalK keys >= F (scores crowded into one bin), every block
+// instead selects its own k best (a floor from its own maxima, then 11-bit
+// digits) and block 0 merges those lists: the row's top k lies in the union
+// of the blocks' top k (same tie rule).  Either way the result is exact.
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThreads)
     topk_cluster_kernel(IndexArgs a) {
   extern __shared__ unsigned int keys[];  // [kClusterSlice]; block 0 reuses it for the gathered lists
-  __shared__ unsigned int hist[2048];
+  __shared__ unsigned int hist[2048];     // this block's histogram of maxima (read by the peers)
+  __shared__ unsigned int hsum[2048];     // the cluster's
   __shared__ unsigned int cand_key[kLocalK];
   __shared__ int cand_idx[kLocalK];
   __shared__ int s_warp[33];
-  __shared__ int s_count;
+  __shared__ int s_count, s_count2;  // list lengths: first pass, and the per-block top k
+  __shared__ int s_cnt[kCluster];
   __shared__ unsigned int s_digit;
   __shared__ int s_above;
   cg::cluster_group cl = cg::this_cluster();
@@ -488,52 +496,94 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
   __syncthreads();
   const unsigned int tmax = stage_keys<8>(sc + lo, n, keys);
+  // one count per thread (a thread without keys counts in bin 0, below
+  // every finite score), 8192 over the cluster
+  atomicAdd(&hist[tmax >> 21], 1u);
   auto kslot = [](int i) { return kpos(i); };
-  if (n <= k) {
-    // the whole slice is a candidate list
-    for (int i = tid; i < n; i += blockDim.x) {
-      cand_key[i] = keys[kpos(i)];
-      cand_idx[i] = lo + i;
-    }
-    if (tid == 0) s_count = n;
-  } else {
-    // floor: the lowest key of the 2048-bin bucket holding the k-th largest
-    // per-thread maximum (each thread's maximum is one of its keys, so at
-    // least k keys lie at or above it); no floor when k exceeds the threads
-    unsigned int floor_v = 0u;
-    if (k <= (int)blockDim.x) {
-      atomicAdd(&hist[tmax >> 21], 1u);
-      __syncthreads();
-      find_digit2048(hist, k, s_warp, &s_digit, &s_above);
-      floor_v = s_digit << 21;
-    }
-    unsigned int T;
-    int need;
-    block_select(keys, n, kslot, floor_v, k, hist, s_warp, &s_digit, &s_above, &T, &need);
-    const int cnt = block_compact(keys, n, kslot, T, need, s_warp, [&](int i, int o) {
-      cand_key[o] = keys[kpos(i)];
-      cand_idx[o] = lo + i;
-    });
-    if (tid == 0) s_count = cnt;
+  cl.sync();  // every block's histogram of maxima is complete
+  for (int i = tid; i < 2048; i += blockDim.x) {
+    unsigned int c[kCluster];
+#pragma unroll
+    for (int r = 0; r < kCluster; ++r) c[r] = cl.map_shared_rank(hist, r)[i];
+    unsigned int t = 0;
+#pragma unroll
+    for (int r = 0; r < kCluster; ++r) t += c[r];
+    hsum[i] = t;
   }
-  cl.sync();  // every block's candidate list is complete
+  __syncthreads();
+  find_digit2048(hsum, k, s_warp, &s_digit, &s_above);
+  const unsigned int F = s_digit << 21;
+  {
+    // this block's keys >= F, in index order (thread t walks its own run)
+    const int run = (n + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(n, tid * run), i1 = min(n, i0 + run);
+    int cnt = 0;
+#pragma unroll 8
+    for (int i = i0; i < i1; ++i) cnt += keys[kpos(i)] >= F;
+    int tot;
+    int o = block_incl_scan(cnt, s_warp, &tot) - cnt;
+    if (tot <= kLocalK)
+      for (int i = i0; i < i1; ++i) {
+        const unsigned int u = keys[kpos(i)];
+        if (u >= F) {
+          cand_key[o] = u;
+          cand_idx[o] = lo + i;
+          ++o;
+        }
+      }
+    if (tid == 0) s_count = tot;
+  }
+  cl.sync();  // every block's list (or its count alone, when too long) is in place
+  if (tid < kCluster) s_cnt[tid] = *cl.map_shared_rank(&s_count, tid);
+  __syncthreads();
+  bool overflow = false;
+#pragma unroll
+  for (int r = 0; r < kCluster; ++r) overflow |= s_cnt[r] > kLocalK;
+  if (overflow) {
+    // the same decision in every block: each selects its own k best
+    if (n <= k) {
+      for (int i = tid; i < n; i += blockDim.x) {
+        cand_key[i] = keys[kpos(i)];
+        cand_idx[i] = lo + i;
+      }
+      if (tid == 0) s_count2 = n;
+    } else {
+      // floor: the lowest key of the bin holding the k-th largest of this
+      // block's maxima (hist is this block's, no longer read by the peers);
+      // no floor when k exceeds the threads
+      unsigned int floor_v = 0u;
+      if (k <= (int)blockDim.x) {
+        find_digit2048(hist, k, s_warp, &s_digit, &s_above);
+        floor_v = s_digit << 21;
+      }
+      unsigned int T;
+      int need;
+      block_select(keys, n, kslot, floor_v, k, hist, s_warp, &s_digit, &s_above, &T, &need);
+      const int cnt = block_compact(keys, n, kslot, T, need, s_warp, [&](int i, int o) {
+        cand_key[o] = keys[kpos(i)];
+        cand_idx[o] = lo + i;
+      });
+      if (tid == 0) s_count2 = cnt;
+    }
+    cl.sync();  // every block's candidate list is complete
+    if (tid < kCluster) s_cnt[tid] = *cl.map_shared_rank(&s_count2, tid);
+    __syncthreads();
+  }
   if (rank == 0) {
     // gather the lists in rank order into keys[0 .. total) and the indices
-    // into keys[16384 ..] (total <= 8 k <= 16384)
+    // into keys[16384 ..] (total <= 8 kLocalK = 16384)
     int offs[kCluster + 1];
     offs[0] = 0;
 #pragma unroll
-    for (int r = 0; r < kCluster; ++r) offs[r + 1] = offs[r] + *cl.map_shared_rank(&s_count, r);
+    for (int r = 0; r < kCluster; ++r) offs[r + 1] = offs[r] + s_cnt[r];
     const int total = offs[kCluster];
     int* gidx = reinterpret_cast<int*>(keys + 16384);
-#pragma unroll 1
-    for (int r = 0; r < kCluster; ++r) {
-      const unsigned int* rk = cl.map_shared_rank(cand_key, r);
-      const int* ri = cl.map_shared_rank(cand_idx, r);
-      for (int i = tid; i < offs[r + 1] - offs[r]; i += blockDim.x) {
-        keys[offs[r] + i] = rk[i];
-        gidx[offs[r] + i] = ri[i];
-      }
+    for (int i = tid; i < total; i += blockDim.x) {
+      int r = 0;
+#pragma unroll
+      for (int q = 1; q < kCluster; ++q) r += i >= offs[q];
+      keys[i] = cl.map_shared_rank(cand_key, r)[i - offs[r]];
+      gidx[i] = cl.map_shared_rank(cand_idx, r)[i - offs[r]];
     }
     __syncthreads();
     auto plain = [](int i) { return i; };

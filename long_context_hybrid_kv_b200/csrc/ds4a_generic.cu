@@ -74,16 +74,28 @@ __device__ __forceinline__ const uint16_t* term_row(const CompressArgs& a, bool 
   return a.ring + (((int64_t)b * S + st) * a.ring_cap + (tok % a.ring_cap)) * a.c;
 }
 
-// Append mode: store the new token's rows of every stream in its ring slot
-// (threads tid0, tid0 + nthr, ... of the block; 16-byte pieces when c is a
-// multiple of 8).  Returns the entry the token closes, or -1.
-__device__ __forceinline__ int append_token(const CompressArgs& a, int b, int tid0, int nthr, int* newtok) {
-  const int p = a.app_pos[b];
-  *newtok = p;
+// Append mode: the entry that sequence b's new token (position p) closes,
+// or -1 (no entry closes, a bad position, or an entry past the pool).
+__device__ __forceinline__ int closing_entry(const CompressArgs& a, int p, bool report) {
   if (p < 0) {
-    if (tid0 == 0) raise_err(a.err, DS4A_DEV_BAD_POS);
+    if (report) raise_err(a.err, DS4A_DEV_BAD_POS);
     return -1;
   }
+  if ((p + 1) % a.m != 0) return -1;
+  const int i = (p + 1) / a.m - 1;
+  if (i >= a.n_cap) {
+    if (report) raise_err(a.err, DS4A_DEV_BAD_INDEX);
+    return -1;
+  }
+  return i;
+}
+
+// Append mode: store the new token's rows of every stream (position p >= 0)
+// in its ring slot (threads tid0, tid0 + nthr, ... of the block; 16-byte
+// pieces when c is a multiple of 8).  The pooling of the entry the token
+// closes reads the token's rows from the inputs, not from the ring, so the
+// store may come after it.
+__device__ __forceinline__ void append_token(const CompressArgs& a, int b, int p, int tid0, int nthr) {
   const bool overlap = a.cb != nullptr;
   const int S = overlap ? 4 : 2;
   const uint16_t* srcs[4] = {a.ca, overlap ? a.cb : a.za, a.za, a.zb};
@@ -101,13 +113,6 @@ __device__ __forceinline__ int append_token(const CompressArgs& a, int b, int ti
       a.ring[(((int64_t)b * S + st) * a.ring_cap + slot) * a.c + q] = srcs[st][(int64_t)b * a.c + q];
     }
   }
-  if ((p + 1) % a.m != 0) return -1;
-  const int i = (p + 1) / a.m - 1;
-  if (i >= a.n_cap) {
-    if (tid0 == 0) raise_err(a.err, DS4A_DEV_BAD_INDEX);
-    return -1;
-  }
-  return i;
 }
 
 // Store channels (ch, ch + 1) of entry i of sequence b: as bf16 at dst, or
@@ -169,8 +174,12 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a) {
   int i = a.entry_begin + blockIdx.x, newtok = -1;
   if (a.app_pos != nullptr) {
     pdl_wait();
-    i = append_token(a, b, tid, kCompressThreads, &newtok);
-    if (i < 0) return;
+    newtok = a.app_pos[b];
+    i = closing_entry(a, newtok, tid == 0);
+    if (i < 0) {
+      if (newtok >= 0) append_token(a, b, newtok, tid, kCompressThreads);
+      return;
+    }
   }
   const int n_terms = (overlap && i >= 1) ? 2 * m : m;
 
@@ -215,6 +224,8 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a) {
       }
     }
   }
+  // the token's rows into the ring (their loads overlap the merge below)
+  if (a.app_pos != nullptr) append_token(a, b, newtok, tid, kCompressThreads);
   // merge the G partials of every channel
   float* s_m = csm;                 // [G * c]
   float* s_l = s_m + G * c;         // [G * c]
@@ -328,13 +339,12 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
   int i = a.entry_begin + blockIdx.x / Z, newtok = -1;
   if (a.app_pos != nullptr) {
     pdl_wait();
-    i = zr == 0 ? append_token(a, b, tid, kCompressThreads, &newtok) : -2;
-    if (zr != 0) {
-      const int p = a.app_pos[b];
-      newtok = p;
-      i = (p >= 0 && (p + 1) % m == 0 && (p + 1) / m - 1 < a.n_cap) ? (p + 1) / m - 1 : -1;
+    newtok = a.app_pos[b];
+    i = closing_entry(a, newtok, zr == 0 && tid == 0);
+    if (i < 0) {
+      if (zr == 0 && newtok >= 0) append_token(a, b, newtok, tid, kCompressThreads);
+      return;
     }
-    if (i < 0) return;
   }
   const int n_terms = (overlap && i >= 1) ? 2 * m : m;
   const int tz0 = (int)((int64_t)zr * n_terms / Z), tz1 = (int)((int64_t)(zr + 1) * n_terms / Z);
@@ -376,6 +386,8 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
       }
     }
   }
+  // block 0 stores the token's rows into the ring (after its term loads)
+  if (a.app_pos != nullptr && zr == 0) append_token(a, b, newtok, tid, kCompressThreads);
   // block partials: [G][c] each, then one (M, L, A) per channel
   float* s_m = csm;
   float* s_l = s_m + G * c;

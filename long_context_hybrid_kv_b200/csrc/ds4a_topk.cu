@@ -461,9 +461,9 @@ constexpr int kLocalK = 2048;  // largest k of the local-candidate cluster kerne
 // of the blocks' top k (same tie rule).  Either way the result is exact.
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThreads)
     topk_cluster_kernel(IndexArgs a) {
-  extern __shared__ unsigned int keys[];  // [kClusterSlice]; block 0 reuses it for the gathered lists
-  __shared__ unsigned int hist[2048];     // this block's histogram of maxima (read by the peers)
-  __shared__ unsigned int hsum[2048];     // the cluster's
+  extern __shared__ __align__(16) unsigned int keys[];  // [kClusterSlice]; block 0 reuses it for the gathered lists
+  __shared__ __align__(16) unsigned int hist[2048];  // this block's histogram of maxima (read by the peers)
+  __shared__ __align__(16) unsigned int hsum[2048];  // the cluster's
   __shared__ unsigned int cand_key[kLocalK];
   __shared__ int cand_idx[kLocalK];
   __shared__ int s_warp[33];
@@ -501,14 +501,19 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kClusterThrea
   atomicAdd(&hist[tmax >> 21], 1u);
   auto kslot = [](int i) { return kpos(i); };
   cl.sync();  // every block's histogram of maxima is complete
-  for (int i = tid; i < 2048; i += blockDim.x) {
-    unsigned int c[kCluster];
+  for (int i = tid; i < 512; i += blockDim.x) {  // four bins per 16-byte read
+    uint4 c[kCluster];
 #pragma unroll
-    for (int r = 0; r < kCluster; ++r) c[r] = cl.map_shared_rank(hist, r)[i];
-    unsigned int t = 0;
+    for (int r = 0; r < kCluster; ++r) c[r] = reinterpret_cast<const uint4*>(cl.map_shared_rank(hist, r))[i];
+    uint4 t = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int r = 0; r < kCluster; ++r) t += c[r];
-    hsum[i] = t;
+    for (int r = 0; r < kCluster; ++r) {
+      t.x += c[r].x;
+      t.y += c[r].y;
+      t.z += c[r].z;
+      t.w += c[r].w;
+    }
+    reinterpret_cast<uint4*>(hsum)[i] = t;
   }
   __syncthreads();
   find_digit2048(hsum, k, s_warp, &s_digit, &s_above);

@@ -173,6 +173,33 @@ def test_index_topk_large_rows_cluster_path():
     assert np.array_equal(gidx[0, 0], np.arange(FLASH.topk))
 
 
+def test_index_topk_cluster_crowded_scores():
+    # keys within ~2 % of one row: the scores are distinct but crowd into one
+    # or two histogram bins of the cluster selector, whose floor then leaves
+    # more candidates than a block keeps, so every block selects its own k
+    # best before block 0 merges (the selector's second path)
+    n_c = 40000
+    row = nf("crowd.row", (1, 1, FLASH.idx_dim))
+    noise = nf("crowd.noise", (1, n_c, FLASH.idx_dim))
+    ki = host.f32_to_bf16_bits((row * (1.0 + 0.02 * noise)).astype(np.float32)).reshape(1, n_c, FLASH.idx_dim)
+    qi, wi, ki, qpos, gidx, gsc = _index_case(1, [4 * n_c - 1, 4 * 30000 - 1], n_c, FLASH, "crowd", ki=ki)
+    _check_index(qi, wi, ki, qpos, gidx, gsc, FLASH, n_c)
+
+
+@pytest.mark.parametrize("k", [1500, 2048, 3000])
+def test_index_topk_cluster_large_k(k):
+    # k above the block's 1024 threads (no per-block floor in the second
+    # path), at the local-candidate kernel's limit (2048), and above it (the
+    # multi-pass cluster kernel)
+    import dataclasses
+
+    cfg_py = dataclasses.replace(FLASH, topk=k)
+    n_c = 30000
+    pos = [4 * n_c - 1, 4 * (k + 700) - 1]
+    qi, wi, ki, qpos, gidx, gsc = _index_case(1, pos, n_c, cfg_py, f"bigk{k}")
+    _check_index(qi, wi, ki, qpos, gidx, gsc, cfg_py, n_c)
+
+
 def test_index_topk_beyond_cluster_rows():
     # longer than the cluster selector's 262144: the global-memory selector
     n_c = 262144 + 1000

@@ -487,6 +487,171 @@ __global__ void __launch_bounds__(kCompressThreads) compress_split_kernel(Compre
   }
 }
 
+// Long entries (HCA decode: m' = 128 terms) when there are few of them, c =
+// 512: the 8 blocks of a cluster take 64 channels each over all of the
+// entry's terms, so each block's pooled values are final and only the
+// RMSNorm sum of squares crosses blocks (one distributed-shared-memory read
+// of 8 partial sums).  256 threads, two blocks per SM (so that 32 sequences'
+// entries fit the SMs at once); thread (g, cc): terms g, g + 32, ... of the
+// channel vector cc (8 channels); the 32 partial softmaxes of a channel
+// merge inside the warp (4 term groups) and then over the 8 warps.  Same
+// arithmetic as compress_kernel (log2-unit softmax with a lazy reference),
+// merged in a different order.
+constexpr int kChanZ = 8, kChanC = 512, kChanCz = kChanC / kChanZ, kChanNC = kChanCz / 8, kChanThreads = 256;
+
+// merge the partial (reference, sum, accumulator) (m2, l2, a2) into (m, l, acc)
+__device__ __forceinline__ void merge_partial(float& mx, float& l, float& acc, float m2, float l2, float a2) {
+  if (m2 == -INFINITY) return;
+  if (mx == -INFINITY) {
+    mx = m2;
+    l = l2;
+    acc = a2;
+    return;
+  }
+  const float M = fmaxf(mx, m2);
+  const float e1 = ex2_approx(mx - M), e2 = ex2_approx(m2 - M);
+  l = l * e1 + l2 * e2;
+  acc = acc * e1 + a2 * e2;
+  mx = M;
+}
+
+__global__ void __cluster_dims__(kChanZ, 1, 1) __launch_bounds__(kChanThreads, 2)
+    compress_chan_kernel(const __grid_constant__ CompressArgs a) {
+  constexpr int V = 8, NC = kChanNC, G = kChanThreads / NC;
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  __shared__ float s_m[kChanThreads / 32][kChanCz], s_l[kChanThreads / 32][kChanCz],
+      s_a[kChanThreads / 32][kChanCz];
+  __shared__ float s_v[kChanCz];
+  __shared__ float s_red[kChanThreads / 32];
+  __shared__ float s_tot;
+  const int m = a.m, c = kChanC;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cc = tid % NC, g = tid / NC;
+  const int zr = (int)cl.block_rank();
+  const int ch0 = zr * kChanCz;
+  const int b = blockIdx.y;
+  const bool overlap = a.cb != nullptr;
+  pdl_trigger();
+  // every block of a cluster serves the same entry, so all take the same
+  // early exit; in append mode everything waits (the ring is a library
+  // output), otherwise only the pool write does
+  int i = a.entry_begin + blockIdx.x / kChanZ, newtok = -1;
+  if (a.app_pos != nullptr) {
+    pdl_wait();
+    newtok = a.app_pos[b];
+    i = closing_entry(a, newtok, zr == 0 && tid == 0);
+    if (i < 0) {
+      if (zr == 0 && newtok >= 0) append_token(a, b, newtok, tid, kChanThreads);
+      return;
+    }
+  }
+  const int n_terms = (overlap && i >= 1) ? 2 * m : m;
+  float mx[V], l[V], acc[V];
+#pragma unroll
+  for (int u = 0; u < V; ++u) { mx[u] = -INFINITY; l[u] = 0.f; acc[u] = 0.f; }
+  const int cv = ch0 + cc * V;
+  for (int t0 = g; t0 < n_terms; t0 += 4 * G) {
+    float vals[4][V], zs[4][V], bs[4][V];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int term = t0 + u * G;
+      if (term < n_terms) {
+        const bool half_a = term < m;
+        const int r = half_a ? term : term - m;
+        const int tok = half_a ? i * m + r : (i - 1) * m + r;
+        VecLoad<V>::load(term_row(a, half_a, false, b, tok, newtok) + cv, vals[u]);
+        VecLoad<V>::load(term_row(a, half_a, true, b, tok, newtok) + cv, zs[u]);
+        VecLoad<V>::load_f((half_a ? a.bias_a : a.bias_b) + (int64_t)r * c + cv, bs[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (t0 + u * G >= n_terms) break;
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const float x = (zs[u][q] + bs[u][q]) * kLog2eC;
+        if (x > mx[q] + 8.f) {
+          const float sc = ex2_approx(mx[q] - x);  // 0 while empty
+          l[q] *= sc;
+          acc[q] *= sc;
+          mx[q] = x;
+        }
+        const float e = ex2_approx(x - mx[q]);
+        l[q] += e;
+        acc[q] = fmaf(e, vals[u][q], acc[q]);
+      }
+    }
+  }
+  // block 0 stores the token's rows into the ring (after its term loads)
+  if (a.app_pos != nullptr && zr == 0) append_token(a, b, newtok, tid, kChanThreads);
+  // the warp's 4 term groups of each channel vector (lanes cc, cc + 8, ...)
+#pragma unroll
+  for (int o = NC; o < 32; o <<= 1)
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, mx[q], o);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l[q], o);
+      const float a2 = __shfl_xor_sync(0xffffffffu, acc[q], o);
+      merge_partial(mx[q], l[q], acc[q], m2, l2, a2);
+    }
+  if (lane < NC) {
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      s_m[warp][cc * V + q] = mx[q];
+      s_l[warp][cc * V + q] = l[q];
+      s_a[warp][cc * V + q] = acc[q];
+    }
+  }
+  __syncthreads();
+  float ss = 0.f;
+  if (tid < kChanCz) {
+    float M = -INFINITY, Ls = 0.f, A = 0.f;
+    for (int w = 0; w < kChanThreads / 32; ++w) merge_partial(M, Ls, A, s_m[w][tid], s_l[w][tid], s_a[w][tid]);
+    const float v = A / Ls;
+    s_v[tid] = v;
+    ss = v * v;
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) s_red[warp] = ss;
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kChanThreads / 32; ++w) t += s_red[w];
+    s_tot = t;
+  }
+  cl.sync();  // every block's sum of squares is in place
+  float tot = 0.f;
+#pragma unroll
+  for (int r = 0; r < kChanZ; ++r) tot += *cl.map_shared_rank(&s_tot, r);
+  cl.sync();  // no block leaves while a peer may still read its sum
+  if (a.app_pos == nullptr) pdl_wait();
+  if (warp != 0) return;
+  // warp 0: the block's 64 channels as 32 pairs (a whole 64-channel run, as
+  // the block-scaled store wants)
+  uint16_t* dst = a.qfmt ? nullptr : a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c + ch0;
+  if (a.norm_g == nullptr) {
+    if (a.qfmt) store_entry_pair(a, b, i, ch0 + 2 * lane, s_v[2 * lane], s_v[2 * lane + 1], nullptr);
+    else *reinterpret_cast<unsigned int*>(dst + 2 * lane) = f2_to_bf2x2(s_v[2 * lane], s_v[2 * lane + 1]);
+    return;
+  }
+  const float rstd = rsqrtf(tot / (float)c + a.eps);
+  const int R = a.rope_dim;
+  const int pos = i * m;
+  const int k = 2 * lane, ch = ch0 + k;
+  float x0 = s_v[k] * rstd * a.norm_g[ch];
+  float x1 = s_v[k + 1] * rstd * a.norm_g[ch + 1];
+  if (ch >= c - R) {
+    float cs, sn;
+    rope_cos_sin(pos, a.rope.t[(ch - (c - R)) >> 1], &cs, &sn);
+    const float y0 = x0 * cs - x1 * sn;
+    const float y1 = x0 * sn + x1 * cs;
+    x0 = y0;
+    x1 = y1;
+  }
+  store_entry_pair(a, b, i, ch, x0, x1, a.qfmt ? nullptr : dst + k);
+}
+
 // whether a job runs in the one-block-per-entry kernel with 8-wide loads
 static bool plain8(const CompressArgs& a) {
   const int n_terms = a.cb != nullptr ? 2 * a.m : a.m;
@@ -527,7 +692,13 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
   const int NC = a.c / V;
   const int G = NC >= kCompressThreads ? 1 : kCompressThreads / NC;
   const int n_terms = a.cb != nullptr ? 2 * a.m : a.m;
-  // long entries, few of them: split each entry's terms over a cluster
+  // long entries of 512 channels, few of them (decode): an 8-block cluster
+  // per entry, 64 channels per block
+  if (V == 8 && a.c == kChanC && n_terms >= 64 && (int64_t)n * a.B <= 32) {
+    TraceScope tr("compress", s);
+    return launch_pdl(compress_chan_kernel, dim3(n * kChanZ, a.B), dim3(kChanThreads), 0, s, a);
+  }
+  // other long entries, few of them: split each entry's terms over a cluster
   int Z = 1;
   if (V == 8 && n_terms >= 64)
     while (Z < 8 && (int64_t)n * a.B * Z * 2 <= 148 && n_terms / (2 * Z) >= 16 && a.c % (2 * Z * 2) == 0) Z *= 2;

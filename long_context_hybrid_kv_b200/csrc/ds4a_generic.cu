@@ -154,6 +154,105 @@ __device__ __forceinline__ void store_entry_pair(const CompressArgs& a, int b, i
   }
 }
 
+// Short entries of 512 channels (CSA: m = 4, at most 16 terms), one
+// 256-thread block per entry: thread p pools channels 2p, 2p + 1 over all
+// of the entry's terms with every load in flight at once, so no partial
+// softmaxes are merged; the block adds the RMSNorm sum of squares.  Warp w
+// holds channels 64w .. 64w + 63 (a whole run for the block-scaled store).
+// The softmax takes the exact maximum of the (at most 16) logits first.
+constexpr int kShortC = 512, kShortTerms = 16, kShortThreads = kShortC / 2;
+
+__device__ __forceinline__ void compress_short(const CompressArgs& a) {
+  constexpr int c = kShortC;
+  const int m = a.m, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, b = blockIdx.y;
+  const bool overlap = a.cb != nullptr;
+  __shared__ float s_red_short[kShortThreads / 32];
+  pdl_trigger();
+  int i = a.entry_begin + blockIdx.x, newtok = -1;
+  if (a.app_pos != nullptr) {
+    pdl_wait();
+    newtok = a.app_pos[b];
+    i = closing_entry(a, newtok, tid == 0);
+    if (i < 0) {
+      if (newtok >= 0) append_token(a, b, newtok, tid, kShortThreads);
+      return;
+    }
+  }
+  const int n_terms = (overlap && i >= 1) ? 2 * m : m;
+  const int ch = 2 * tid;
+  float v0 = 0.f, v1 = 0.f, ss = 0.f;
+  {
+    float x0[kShortTerms], x1[kShortTerms], c0[kShortTerms], c1[kShortTerms];
+    float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < kShortTerms; ++t) {
+      x0[t] = x1[t] = -INFINITY;
+      c0[t] = c1[t] = 0.f;
+      if (t < n_terms) {
+        const bool half_a = t < m;
+        const int r = half_a ? t : t - m;
+        const int tok = half_a ? i * m + r : (i - 1) * m + r;
+        const float2 cf = bf2x2_to_f2(*reinterpret_cast<const unsigned int*>(term_row(a, half_a, false, b, tok, newtok) + ch));
+        const float2 zf = bf2x2_to_f2(*reinterpret_cast<const unsigned int*>(term_row(a, half_a, true, b, tok, newtok) + ch));
+        const float2 bb = *reinterpret_cast<const float2*>((half_a ? a.bias_a : a.bias_b) + (int64_t)r * c + ch);
+        x0[t] = (zf.x + bb.x) * kLog2eC;
+        x1[t] = (zf.y + bb.y) * kLog2eC;
+        c0[t] = cf.x;
+        c1[t] = cf.y;
+        M0 = fmaxf(M0, x0[t]);
+        M1 = fmaxf(M1, x1[t]);
+      }
+    }
+    float l0 = 0.f, l1 = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int t = 0; t < kShortTerms; ++t) {
+      if (t < n_terms) {
+        const float e0 = ex2_approx(x0[t] - M0), e1 = ex2_approx(x1[t] - M1);
+        l0 += e0;
+        l1 += e1;
+        a0 = fmaf(e0, c0[t], a0);
+        a1 = fmaf(e1, c1[t], a1);
+      }
+    }
+    v0 = a0 / l0;
+    v1 = a1 / l1;
+    ss = v0 * v0 + v1 * v1;
+  }
+  // the token's rows into the ring (after the entry's term loads)
+  if (a.app_pos != nullptr) append_token(a, b, newtok, tid, kShortThreads);
+  float tot = 0.f;
+  if (a.norm_g != nullptr) {
+    ss = warp_sum(ss);
+    if (lane == 0) s_red_short[warp] = ss;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kShortThreads / 32; ++w) tot += s_red_short[w];
+  }
+  if (a.app_pos == nullptr) pdl_wait();  // a preceding kernel may still read the entry this one overwrites
+  uint16_t* dst = a.qfmt ? nullptr : a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c + ch;
+  if (a.norm_g == nullptr) {
+    store_entry_pair(a, b, i, ch, v0, v1, dst);
+    return;
+  }
+  const float rstd = rsqrtf(tot / (float)c + a.eps);
+  const int R = a.rope_dim;
+  float x0 = v0 * rstd * a.norm_g[ch];
+  float x1 = v1 * rstd * a.norm_g[ch + 1];
+  if (ch >= c - R) {
+    float cs, sn;
+    rope_cos_sin(i * m, a.rope.t[(ch - (c - R)) >> 1], &cs, &sn);
+    const float y0 = x0 * cs - x1 * sn;
+    const float y1 = x0 * sn + x1 * cs;
+    x0 = y0;
+    x1 = y1;
+  }
+  store_entry_pair(a, b, i, ch, x0, x1, dst);
+}
+
+__global__ void __launch_bounds__(kShortThreads) compress_short_kernel(const __grid_constant__ CompressArgs a) {
+  compress_short(a);
+}
+
 template <int V>
 __device__ __forceinline__ void compress_body(const CompressArgs& a) {
   extern __shared__ float csm[];
@@ -308,6 +407,14 @@ struct CompressPair {
 template <int V>
 __global__ void __launch_bounds__(kCompressThreads) compress_pair_kernel(const __grid_constant__ CompressPair p) {
   compress_body<V>(p.j[blockIdx.z]);
+}
+__global__ void __launch_bounds__(kShortThreads) compress_short_pair_kernel(const __grid_constant__ CompressPair p) {
+  compress_short(p.j[blockIdx.z]);
+}
+
+// whether an entry shape runs in the short-entry kernels
+static bool short_entry(const CompressArgs& a) {
+  return a.c == kShortC && (a.cb != nullptr ? 2 * a.m : a.m) <= kShortTerms;
 }
 
 // Long entries (HCA: m' = 128 terms) when there are few of them (decode):
@@ -659,6 +766,14 @@ static bool plain8(const CompressArgs& a) {
 }
 
 cudaError_t launch_compress_jobs(const CompressArgs* jobs, int n_jobs, cudaStream_t s) {
+  if (n_jobs == 2 && jobs[0].app_pos && jobs[1].app_pos && short_entry(jobs[0]) && short_entry(jobs[1]) &&
+      jobs[0].B == jobs[1].B && jobs[0].B > 0) {
+    CompressPair p;
+    p.j[0] = jobs[0];
+    p.j[1] = jobs[1];
+    TraceScope tr("compress", s);
+    return launch_pdl(compress_short_pair_kernel, dim3(1, jobs[0].B, 2), dim3(kShortThreads), 0, s, p);
+  }
   if (n_jobs == 2 && jobs[0].app_pos && jobs[1].app_pos && plain8(jobs[0]) && plain8(jobs[1]) &&
       jobs[0].B == jobs[1].B && jobs[0].B > 0) {
     size_t smem = 0;
@@ -692,6 +807,10 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
   const int NC = a.c / V;
   const int G = NC >= kCompressThreads ? 1 : kCompressThreads / NC;
   const int n_terms = a.cb != nullptr ? 2 * a.m : a.m;
+  if (short_entry(a)) {
+    TraceScope tr("compress", s);
+    return launch_pdl(compress_short_kernel, dim3(n, a.B), dim3(kShortThreads), 0, s, a);
+  }
   // long entries of 512 channels, few of them (decode): an 8-block cluster
   // per entry, 64 channels per block
   if (V == 8 && a.c == kChanC && n_terms >= 64 && (int64_t)n * a.B <= 32) {

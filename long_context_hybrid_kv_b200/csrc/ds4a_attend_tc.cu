@@ -182,7 +182,7 @@ struct DenseKV {
 template <bool kCompact, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap kvmap, DenseKV dkv, AttendArgs a, int n_items,
-                     const __grid_constant__ CUtensorMap qmap) {
+                     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -510,10 +510,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(1, 256);
       float cs = 1.f, sn = 0.f;
       const int R = a.R;
-      // both go straight from registers to global memory: the final output
-      // as 4-byte words (two dims of one head; a warp writes two 64-byte
-      // runs per store), split partials as coalesced 128-byte rows
-      unsigned int* orow = reinterpret_cast<unsigned int*>(a.out + (int64_t)it.row * kH * kD);
+      // The final output goes out one 128-dim chunk at a time through the
+      // P^T buffer (free: the item's PV products are done) as two 64-head x
+      // 64-dim boxes (128-byte swizzle) that one thread stores by TMA, so the
+      // warps do not wait on the global writes; split partials go straight
+      // from registers to global memory as coalesced 128-byte rows.
       const bool odd = r & 1;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -524,10 +525,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(t_lane + 128u + 64u * c + (uint32_t)h0, v);
         tmem_ld_wait();
         if (final_out) {
+          if (c > 0) {
+            if (st == 0) bulk_wait_read0();  // the previous chunk's boxes have been read
+            named_bar(1, 256);
+          }
           // lanes r and r^1 hold dims d and d^1: one exchange per head pair
           // gives the even lane both dims of the even head and the odd lane
           // both dims of the odd head, so each lane rotates its pair (rope
-          // slice, by -pos) and writes one 4-byte word
+          // slice, by -pos) and writes one 4-byte word of the box
+          const uint32_t dd = (uint32_t)(r & 62);  // the pair's first dim within its box
+          const uint32_t box = p_base + (uint32_t)(r >> 6) * 8192u;
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const float got = __shfl_xor_sync(0xffffffffu, odd ? v[i] : v[i + 1], 1);
@@ -536,13 +543,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             float2 x = mul_f2(make_float2(odd ? got : v[i], odd ? v[i + 1] : got), make_float2(s, s));
             if (rot)  // (x0 cs + x1 sn, -x0 sn + x1 cs)
               x = fma_f2(make_float2(x.x, x.x), make_float2(cs, -sn), mul_f2(make_float2(x.y, x.y), make_float2(sn, cs)));
-            orow[h * (kD / 2) + 64 * c + (r >> 1)] = f2_to_bf2x2(x.x, x.y);
+            st_shared32(box + (uint32_t)h * 128u + ((((dd >> 3) ^ (uint32_t)(h & 7))) << 4) + (dd & 7u) * 2u,
+                        f2_to_bf2x2(x.x, x.y));
+          }
+          fence_async_smem();
+          named_bar(1, 256);
+          if (st == 0) {
+            tma_store_2d(&omap, 128 * c, it.row * kH, p_base);
+            tma_store_2d(&omap, 128 * c + 64, it.row * kH, p_base + 8192u);
+            bulk_commit();
           }
         } else {
           float* part = a.ws + ((int64_t)it.row * a.n_splits + it.split) * (2 * kH + kH * kD);
 #pragma unroll
           for (int i = 0; i < 32; ++i) part[2 * kH + (h0 + i) * kD + d] = v[i];
         }
+      }
+      if (final_out) {
+        // the boxes have been read before the next item's P^T goes in
+        if (st == 0) bulk_wait_read0();
+        named_bar(1, 256);
       }
       tc_fence_before();
       mbar_arrive(bar(kEpiDone));
@@ -892,6 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (pt == 0 && q_loads > 0) mbar_drain(bar(kQRaw), (q_loads - 1) & 1u);
   }
 
+  if (tid == 0) bulk_wait0();  // the output stores have completed
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -942,6 +963,19 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  // the output as rows of 512 (one per head), for the final output's TMA
+  // stores (64 heads x 64 dims boxes)
+  CUtensorMap omap;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows * kH};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kH};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   // HCA keys are consecutive pool entries: a row view of the pool for TMA
   // tile loads (when the sequences are a whole number of rows apart)
   CUtensorMap kvmap;
@@ -966,14 +1000,14 @@ cudaError_t launch_attend_tc(const AttendArgs& a0, cudaStream_t s) {
     TraceScope tr("attend_tc", s);
     if (fp8)
       e = compact ? launch_pdl(attend_tc_kernel<true, true>, dim3(grid), dim3(kThreads), kSmemBytes8, s, kvmap, dkv,
-                               a, n_items, qmap)
+                               a, n_items, qmap, omap)
                   : launch_pdl(attend_tc_kernel<false, true>, dim3(grid), dim3(kThreads), kSmemBytes8, s, kvmap, dkv,
-                               a, n_items, qmap);
+                               a, n_items, qmap, omap);
     else
       e = compact ? launch_pdl(attend_tc_kernel<true, false>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap, dkv,
-                               a, n_items, qmap)
+                               a, n_items, qmap, omap)
                   : launch_pdl(attend_tc_kernel<false, false>, dim3(grid), dim3(kThreads), kSmemBytes, s, kvmap,
-                               dkv, a, n_items, qmap);
+                               dkv, a, n_items, qmap, omap);
   }
   if (e != cudaSuccess || a.n_splits == 1) return e;
   return launch_attend_combine(a, s);

@@ -230,6 +230,9 @@ __device__ __forceinline__ void cp_async_wait() {
 __device__ __forceinline__ void st_shared_zero16(uint32_t dst) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
 }
+__device__ __forceinline__ void st_shared32(uint32_t dst, uint32_t a) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(dst), "r"(a) : "memory");
+}
 __device__ __forceinline__ void st_shared16(uint32_t dst, uint32_t a, uint32_t b, uint32_t c,
                                             uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -294,6 +297,20 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(pol)
       : "memory");
 }
+
+// TMA store of a box from this block's shared memory (tiled mode; x * element
+// size a multiple of 16, coordinates non-negative), in the thread's bulk
+// group; commit, then wait until the group has read its shared memory
+// (.read) or has completed
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // hint: bring `bytes` (a multiple of 16, 16-byte aligned) at p into L2
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {

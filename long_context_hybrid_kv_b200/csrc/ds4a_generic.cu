@@ -154,16 +154,18 @@ __device__ __forceinline__ void store_entry_pair(const CompressArgs& a, int b, i
   }
 }
 
-// Short entries of 512 channels (CSA: m = 4, at most 16 terms), one
-// 256-thread block per entry: thread p pools channels 2p, 2p + 1 over all
-// of the entry's terms with every load in flight at once, so no partial
-// softmaxes are merged; the block adds the RMSNorm sum of squares.  Warp w
-// holds channels 64w .. 64w + 63 (a whole run for the block-scaled store).
-// The softmax takes the exact maximum of the (at most 16) logits first.
+// Short entries (CSA: m = 4, at most 16 terms) of up to 512 channels, a
+// multiple of 64 (the K=V entries' 512, the indexer keys' 128), one
+// 256-thread block per entry: thread p < c / 2 pools channels 2p, 2p + 1
+// over all of the entry's terms with every load in flight at once, so no
+// partial softmaxes are merged; the block adds the RMSNorm sum of squares.
+// Warp w holds channels 64w .. 64w + 63 (a whole run for the block-scaled
+// store).  The softmax takes the exact maximum of the (at most 16) logits
+// first.
 constexpr int kShortC = 512, kShortTerms = 16, kShortThreads = kShortC / 2;
 
 __device__ __forceinline__ void compress_short(const CompressArgs& a) {
-  constexpr int c = kShortC;
+  const int c = a.c;
   const int m = a.m, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, b = blockIdx.y;
   const bool overlap = a.cb != nullptr;
   __shared__ float s_red_short[kShortThreads / 32];
@@ -181,7 +183,7 @@ __device__ __forceinline__ void compress_short(const CompressArgs& a) {
   const int n_terms = (overlap && i >= 1) ? 2 * m : m;
   const int ch = 2 * tid;
   float v0 = 0.f, v1 = 0.f, ss = 0.f;
-  {
+  if (ch < c) {
     float x0[kShortTerms], x1[kShortTerms], c0[kShortTerms], c1[kShortTerms];
     float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
@@ -229,6 +231,7 @@ __device__ __forceinline__ void compress_short(const CompressArgs& a) {
     for (int w = 0; w < kShortThreads / 32; ++w) tot += s_red_short[w];
   }
   if (a.app_pos == nullptr) pdl_wait();  // a preceding kernel may still read the entry this one overwrites
+  if (ch >= c) return;
   uint16_t* dst = a.qfmt ? nullptr : a.pool + (int64_t)b * a.pool_bstride + (int64_t)i * c + ch;
   if (a.norm_g == nullptr) {
     store_entry_pair(a, b, i, ch, v0, v1, dst);
@@ -408,13 +411,12 @@ template <int V>
 __global__ void __launch_bounds__(kCompressThreads) compress_pair_kernel(const __grid_constant__ CompressPair p) {
   compress_body<V>(p.j[blockIdx.z]);
 }
-__global__ void __launch_bounds__(kShortThreads) compress_short_pair_kernel(const __grid_constant__ CompressPair p) {
-  compress_short(p.j[blockIdx.z]);
-}
-
-// whether an entry shape runs in the short-entry kernels
+// whether an entry shape runs in the short-entry kernel: bulk compression
+// (a prefill); one entry per sequence (decode) measured faster in the
+// 512-thread kernels, whose wider loads put fewer load instructions behind
+// the wait for the ring
 static bool short_entry(const CompressArgs& a) {
-  return a.c == kShortC && (a.cb != nullptr ? 2 * a.m : a.m) <= kShortTerms;
+  return a.app_pos == nullptr && a.c <= kShortC && a.c % 64 == 0 && (a.cb != nullptr ? 2 * a.m : a.m) <= kShortTerms;
 }
 
 // Long entries (HCA: m' = 128 terms) when there are few of them (decode):
@@ -766,14 +768,6 @@ static bool plain8(const CompressArgs& a) {
 }
 
 cudaError_t launch_compress_jobs(const CompressArgs* jobs, int n_jobs, cudaStream_t s) {
-  if (n_jobs == 2 && jobs[0].app_pos && jobs[1].app_pos && short_entry(jobs[0]) && short_entry(jobs[1]) &&
-      jobs[0].B == jobs[1].B && jobs[0].B > 0) {
-    CompressPair p;
-    p.j[0] = jobs[0];
-    p.j[1] = jobs[1];
-    TraceScope tr("compress", s);
-    return launch_pdl(compress_short_pair_kernel, dim3(1, jobs[0].B, 2), dim3(kShortThreads), 0, s, p);
-  }
   if (n_jobs == 2 && jobs[0].app_pos && jobs[1].app_pos && plain8(jobs[0]) && plain8(jobs[1]) &&
       jobs[0].B == jobs[1].B && jobs[0].B > 0) {
     size_t smem = 0;

@@ -74,6 +74,10 @@ COMPRESS_CASES = {
     "csa_ix_prefill": (128, 4, True, False, 0, 2, 0, 516, (0, 129)),
     "hca_kv": (512, 128, False, True, 64, 2, 0, 640, (0, 5)),
     "hca_kv_decode": (512, 128, False, True, 64, 3, 130944, 128, (1023, 1024)),
+    # many long entries: one block per entry, not the channel-split cluster
+    "hca_kv_many": (512, 128, False, True, 64, 2, 0, 5120, (0, 40)),
+    # long entries of another width: the term-split cluster kernel
+    "hca_256_split": (256, 128, False, True, 32, 2, 0, 640, (0, 5)),
     "toy_kv": (8, 2, True, True, 2, 1, 0, 64, (0, 32)),
     "toy_ix": (4, 2, True, False, 0, 1, 0, 64, (0, 32)),
     "mid_entries": (256, 4, True, True, 32, 1, 40, 60, (11, 25)),
